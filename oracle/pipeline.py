@@ -1,0 +1,83 @@
+"""Oracle compositions of the whole CSA / HCA forward pass (test
+infrastructure only; see the package docstring).
+
+The steps are taken in the order of the DeepSeek-V4 reading notes
+("DeepSeekV4技术报告阅读笔记", 2.3-2.5): compress (eq. 9-12 or 20-23), RMSNorm +
+partial RoPE of the entries and of the window rows, indexer scores (eq. 16),
+top-k (eq. 17), shared-KV MQA with window and sink (eq. 19 / 26 / 27) and
+the R_{-t} de-rotation of the output.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (attend, compress, fp8mix_decode, fp8mix_encode, index_scores,
+               matmul, norm_rope_rows, nvis, round_bf16, topk, _f64)
+
+
+def store(x: np.ndarray, fmt: str, rope_dims: int) -> np.ndarray:
+    """Round fp64 values to a storage format and return the stored values:
+    'f32' (nearest fp32), 'bf16' (nearest bf16), 'fp8mix' (E4M3 with a
+    per-row scale on the non-RoPE dims, bf16 on the RoPE dims)."""
+    if fmt == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if fmt == "bf16":
+        return round_bf16(x)
+    codes, rope, scale = fp8mix_encode(x, rope_dims)
+    c = x.shape[-1]
+    # rope holds bf16-exact values: the fp32 -> bf16 cast below is exact
+    bits = torch.from_numpy(rope.astype(np.float32)).to(torch.bfloat16).view(torch.int16)
+    bits = bits.numpy().view(np.uint16)
+    return fp8mix_decode(codes, bits, scale, c, rope_dims)
+
+
+def cache_values(rec, scale, fmt: str, c: int, rope_dims: int) -> np.ndarray:
+    """fp64 values of a cache held in the library's layout: f32 / bf16 rows
+    [.., rows, c], or fp8mix records [.., rows, (c-rope) + 2*rope bytes] with
+    an fp32 scale per row."""
+    if fmt in ("f32", "bf16"):
+        return _f64(rec)
+    rec = rec.detach().cpu()
+    lead = rec.shape[:-1]
+    nf = c - rope_dims
+    r2 = rec.reshape(-1, rec.shape[-1])
+    codes = r2[:, :nf].contiguous().numpy()
+    bits = r2[:, nf:].contiguous().view(torch.int16).numpy().view(np.uint16)
+    sc = scale.detach().cpu().reshape(-1).numpy().astype(np.float32)
+    return fp8mix_decode(codes, bits, sc, c, rope_dims).reshape(*lead, c)
+
+
+def compress_seq(wl, W: dict, H):
+    """(kv [N][c], kI [N][c_I] or None, win [T][c]) of one sequence, each
+    rounded to its storage format."""
+    H = _f64(H)
+    if wl.variant == "csa":
+        raw = compress(H, wl.m, W["Wkv_a"], W["Wz_a"], W["B_a"],
+                       W["Wkv_b"], W["Wz_b"], W["B_b"])
+        kI = compress(H, wl.m, W["WIkv_a"], W["WIz_a"], W["BI_a"],
+                      W["WIkv_b"], W["WIz_b"], W["BI_b"])
+        kI = store(kI, wl.act, 0)
+    else:
+        raw = compress(H, wl.m, W["Wkv_a"], W["Wz_a"], W["B_a"])
+        kI = None
+    kv = norm_rope_rows(raw, wl.rope_dims, wl.rope_base, wl.rms_eps, 0.0, float(wl.m))
+    kv = store(kv, wl.kv, wl.rope_dims)
+    Ca = matmul(H, W["Wkv_a"])
+    win = norm_rope_rows(Ca, wl.rope_dims, wl.rope_base, wl.rms_eps, 0.0, 1.0)
+    win = store(win, wl.kv, wl.rope_dims)
+    return kv, kI, win
+
+
+def select(wl, t0s, qI, w, kI):
+    """(idx [Q][k], scores [Q][N], nvis [Q], kth [Q]) of eq. 16-17."""
+    N = kI.shape[0]
+    scores = index_scores(t0s, wl.m, qI, w, kI)
+    nv = np.array([nvis(t, wl.m, N) for t in t0s], dtype=np.int32)
+    idx, kth = topk(scores, nv, wl.topk)
+    return idx, scores, nv, kth
+
+
+def attend_wl(wl, t0s, q, idx, kv, win, win_pos0, sink, rope_shift=0.0):
+    return attend(t0s, q, idx, wl.m, kv, wl.n_win, win, win_pos0, sink,
+                  wl.rope_dims, wl.rope_base, wl.softmax_scale, rope_shift)

@@ -1,0 +1,470 @@
+"""Pins of the CPU oracle against facts other than its own code: the OCP E4M3
+and bf16 definitions as implemented by torch's casts, closed forms, invariants
+the DeepSeek-V4 pages state, special cases that reduce to library routines
+(numpy matmul / complex arithmetic / sort, torch SDPA) and brute force on tiny
+inputs.  Each test names the passage it follows."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import pipeline as P
+from long_context_sparse_09_b200.configs import WORKLOADS
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- formats ---
+
+def test_e4m3_decode_all_codes_match_torch():
+    """OCP E4M3 (PaperTrace 2.5: the non-RoPE dims are FP8): every code."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).double().numpy()
+    for c in range(256):
+        v = oracle.e4m3_decode(c)
+        if math.isnan(ref[c]):
+            assert math.isnan(v), c
+        else:
+            assert v == ref[c], (c, v, ref[c])
+
+
+def test_e4m3_encode_matches_torch_cast_in_range():
+    r = rng(1)
+    reps = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(
+        torch.float8_e4m3fn).float().numpy()
+    reps = np.unique(reps[np.isfinite(reps)])
+    mids = (reps[1:] + reps[:-1]) / 2  # exact ties in fp32
+    xs = np.concatenate([reps, mids, r.normal(0, 40, 4000), r.normal(0, 0.01, 2000),
+                         r.uniform(-448, 448, 2000)]).astype(np.float32)
+    xs = xs[np.abs(xs) <= 448]
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(x)) for x in xs], dtype=np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    # -0.0 / +0.0 may differ only in the sign bit of a zero
+    bad = [i for i in bad if not (xs[i] == 0 or (got[i] & 0x7F) == 0 == (ref[i] & 0x7F))]
+    assert not bad, [(float(xs[i]), got[i], ref[i]) for i in bad[:5]]
+
+
+def test_e4m3_encode_saturates():
+    assert oracle.e4m3_encode(1e6) == 0x7E and oracle.e4m3_decode(0x7E) == 448.0
+    assert oracle.e4m3_encode(-470.0) == 0xFE
+
+
+def test_bf16_round_matches_torch():
+    r = rng(2)
+    x = np.concatenate([r.normal(0, 1, 5000), r.normal(0, 1e-30, 100),
+                        r.normal(0, 1e30, 100)]).astype(np.float32)
+    # exact ties: a bf16 value plus half its ulp
+    base = torch.from_numpy(r.normal(0, 1, 500).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    ulp = np.array([np.spacing(np.float32(abs(b))) * 2 ** 16 for b in base], dtype=np.float32)
+    ties = (base + np.sign(base) * ulp / 2).astype(np.float32)
+    x = np.concatenate([x, ties]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    got = oracle.round_bf16(x.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_fp8mix_roundtrip_error_bound():
+    """Quantise -> dequantise error <= half an E4M3 ulp times the scale; the
+    largest magnitude maps to 448 exactly; RoPE dims are bf16."""
+    r = rng(3)
+    x = r.normal(0, 1, (64, 128))
+    x[5, :96] = 0.0  # all-zero FP8 part: scale 1
+    codes, rope, scale = oracle.fp8mix_encode(x, 32)
+    bits = torch.from_numpy(rope.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    y = oracle.fp8mix_decode(codes, bits, scale, 128, 32)
+    assert scale[5] == 1.0
+    for i in range(64):
+        xs = (x[i, :96].astype(np.float32) / scale[i]).astype(np.float64)
+        if i != 5:
+            assert np.max(np.abs([oracle.e4m3_decode(c) for c in codes[i]])) == 448.0
+        q = y[i, :96] / scale[i]
+        # E4M3 spacing at |v|: 2^(floor(log2|v|)-3), 2^-9 below 2^-6
+        e = np.floor(np.log2(np.maximum(np.abs(xs), 2.0 ** -6)))
+        half_ulp = 2.0 ** (e - 3) / 2
+        assert np.all(np.abs(q - xs) <= half_ulp * (1 + 1e-6)), i
+    np.testing.assert_array_equal(y[:, 96:], oracle.round_bf16(x[:, 96:]))
+
+
+# ------------------------------------------------------------- RoPE / norm --
+
+def test_rope_is_complex_rotation():
+    """Notes 2.5.2: R_n rotates 2-D sub-spaces; pair p as a complex number
+    times exp(i * pos * base^(-2p/r))."""
+    r = rng(4)
+    x = r.normal(0, 1, 64)
+    for pos in (0.0, 1.0, 17.0, 1048576.0, -3.0):
+        y = oracle.rope(x, 64, 10000.0, pos)
+        z = x[0::2] + 1j * x[1::2]
+        th = 10000.0 ** (-2.0 * np.arange(32) / 64)
+        w = z * np.exp(1j * pos * th)
+        np.testing.assert_allclose(y[0::2], w.real, atol=1e-12)
+        np.testing.assert_allclose(y[1::2], w.imag, atol=1e-12)
+
+
+def test_rope_group_properties():
+    """Notes 2.5.2: R_n^T = R_{-n}, R_m R_n = R_{m+n}; only the last dims move."""
+    r = rng(5)
+    x = r.normal(0, 1, 96)
+    y = oracle.rope(oracle.rope(x, 32, 10000.0, 37.0), 32, 10000.0, 100.0)
+    np.testing.assert_allclose(y, oracle.rope(x, 32, 10000.0, 137.0), atol=1e-12)
+    np.testing.assert_allclose(oracle.rope(oracle.rope(x, 32, 1e4, 5.0), 32, 1e4, -5.0), x, atol=1e-13)
+    np.testing.assert_array_equal(oracle.rope(x, 32, 1e4, 9.0)[:64], x[:64])
+
+
+def test_rmsnorm_invariant():
+    """Notes 2.5.1: RMSNorm(x) = x / RMS(x) (gain 1): a positive multiple of x
+    whose mean square is ms / (ms + eps)."""
+    r = rng(6)
+    x = r.normal(0, 3, 200)
+    for eps in (0.0, 1e-6, 0.5):
+        y = oracle.rmsnorm(x, eps)
+        ms = np.mean(x ** 2)
+        assert np.mean(y ** 2) == pytest.approx(ms / (ms + eps), rel=1e-12)
+        ratio = y / x
+        assert np.all(ratio > 0) and np.ptp(ratio) < 1e-12
+
+
+# ------------------------------------------------------------- compression --
+
+def _comp_case(T=24, d=16, width=8, m=4, seed=7, zero_z=False):
+    r = rng(seed)
+    H = r.normal(0, 1, (T, d))
+    W = {k: r.normal(0, d ** -0.5, (d, width)) for k in ("Wkv_a", "Wkv_b", "Wz_a", "Wz_b")}
+    B = {k: r.normal(0, 0.3, (m, width)) for k in ("B_a", "B_b")}
+    if zero_z:
+        W["Wz_a"][:] = 0
+        W["Wz_b"][:] = 0
+        B["B_a"][:] = 0
+        B["B_b"][:] = 0
+    return H, W, B
+
+
+def test_compress_weights_sum_to_one():
+    """Notes eq. 11: each column of the 2m x c weight block sums to 1; for
+    i = 0 the b rows drop out (weight 0).  HCA (eq. 22): m slots only."""
+    H, W, B = _comp_case()
+    out, S = oracle.compress(H, 4, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"],
+                             W["Wz_b"], B["B_b"], want_S=True)
+    np.testing.assert_allclose(S.sum(axis=1), 1.0, atol=1e-12)
+    assert np.all(S[0, 4:] == 0) and np.all(S[1:, 4:] > 0)
+    out, S = oracle.compress(H, 4, W["Wkv_a"], W["Wz_a"], B["B_a"], want_S=True)
+    np.testing.assert_allclose(S.sum(axis=1), 1.0, atol=1e-12)
+    assert np.all(S[:, 4:] == 0)
+
+
+def test_compress_uniform_weights_give_block_means():
+    """Eq. 11-12 with Z = 0 and B = 0: the softmax is uniform, so entry i is
+    the mean of the m a-rows and m b-rows (only the a-rows for i = 0)."""
+    m = 4
+    H, W, B = _comp_case(zero_z=True)
+    out = oracle.compress(H, m, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"],
+                          W["Wz_b"], B["B_b"])
+    Ca, Cb = H @ W["Wkv_a"], H @ W["Wkv_b"]
+    for i in range(H.shape[0] // m):
+        a = Ca[m * i: m * i + m]
+        if i == 0:
+            ref = a.mean(axis=0)
+        else:
+            ref = np.concatenate([a, Cb[m * i - m: m * i]]).mean(axis=0)
+        np.testing.assert_allclose(out[i], ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("branch,slot", [("a", 0), ("a", 3), ("b", 1), ("b", 2)])
+def test_compress_dominant_slot_selects_token(branch, slot):
+    """Eq. 11-12 / PaperTrace 2.1: entry i takes tokens 4i..4i+3 as C^a and
+    4i-4..4i-1 as C^b.  A huge bias on one slot makes the entry equal to that
+    token's row (pins the token-to-slot map and the b-branch shift)."""
+    m = 4
+    H, W, B = _comp_case(m=m)
+    B["B_a"][:] = 0
+    B["B_b"][:] = 0
+    B[f"B_{branch}"][slot, :] = 200.0
+    out = oracle.compress(H, m, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"],
+                          W["Wz_b"], B["B_b"])
+    Ca, Cb = H @ W["Wkv_a"], H @ W["Wkv_b"]
+    for i in range(1, H.shape[0] // m):
+        ref = Ca[m * i + slot] if branch == "a" else Cb[m * (i - 1) + slot]
+        np.testing.assert_allclose(out[i], ref, atol=1e-9)
+
+
+def test_compress_each_token_in_two_entries():
+    """PaperTrace 2.1: every token enters exactly two CSA entries (its own
+    block as C^a, the next as C^b); HCA blocks do not overlap."""
+    m = 4
+    H, W, B = _comp_case(T=32, m=m)
+    base = oracle.compress(H, m, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"], W["Wz_b"], B["B_b"])
+    base_h = oracle.compress(H, m, W["Wkv_a"], W["Wz_a"], B["B_a"])
+    for j in (0, 5, 11, 27):
+        H2 = H.copy()
+        H2[j] += 1.0
+        out = oracle.compress(H2, m, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"], W["Wz_b"], B["B_b"])
+        changed = set(np.nonzero(np.any(out != base, axis=1))[0])
+        want = {j // m, j // m + 1} & set(range(len(base)))
+        assert changed == want, (j, changed)
+        out_h = oracle.compress(H2, m, W["Wkv_a"], W["Wz_a"], B["B_a"])
+        assert set(np.nonzero(np.any(out_h != base_h, axis=1))[0]) == {j // m}
+
+
+def test_hca_group_of_one_is_identity():
+    """Eq. 22-23 with m' = 1: softmax over one slot is 1, so C^Comp = C = H W."""
+    H, W, B = _comp_case()
+    out = oracle.compress(H, 1, W["Wkv_a"], W["Wz_a"], B["B_a"][:1])
+    np.testing.assert_allclose(out, H @ W["Wkv_a"], atol=1e-12)
+
+
+def test_compress_entry_range_matches_full():
+    H, W, B = _comp_case(T=40)
+    full = oracle.compress(H, 4, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"], W["Wz_b"], B["B_b"])
+    part = oracle.compress(H, 4, W["Wkv_a"], W["Wz_a"], B["B_a"], W["Wkv_b"], W["Wz_b"], B["B_b"], i0=3, i1=7)
+    np.testing.assert_array_equal(part, full[3:7])
+
+
+# ------------------------------------------------------------------ index --
+
+def test_nvis_is_complete_blocks():
+    """Notes 2.3.2 / PaperTrace 2.4: only complete blocks are visible.  Brute
+    force: entry s is visible iff every token of its a-window is <= t0."""
+    for m in (1, 4, 128):
+        for t0 in range(0, 3 * m + 2):
+            brute = sum(1 for s in range(10) if all(tok <= t0 for tok in range(m * s, m * s + m)))
+            assert oracle.nvis(t0, m, 10) == min(brute, 10)
+
+
+def test_index_scores_closed_forms():
+    """Eq. 16: since ReLU(x) - ReLU(-x) = x and ReLU(x) + ReLU(-x) = |x|,
+    I(q) - I(-q) = (sum_h w_h q_h) . K_s and I(q) + I(-q) = sum_h w_h |q_h.K_s|;
+    with one head and w = 1, I = ReLU(q . K_s)."""
+    r = rng(8)
+    Q, nh, cI, N, m = 3, 5, 16, 40, 4
+    qI = r.normal(0, 1, (Q, nh, cI))
+    w = r.normal(0, 1, (Q, nh))
+    K = r.normal(0, 1, (N, cI))
+    t0 = [1000, 1000, 1000]
+    Ip = oracle.index_scores(t0, m, qI, w, K)
+    Im = oracle.index_scores(t0, m, -qI, w, K)
+    lin = np.einsum("qh,qhe->qe", w, qI) @ K.T
+    np.testing.assert_allclose(Ip - Im, lin, atol=1e-11)
+    absd = np.einsum("qh,qhs->qs", w, np.abs(np.einsum("qhe,se->qhs", qI, K)))
+    np.testing.assert_allclose(Ip + Im, absd, atol=1e-11)
+    one = oracle.index_scores(t0, m, qI[:, :1], np.ones((Q, 1)), K)
+    np.testing.assert_allclose(one, np.maximum(qI[:, 0] @ K.T, 0), atol=1e-12)
+
+
+def test_index_scores_mask_invisible():
+    r = rng(9)
+    qI, w, K = r.normal(0, 1, (3, 2, 8)), r.normal(0, 1, (3, 2)), r.normal(0, 1, (10, 8))
+    sc = oracle.index_scores([2, 3, 13], 4, qI, w, K)
+    assert np.all(np.isneginf(sc[0])) and np.isfinite(sc[1, 0]) and np.all(np.isneginf(sc[1, 1:]))
+    assert np.all(np.isfinite(sc[2, :3])) and np.all(np.isneginf(sc[2, 3:]))
+
+
+# ------------------------------------------------------------------ top-k --
+
+def test_topk_matches_full_sort():
+    """Eq. 17 by brute force: a stable sort by (-score, index)."""
+    r = rng(10)
+    Q, N, k = 6, 300, 17
+    sc = np.round(r.normal(0, 1, (Q, N)), 1)  # many exact ties
+    nv = np.array([300, 250, 17, 5, 0, 100], dtype=np.int32)
+    idx, kth = oracle.topk(sc, nv, k)
+    for q in range(Q):
+        order = np.lexsort((np.arange(nv[q]), -sc[q, : nv[q]]))[:k]
+        want = np.sort(order)
+        got = idx[q][idx[q] >= 0]
+        np.testing.assert_array_equal(got, want)
+        assert np.all(idx[q][len(want):] == -1)
+        if len(want):
+            assert kth[q] == sc[q, order[-1]]
+
+
+def test_topk_zero_weights_take_lowest_indices():
+    """All scores equal (w = 0): the tie rule keeps indices 0..k-1."""
+    sc = oracle.index_scores([10 ** 6], 4, np.ones((1, 2, 4)), np.zeros((1, 2)), np.ones((50, 4)))
+    idx, _ = oracle.topk(sc, np.array([50], np.int32), 8)
+    np.testing.assert_array_equal(idx[0], np.arange(8))
+
+
+# -------------------------------------------------------------- attention --
+
+def _sdpa_with_sink(q, keys, sink, scale):
+    """torch SDPA (fp64, CPU) over [keys, sink column]: the sink is a key with
+    logit z'_h (added through the mask) and a zero value."""
+    Qn, nh, c = q.shape
+    outs = []
+    for i in range(Qn):
+        K = torch.from_numpy(keys[i])  # [n, c]
+        n = K.shape[0]
+        Kx = torch.cat([K, torch.zeros(1, c, dtype=torch.float64)])
+        Vx = Kx.clone()
+        qq = torch.from_numpy(q[i]).unsqueeze(1)  # [nh, 1, c]
+        mask = torch.zeros(nh, 1, n + 1, dtype=torch.float64)
+        mask[:, 0, n] = torch.from_numpy(sink)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            qq, Kx.expand(nh, n + 1, c), Vx.expand(nh, n + 1, c), attn_mask=mask, scale=scale)
+        outs.append(o[:, 0].numpy())
+    return np.stack(outs)
+
+
+def test_attend_matches_sdpa_with_sink_column():
+    """Eq. 19 + eq. 27 with no RoPE dims: shared-KV MQA over selected entries
+    and window rows, the sink adding exp(z'_h) to the denominator -- the same
+    as textbook attention with one extra zero-valued key of logit z'_h."""
+    r = rng(11)
+    Q, nh, c, N, m, nwin = 4, 3, 16, 20, 4, 5
+    q = r.normal(0, 1, (Q, nh, c))
+    kv = r.normal(0, 1, (N, c))
+    win = r.normal(0, 1, (40, c))
+    sink = r.normal(0, 1, nh)
+    t0 = np.array([3, 20, 39, 70], np.int32)
+    win_pos0 = 0
+    win_full = r.normal(0, 1, (80, c))
+    idx = np.array([[-1, -1, -1], [0, 2, 4], [1, 5, 9], [3, 7, 16]], np.int32)
+    scale = 0.37
+    out, mass = oracle.attend(t0, q, idx, m, kv, nwin, win_full, win_pos0, sink, 0, 1e4, scale)
+    keys = []
+    for i in range(Q):
+        sel = [kv[s] for s in idx[i] if s >= 0]
+        lo = max(0, t0[i] - nwin + 1)
+        keys.append(np.array(sel + [win_full[t] for t in range(lo, t0[i] + 1)]))
+    ref = _sdpa_with_sink(q, keys, sink, scale)
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+    np.testing.assert_allclose(mass, 1.0, atol=1e-12)
+    # HCA: all visible entries (floor((t0+1)/m)) and the window
+    out_d, _ = oracle.attend(t0, q, None, m, kv, nwin, win_full, win_pos0, sink, 0, 1e4, scale)
+    keys = []
+    for i in range(Q):
+        nv = min(N, (t0[i] + 1) // m)
+        lo = max(0, t0[i] - nwin + 1)
+        keys.append(np.array([kv[s] for s in range(nv)] + [win_full[t] for t in range(lo, t0[i] + 1)]))
+    np.testing.assert_allclose(out_d, _sdpa_with_sink(q, keys, sink, scale), atol=1e-12)
+
+
+def test_attend_sink_limits():
+    """Eq. 27: z' -> -inf gives plain softmax attention; z' -> +inf drives
+    every weight, hence the output, to 0 (PaperTrace 2.4)."""
+    r = rng(12)
+    q, kv, win = r.normal(0, 1, (2, 2, 8)), r.normal(0, 1, (6, 8)), r.normal(0, 1, (30, 8))
+    t0 = np.array([23, 25], np.int32)
+    out_hi, _ = oracle.attend(t0, q, None, 4, kv, 3, win, 0, np.array([60.0, 60.0]), 0, 1e4, 0.3)
+    assert np.max(np.abs(out_hi)) < 1e-20
+    out_lo, _ = oracle.attend(t0, q, None, 4, kv, 3, win, 0, np.array([-1e300, -1e300]), 0, 1e4, 0.3)
+    keys = [np.concatenate([kv, win[21:24]]), np.concatenate([kv, win[23:26]])]
+    ref = []
+    for i in range(2):
+        z = 0.3 * q[i] @ keys[i].T
+        p = np.exp(z - z.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        ref.append(p @ keys[i])
+    np.testing.assert_allclose(out_lo, np.stack(ref), atol=1e-12)
+
+
+def test_attend_derotation_undoes_the_key_rotation():
+    """Notes 2.5.2: o~_t = R_{-t} o_t.  A single key -- the window row of token
+    t0 itself, stored as R_{t0} u -- gets weight 1, so the output is u."""
+    r = rng(13)
+    c, rd = 32, 16
+    u = r.normal(0, 1, c)
+    t0 = 1000
+    row = oracle.rope(u, rd, 1e4, float(t0))
+    win = np.zeros((5, c))
+    win[4] = row
+    q = r.normal(0, 1, (1, 2, c))
+    out, _ = oracle.attend(np.array([t0], np.int32), q, None, 4, np.zeros((0, c)), 1, win,
+                           t0 - 4, np.array([-1e300] * 2), rd, 1e4, 0.1)
+    np.testing.assert_allclose(out[0, 0], u, atol=1e-10)
+    np.testing.assert_allclose(out[0, 1], u, atol=1e-10)
+
+
+def test_attend_rejects_invisible_selection():
+    r = rng(14)
+    with pytest.raises(ValueError):
+        oracle.attend(np.array([7], np.int32), r.normal(0, 1, (1, 1, 8)),
+                      np.array([[2]], np.int32), 4, r.normal(0, 1, (9, 8)), 0, None, 0,
+                      np.zeros(1), 0, 1e4, 0.3)
+
+
+# ------------------------------------------------------ end-to-end (oracle) --
+
+TINY = WORKLOADS["tiny_csa_prefill_f32"].with_(T=64, d=48, c=32, rope_dims=8, n_h=3,
+                                                n_hI=2, c_I=8, topk=4, n_win=6)
+
+
+def _tiny_inputs(wl, seed=0):
+    from long_context_sparse_09_b200 import synth
+    wl = wl.with_(seed=seed)
+    return wl, synth.weights(wl), synth.prefill_inputs(wl)
+
+
+def _e2e(wl, W, inp, q_override=None, rope_shift=0.0, H_override=None):
+    H = inp["H"][0] if H_override is None else H_override
+    kv, kI, win = P.compress_seq(wl, W, H)
+    t0s = inp["q_pos"].numpy()
+    q = inp["q"] if q_override is None else q_override
+    if wl.variant == "csa":
+        idx, *_ = P.select(wl, t0s, inp["qI"], inp["w"], kI)
+    else:
+        idx = None
+    out, mass = P.attend_wl(wl, t0s, q, idx, kv, win, 0, inp["sink"], rope_shift)
+    return out, idx, mass
+
+
+def test_e2e_causality():
+    """Notes 2.3.2: a query never sees a later token.  Perturbing tokens
+    after t0 leaves O[t0] and the top-k of t0 bit-identical."""
+    wl, W, inp = _tiny_inputs(TINY)
+    out0, idx0, mass = _e2e(wl, W, inp)
+    np.testing.assert_allclose(mass, 1.0, atol=1e-12)
+    t0 = 37
+    H2 = inp["H"][0].clone()
+    H2[t0 + 1:] += torch.randn(H2[t0 + 1:].shape, generator=torch.Generator().manual_seed(5))
+    out1, idx1, _ = _e2e(wl, W, inp, H_override=H2)
+    np.testing.assert_array_equal(out1[: t0 + 1], out0[: t0 + 1])
+    np.testing.assert_array_equal(idx1[: t0 + 1], idx0[: t0 + 1])
+    assert np.any(out1[t0 + 1:] != out0[t0 + 1:])
+
+
+def test_e2e_dense_when_k_covers_all_entries():
+    """With k >= the number of visible entries, CSA attends every visible
+    entry: the same as dense (HCA-style) attention over the same cache."""
+    wl, W, inp = _tiny_inputs(TINY.with_(topk=64))
+    H = inp["H"][0]
+    kv, kI, win = P.compress_seq(wl, W, H)
+    t0s = inp["q_pos"].numpy()
+    idx, *_ = P.select(wl, t0s, inp["qI"], inp["w"], kI)
+    sparse, _ = P.attend_wl(wl, t0s, inp["q"], idx, kv, win, 0, inp["sink"])
+    dense, _ = P.attend_wl(wl, t0s, inp["q"], None, kv, win, 0, inp["sink"])
+    np.testing.assert_allclose(sparse, dense, atol=1e-13)
+
+
+@pytest.mark.parametrize("variant", ["csa", "hca"])
+def test_e2e_rope_shift_invariance(variant):
+    """Notes 2.5.2: with q and keys rotated at their positions and the output
+    de-rotated by R_{-t}, O depends on relative positions only: shifting every
+    RoPE position by the same amount leaves O unchanged."""
+    wl = TINY if variant == "csa" else TINY.with_(variant="hca", m=8, n_hI=0, c_I=0, topk=0)
+    wl, W, inp = _tiny_inputs(wl, seed=3)
+    u = inp["q"].double().numpy()
+    t0s = inp["q_pos"].numpy()
+    outs = []
+    for shift in (0.0, 4096.0):
+        q = np.stack([[oracle.rope(u[i, h], wl.rope_dims, wl.rope_base, t0s[i] + shift)
+                       for h in range(wl.n_h)] for i in range(len(t0s))])
+        H = inp["H"][0]
+        raw_kv, kI, _ = None, None, None
+        if wl.variant == "csa":
+            raw = oracle.compress(H, wl.m, W["Wkv_a"], W["Wz_a"], W["B_a"], W["Wkv_b"], W["Wz_b"], W["B_b"])
+            kI = oracle.compress(H, wl.m, W["WIkv_a"], W["WIz_a"], W["BI_a"], W["WIkv_b"], W["WIz_b"], W["BI_b"])
+        else:
+            raw = oracle.compress(H, wl.m, W["Wkv_a"], W["Wz_a"], W["B_a"])
+        kv = oracle.norm_rope_rows(raw, wl.rope_dims, wl.rope_base, wl.rms_eps, shift, wl.m)
+        win = oracle.norm_rope_rows(oracle.matmul(H, W["Wkv_a"]), wl.rope_dims, wl.rope_base,
+                                    wl.rms_eps, shift, 1.0)
+        idx = P.select(wl, t0s, inp["qI"], inp["w"], kI)[0] if wl.variant == "csa" else None
+        out, _ = P.attend_wl(wl, t0s, q, idx, kv, win, 0, inp["sink"], rope_shift=shift)
+        outs.append(out)
+    np.testing.assert_allclose(outs[0], outs[1], atol=1e-9)
