@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA / HCA forward-pass hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  * decode workloads: the compressed cache (entries, indexer keys, window) is
+    resident in HBM; a step scores every visible entry of every sequence
+    (indexer), selects the top k, and attends over the selected entries plus
+    the window (csa_index_topk + csa_attend; hca_attend for HCA);
+  * prefill workloads: csa_compress of the whole sequence, then index/top-k
+    and attention for every token.
+One process per GPU (torchrun for N > 1); each rank runs its own batch (weak
+scaling, no data-path collective).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_09_b200 import binding as bd  # noqa: E402
+from long_context_sparse_09_b200 import synth  # noqa: E402
+from long_context_sparse_09_b200.configs import DEFAULT_BENCH, WORKLOADS  # noqa: E402
+
+METRIC = "CSA decode query-tok/s @1M ctx & prefill tok/s; % of HBM / tensor roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# ncu DRAM traffic per launch of the dominant kernel, with the hash of the
+# source file it was measured on (the value is dropped once the file changes).
+NCU_TRAFFIC = {}
+
+
+# ------------------------------------------------------------------ utils --
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def _src_hash(fname):
+    with open(os.path.join(ROOT, "long_context_sparse_09_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons of this GPU, sampled every 50 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device(f"cuda:{local}"))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- workloads --
+class DecodeStep:
+    """Resident cache + one query per sequence; a step = index/top-k + attend."""
+
+    def __init__(self, wl, device, seed_offset=0):
+        self.wl = wl
+        self.p = bd.params_for(wl)
+        inp = synth.decode_inputs(wl.with_(seed=wl.seed + seed_offset), device=device)
+        self.inp = inp
+        B, N = wl.B, inp["N"]
+        self.N = N
+        self.out = torch.empty(B, wl.n_h, wl.c, dtype=torch.bfloat16, device=device)
+        if wl.variant == "csa":
+            self.idx = torch.empty(B, wl.topk, dtype=torch.int32, device=device)
+            self.ws_i = torch.empty(max(bd.index_topk_workspace_bytes(self.p, B, 1, N), 1),
+                                    dtype=torch.uint8, device=device)
+        self.ws_a = torch.empty(max(bd.attend_workspace_bytes(self.p, B, 1, N), 1),
+                                dtype=torch.uint8, device=device)
+
+    def run(self, q=None, qI=None, w=None):
+        i, wl = self.inp, self.wl
+        q = i["q"] if q is None else q
+        if wl.variant == "csa":
+            bd.csa_index_topk(self.p, i["q_pos"], i["qI"] if qI is None else qI,
+                              i["w"] if w is None else w, i["kI"], self.idx,
+                              workspace=self.ws_i)
+            bd.csa_attend(self.p, i["q_pos"], q, self.idx, i["ckv"], i["ckv_scale"], i["win"],
+                          i["win_scale"], i["win_pos0"], i["sink"], self.out,
+                          workspace=self.ws_a)
+        else:
+            bd.hca_attend(self.p, i["q_pos"], q, i["ckv"], i["ckv_scale"], i["win"],
+                          i["win_scale"], i["win_pos0"], i["sink"], self.out,
+                          workspace=self.ws_a)
+
+    # per-step host<->device traffic of the end-to-end leg
+    def step_inputs(self):
+        i = self.inp
+        names = ["q", "q_pos"] + (["qI", "w"] if self.wl.variant == "csa" else [])
+        return {k: i[k] for k in names}
+
+    def units(self):
+        return self.wl.B  # queries per step
+
+    def dominant(self):
+        """(kernel kind, algorithmic bytes per launch, source file)."""
+        wl, B, N = self.wl, self.wl.B, self.N
+        if wl.variant == "csa":
+            nbytes = B * N * wl.c_I * 2 + B * wl.n_hI * (wl.c_I * 2 + 4) + B * 4
+            return "index_scores", nbytes, "index_topk.cu", "hbm"
+        rb = synth.kv_record_bytes(wl)
+        nbytes = B * (N + wl.n_win) * rb + 2 * B * wl.n_h * wl.c * 2
+        return "attend", nbytes, "attend.cu", "hbm"
+
+    def cpu_baseline(self, max_queries=None):
+        """Oracle (as it stands) on the queries of one step; returns
+        (queries, seconds, sample description)."""
+        import numpy as np
+        import oracle
+        from oracle import pipeline as P
+        wl, i = self.wl, self.inp
+        nq = wl.B if max_queries is None else min(wl.B, max_queries)
+        host = {}
+        for b in range(nq):
+            h = {"q": i["q"][b:b + 1].double().cpu().numpy(),
+                 "pos": i["q_pos"][b:b + 1].cpu().numpy(),
+                 "win": P.cache_values(i["win"][b].cpu(), None if i["win_scale"] is None
+                                       else i["win_scale"][b].cpu(), wl.kv, wl.c, wl.rope_dims),
+                 "wp0": int(i["win_pos0"][b])}
+            if wl.variant == "csa":
+                h["qI"] = i["qI"][b:b + 1].double().cpu().numpy()
+                h["w"] = i["w"][b:b + 1].double().cpu().numpy()
+                h["kI"] = i["kI"][b].double().cpu().numpy()
+            else:
+                h["kv"] = P.cache_values(i["ckv"][b].cpu(), None, wl.kv, wl.c, wl.rope_dims)
+            host[b] = h
+        sink = i["sink"].double().cpu().numpy()
+        t_total = 0.0
+        for b in range(nq):
+            h = host[b]
+            t0 = time.perf_counter()
+            if wl.variant == "csa":
+                scores = oracle.index_scores(h["pos"], wl.m, h["qI"], h["w"], h["kI"])
+                nv = np.array([oracle.nvis(int(h["pos"][0]), wl.m, self.N)], np.int32)
+                idx, _ = oracle.topk(scores, nv, wl.topk)
+                t_total += time.perf_counter() - t0
+                # gather the selected rows (outside the timed part: a format
+                # conversion, not the oracle's arithmetic)
+                sel = idx[0][idx[0] >= 0]
+                rows = P.cache_values(i["ckv"][b][torch.from_numpy(sel).long().to(i["ckv"].device)].cpu(),
+                                      None if i["ckv_scale"] is None else
+                                      i["ckv_scale"][b][torch.from_numpy(sel).long().to(i["ckv"].device)].cpu(),
+                                      wl.kv, wl.c, wl.rope_dims)
+                t0 = time.perf_counter()
+                # entries renumbered 0..k-1, all visible at the query position
+                oracle.attend(h["pos"], h["q"], np.arange(len(sel), dtype=np.int32)[None, :],
+                              wl.m, rows, wl.n_win, h["win"], h["wp0"], sink, wl.rope_dims,
+                              wl.rope_base, wl.softmax_scale)
+            else:
+                P.attend_wl(wl, h["pos"], h["q"], None, h["kv"], h["win"], h["wp0"], sink)
+            t_total += time.perf_counter() - t0
+        return nq, t_total, f"{nq} of the {wl.B} queries of one step (full context each)"
+
+
+# -------------------------------------------------------------------- main --
+def run_ours(args, world, rank, local):
+    from long_context_sparse_09_b200 import build
+    if rank == 0 or world == 1:
+        build.build_library()
+    _barrier(world)
+    wl = WORKLOADS[args.workload]
+    dev = torch.device(f"cuda:{local}")
+    torch.manual_seed(0)
+    if wl.mode != "decode":
+        raise SystemExit("prefill benchmarking: use --workload with a decode workload for now")
+    step = DecodeStep(wl, dev, seed_offset=rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    assert bd.device_status() == 0, "device error word set during warm-up"
+    clocks = ClockSampler(dev)
+    time.sleep(0.15)
+    _barrier(world)
+    torch.cuda.synchronize()
+    bd.profile_enable(True)
+    bd.profile_collect()
+    l0 = bd.kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step.run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    launches = bd.kernel_launches() - l0
+    prof = bd.profile_collect()
+    bd.profile_enable(False)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = _max_over_ranks(ms, world)
+    units = step.units() * world
+    value = units / (ms / 1e3)
+
+    # end to end through the public API: pinned host inputs -> device, step,
+    # result -> pinned host, every step
+    host_in = {k: v.cpu().pin_memory() for k, v in step.step_inputs().items()}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, v in host_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        step.run(q=dev_in["q"], qI=dev_in.get("qI"), w=dev_in.get("w"))
+        host_out.copy_(step.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    assert bd.device_status() == 0, "device error word set during the timed steps"
+
+    kind, nbytes, src, bound = step.dominant()
+    kms, kcnt = prof.get(kind, (0.0, 0))
+    hbm, tfl, peak_src = _peaks()
+    roof = None
+    if kcnt:
+        per_launch_ms = kms / kcnt
+        achieved = nbytes / (per_launch_ms / 1e3) / 1e9
+        tr = NCU_TRAFFIC.get(kind)
+        traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
+        roof = {"bound": bound, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": kind,
+                "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
+                "peak_source": peak_src}
+    kernels = {k: {"ms_per_step": round(v[0] / args.steps, 5), "launches": v[1],
+                   "share": round(v[0] / max(sum(x[0] for x in prof.values()), 1e-12), 4)}
+               for k, v in prof.items() if v[1]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nq, secs, sample = step.cpu_baseline()
+        cpu = {"value": round(nq / secs, 4), "unit": "query-tok/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": sample, "seconds": round(secs, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "query-tok/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.T,
+                       "entries_per_seq": step.N, "m": wl.m, "topk": wl.topk,
+                       "n_h": wl.n_h, "c": wl.c, "kv_format": wl.kv, "n_win": wl.n_win,
+                       "l2": "inputs larger than L2 (cache streamed every step)"},
+            "e2e": {"value": round(step.units() * world / (e2e_ms / 1e3), 2),
+                    "unit": "query-tok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 5)},
+            "gpu_launches": launches,
+            "roofline": roof,
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, world, rank, local):
+    """The oracle as it stands on the host cores, same workload and metric."""
+    if rank != 0:
+        return
+    import oracle
+    wl = WORKLOADS[args.workload]
+    # the inputs are generated on the GPU when one is present (fast), then
+    # copied to the host for the oracle
+    dev = torch.device(f"cuda:{local}") if torch.cuda.is_available() else torch.device("cpu")
+    step = DecodeStep.__new__(DecodeStep)
+    step.wl = wl
+    step.inp = synth.decode_inputs(wl, device=dev)
+    step.N = step.inp["N"]
+    nq_per_step = 1
+    total_q, total_s = 0, 0.0
+    for s in range(args.warmup + args.steps):
+        nq, secs, sample = step.cpu_baseline(max_queries=nq_per_step)
+        if s >= args.warmup:
+            total_q += nq
+            total_s += secs
+    v = total_q / total_s
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "query-tok/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total_s / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.T},
+            "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "value": round(v, 4),
+                             "unit": "query-tok/s",
+                             "sample": f"{nq_per_step} query (full {wl.T}-token context) per step"},
+            "e2e": {"value": round(v, 4), "unit": "query-tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = _dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * csa.h -- C ABI of the B200 (sm_100a) CSA / HCA forward pass.
+ *
+ * The operations are those of DeepSeek-V4's Compressed Sparse Attention and
+ * Heavily Compressed Attention as described in "DeepSeekV4技术报告阅读笔记"
+ * (zouxinn.github.io; cited below as [N] with its section / equation numbers)
+ * and "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" (PaperTrace; cited as [P]).
+ *
+ * Conventions for every call
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory, laid
+ *     out row-major with the last dimension contiguous, as stated per
+ *     argument.  The library allocates nothing and keeps no state besides one
+ *     device error word per GPU.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; outputs are valid once the stream has
+ *     reached the call.
+ *   - Argument errors are reported synchronously by the return value before
+ *     anything is launched.  Errors found on the device (an index or window
+ *     row out of range) set bits in the device error word, which
+ *     csa_device_status() reads; the offending element is skipped, never
+ *     dereferenced.
+ *   - Queries are numbered r = b*Q + j for sequence b < B and query j < Q.
+ *     Positions are 0-based token positions within the sequence.
+ *   - A compressed entry s covers tokens m*s .. m*s+m-1 (its a-window) and is
+ *     visible to a query at position t0 iff s < floor((t0+1)/m) ([N] 2.3.2,
+ *     read as "only complete blocks").
+ *   - KV formats: CSA_F32 / CSA_BF16 rows of c values; CSA_KV_FP8MIX rows of
+ *     (c - rope_dims) OCP E4M3 codes followed by rope_dims bf16 values
+ *     ((c - rope_dims) + 2*rope_dims bytes per row) plus one fp32 scale per
+ *     row in a separate plane: value_j = e4m3(code_j) * scale ([P] 2.5: RoPE
+ *     dims in BF16, the rest in FP8).
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* csa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_ARG = 1,         /* null pointer or bad scalar argument */
+  CSA_ERR_SHAPE = 2,       /* inconsistent or unsupported sizes */
+  CSA_ERR_ALIGN = 3,       /* pointer not 16-byte aligned */
+  CSA_ERR_DTYPE = 4,       /* unsupported dtype / KV format combination */
+  CSA_ERR_CUDA = 5,        /* a CUDA launch or query failed */
+  CSA_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out */
+  CSA_ERR_UNSUPPORTED = 7, /* valid request this build does not implement */
+  CSA_ERR_WORKSPACE = 8    /* workspace missing or smaller than required */
+} csa_status;
+
+typedef enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_KV_FP8MIX = 2 } csa_dtype;
+
+/* Device error-word bits (csa_device_status). */
+#define CSA_DEV_BAD_INDEX 0x1u  /* a top-k index >= the visible entries */
+#define CSA_DEV_BAD_WINDOW 0x2u /* a window token outside the window rows */
+#define CSA_DEV_TIMEOUT 0x4u    /* a bounded wait gave up */
+
+typedef struct {
+  int m;          /* tokens per compressed entry (CSA m, HCA m') */
+  int overlap;    /* 1: CSA two-window compressor [N] eq. 11-12;
+                     0: HCA single window [N] eq. 22-23 */
+  int c;          /* entry width (key = value width) */
+  int rope_dims;  /* RoPE on the last rope_dims of c (even, <= c) */
+  int c_I;        /* indexer key width (CSA only) */
+  int n_hI;       /* indexer heads (CSA only) */
+  int n_h;        /* query heads sharing the one KV head */
+  int topk;       /* entries selected per query (CSA only) */
+  int n_win;      /* sliding-window tokens, >= 0 */
+  float rope_base;     /* RoPE base: pair p turns by pos * base^(-2p/rope_dims) */
+  float rms_eps;       /* RMSNorm eps (unit gain) */
+  float softmax_scale; /* logit scale of q.k (the sink logit is not scaled) */
+  int act;        /* csa_dtype of H, weights, q, q^I: CSA_F32 or CSA_BF16 */
+  int kv;         /* csa_dtype of the entry / window caches */
+} csa_params;
+
+/* ---------------------------------------------------------------------------
+ * Compressor weights.  [N] eq. 9-10 (CSA: W^{aKV}, W^{bKV}, W^{aZ}, W^{bZ}
+ * in R^{d x c}, and the same four at width c_I for the indexer keys, [N]
+ * 2.3.2 / [P] 2.2) and eq. 20-21 (HCA: W^{KV}, W^Z); position biases
+ * B^a, B^b in R^{m x c} ([N] eq. 11; the page prints "m x b", read as m x c).
+ *
+ * csa_pack_weights copies the caller's matrices (act dtype, [d][width] each,
+ * as in C = H W) and fp32 biases ([m][width]) into one packed buffer of
+ * csa_packed_weight_bytes() bytes, in the layout csa_compress reads.  For
+ * HCA (overlap = 0) pass the single branch as *_a and NULL for every *_b and
+ * indexer argument.  The packed buffer is caller-owned and may be reused for
+ * any number of csa_compress calls with the same params and d.
+ * ------------------------------------------------------------------------- */
+size_t csa_packed_weight_bytes(const csa_params* p, int d);
+csa_status csa_pack_weights(const csa_params* p, int d,
+                            const void* Wkv_a, const void* Wkv_b,
+                            const void* Wz_a, const void* Wz_b,
+                            const void* WIkv_a, const void* WIkv_b,
+                            const void* WIz_a, const void* WIz_b,
+                            const float* B_a, const float* B_b,
+                            const float* BI_a, const float* BI_b,
+                            void* packed, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_compress: overlapped two-window compression of B sequences of T tokens
+ * ([N] eq. 9-12, [P] 2.1), followed by RMSNorm (unit gain, [N] 2.5.1) and
+ * RoPE at position m*i on the last rope_dims ([N] 2.5.2; the entry position
+ * is read as the first token of its a-window) of each entry i.
+ *   H        [B][T][d]            act dtype
+ *   packed   from csa_pack_weights
+ *   ckv      [B][T/m][row]        kv format: compressed entries (T/m = floor)
+ *   ckv_scale[B][T/m] fp32        CSA_KV_FP8MIX only, else NULL
+ *   kI       [B][T/m][c_I]        act dtype: indexer keys (same compressor
+ *                                 at width c_I, no norm, no RoPE)
+ *   win      [B][T][row]          kv format: per-token window rows, RMSNorm +
+ *                                 RoPE(position j) of C^a_j = h_j W^{aKV}
+ *                                 (the uncompressed KV of the window branch,
+ *                                 [N] 2.5.3); NULL to skip
+ *   win_scale[B][T] fp32          CSA_KV_FP8MIX with win != NULL, else NULL
+ *   workspace / ws_bytes          >= csa_compress_workspace_bytes()
+ * hca_compress is the same with overlap = 0 ([N] eq. 20-23, [P] 2.3) and no
+ * indexer keys (kI must be NULL); its window rows use C_j = h_j W^{KV}.
+ * ------------------------------------------------------------------------- */
+size_t csa_compress_workspace_bytes(const csa_params* p, int B, int T, int d);
+csa_status csa_compress(const csa_params* p, int B, int T, int d,
+                        const void* H, const void* packed,
+                        void* ckv, float* ckv_scale, void* kI,
+                        void* win, float* win_scale,
+                        void* workspace, size_t ws_bytes, csa_stream_t stream);
+csa_status hca_compress(const csa_params* p, int B, int T, int d,
+                        const void* H, const void* packed,
+                        void* ckv, float* ckv_scale,
+                        void* win, float* win_scale,
+                        void* workspace, size_t ws_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_index_topk: Lightning-Indexer scores and top-k selection ([N] eq. 16-17,
+ * [P] 2.2):  I[r][s] = sum_h w[r][h] * ReLU(qI[r][h] . kI[b][s])  for every
+ * visible s, then the topk largest.  Ties are broken towards the lower index.
+ *   q_pos    [B*Q] int32          query positions t0
+ *   qI       [B*Q][n_hI][c_I]     act dtype
+ *   w        [B*Q][n_hI] fp32     head weights
+ *   kI       [B][N][c_I]          act dtype: indexer-key cache
+ *   idx_out  [B*Q][topk] int32    selected entries in ascending order, -1
+ *                                 padded when fewer than topk are visible
+ *   score_out[B*Q][topk] fp32     score of each selected entry (nullable)
+ *   workspace / ws_bytes          >= csa_index_topk_workspace_bytes()
+ * Scores are computed from the stored values with fp32 accumulation.
+ * ------------------------------------------------------------------------- */
+size_t csa_index_topk_workspace_bytes(const csa_params* p, int B, int Q, int N);
+csa_status csa_index_topk(const csa_params* p, int B, int Q,
+                          const int32_t* q_pos, const void* qI, const float* w,
+                          const void* kI, int N, int32_t* idx_out,
+                          float* score_out, void* workspace, size_t ws_bytes,
+                          csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_attend: shared-KV multi-query attention of each query over its
+ * selected entries and its last n_win tokens, in ONE softmax whose
+ * denominator also holds exp(z'_h) ([N] eq. 19, 2.5.3, eq. 27; [P] 2.4),
+ * followed by R_{-t0} on the last rope_dims of each head's output ([N]
+ * 2.5.2).  logits = softmax_scale * q_h . key; key = value = the stored row.
+ *   q_pos    [B*Q] int32           query positions t0
+ *   q        [B*Q][n_h][c]         act dtype, already normalised and rotated
+ *   idx      [B*Q][topk] int32     entries to attend (-1 = unused slot)
+ *   ckv      [B][N][row], ckv_scale [B][N] (FP8MIX only, else NULL)
+ *   win      [B][W][row], win_scale [B][W] (FP8MIX only, else NULL): row w
+ *            of sequence b holds token win_pos0[b] + w; the query attends
+ *            tokens max(0, t0-n_win+1) .. t0, which must all be present
+ *   win_pos0 [B] int32
+ *   sink     [n_h] fp32            sink logits z'_h
+ *   out      [B*Q][n_h][c]         act dtype
+ *   workspace / ws_bytes           >= csa_attend_workspace_bytes()
+ * hca_attend: the same over ALL visible entries s < floor((t0+1)/m) (no
+ * selection, [N] eq. 26, [P] 2.3) plus the window.
+ * ------------------------------------------------------------------------- */
+size_t csa_attend_workspace_bytes(const csa_params* p, int B, int Q, int N);
+csa_status csa_attend(const csa_params* p, int B, int Q, const int32_t* q_pos,
+                      const void* q, const int32_t* idx,
+                      const void* ckv, const float* ckv_scale, int N,
+                      const void* win, const float* win_scale, int W,
+                      const int32_t* win_pos0, const float* sink, void* out,
+                      void* workspace, size_t ws_bytes, csa_stream_t stream);
+csa_status hca_attend(const csa_params* p, int B, int Q, const int32_t* q_pos,
+                      const void* q, const void* ckv, const float* ckv_scale,
+                      int N, const void* win, const float* win_scale, int W,
+                      const int32_t* win_pos0, const float* sink, void* out,
+                      void* workspace, size_t ws_bytes, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Status and diagnostics.
+ * csa_device_status waits for `stream`, returns the device error word of the
+ * current GPU in *flags (CSA_DEV_* bits, 0 = clean) and clears it.
+ * csa_kernel_launches returns how many kernels this library has launched in
+ * this process (all GPUs), a counter for benchmarks.
+ * ------------------------------------------------------------------------- */
+csa_status csa_device_status(csa_stream_t stream, uint32_t* flags);
+const char* csa_status_string(csa_status s);
+uint64_t csa_kernel_launches(void);
+int csa_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Per-kernel device-time profiling.  While enabled, every kernel launch of
+ * the library is bracketed by two CUDA events on its stream (a few us of host
+ * time per launch, nothing on the device timeline).  csa_profile_collect
+ * waits for the recorded events, writes for each kernel kind k <
+ * csa_profile_kernel_count() the summed device time in ms and the number of
+ * launches since the previous collect (arrays of that length, caller-owned),
+ * and starts a new collection.  Kind names come from csa_profile_kernel_name.
+ * ------------------------------------------------------------------------- */
+void csa_profile_enable(int on);
+int csa_profile_kernel_count(void);
+const char* csa_profile_kernel_name(int kind);
+csa_status csa_profile_collect(double* total_ms, uint64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

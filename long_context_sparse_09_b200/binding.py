@@ -1,0 +1,231 @@
+"""Thin Python binding of libcsa.so (include/csa.h) through ctypes.
+
+Argument marshalling only: every step of the CSA / HCA forward pass runs in
+the library's CUDA kernels.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if libcsa.so is missing or fails to load,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_F32, CSA_BF16, CSA_KV_FP8MIX = 0, 1, 2
+_DT = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8mix": CSA_KV_FP8MIX}
+DEV_BAD_INDEX, DEV_BAD_WINDOW, DEV_TIMEOUT = 0x1, 0x2, 0x4
+
+
+class CsaError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn}: status {status} ({msg})")
+        self.status = status
+
+
+class CsaParams(C.Structure):
+    _fields_ = [("m", C.c_int), ("overlap", C.c_int), ("c", C.c_int),
+                ("rope_dims", C.c_int), ("c_I", C.c_int), ("n_hI", C.c_int),
+                ("n_h", C.c_int), ("topk", C.c_int), ("n_win", C.c_int),
+                ("rope_base", C.c_float), ("rms_eps", C.c_float),
+                ("softmax_scale", C.c_float), ("act", C.c_int), ("kv", C.c_int)]
+
+
+def params_for(wl) -> CsaParams:
+    """csa_params of a configs.Workload."""
+    return CsaParams(m=wl.m, overlap=wl.overlap, c=wl.c, rope_dims=wl.rope_dims,
+                     c_I=wl.c_I, n_hI=wl.n_hI, n_h=wl.n_h, topk=wl.topk,
+                     n_win=wl.n_win, rope_base=wl.rope_base, rms_eps=wl.rms_eps,
+                     softmax_scale=wl.softmax_scale, act=_DT[wl.act], kv=_DT[wl.kv])
+
+
+_lib = None
+_vp, _i, _sz = C.c_void_p, C.c_int, C.c_size_t
+_P = C.POINTER(CsaParams)
+
+_SIGS = {
+    "csa_abi_version": (C.c_int, []),
+    "csa_kernel_launches": (C.c_uint64, []),
+    "csa_status_string": (C.c_char_p, [C.c_int]),
+    "csa_device_status": (C.c_int, [_vp, C.POINTER(C.c_uint32)]),
+    "csa_profile_enable": (None, [C.c_int]),
+    "csa_profile_kernel_count": (C.c_int, []),
+    "csa_profile_kernel_name": (C.c_char_p, [C.c_int]),
+    "csa_profile_collect": (C.c_int, [C.POINTER(C.c_double), C.POINTER(C.c_uint64)]),
+    "csa_packed_weight_bytes": (_sz, [_P, _i]),
+    "csa_pack_weights": (C.c_int, [_P, _i] + [_vp] * 12 + [_vp, _vp]),
+    "csa_compress_workspace_bytes": (_sz, [_P, _i, _i, _i]),
+    "csa_compress": (C.c_int, [_P, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "hca_compress": (C.c_int, [_P, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "csa_index_topk_workspace_bytes": (_sz, [_P, _i, _i, _i]),
+    "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "csa_attend_workspace_bytes": (_sz, [_P, _i, _i, _i]),
+    "csa_attend": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp,
+                             _vp, _vp, _sz, _vp]),
+    "hca_attend": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp,
+                             _vp, _vp, _sz, _vp]),
+}
+
+
+def lib():
+    """The loaded libcsa.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library missing: {LIB_PATH} (run "
+                               "`python -m long_context_sparse_09_b200.build`)")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensor expected")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _check(fn, st):
+    if st != 0:
+        raise CsaError(fn, st, lib().csa_status_string(st).decode())
+
+
+def _ws(nbytes, device, workspace):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def kernel_launches() -> int:
+    return int(lib().csa_kernel_launches())
+
+
+def device_status(stream=None) -> int:
+    flags = C.c_uint32(0)
+    _check("csa_device_status", lib().csa_device_status(_stream(stream), C.byref(flags)))
+    return flags.value
+
+
+def profile_enable(on: bool = True):
+    lib().csa_profile_enable(1 if on else 0)
+
+
+def profile_collect() -> dict:
+    """{kernel kind: (total device ms, launches)} since the previous collect."""
+    n = lib().csa_profile_kernel_count()
+    ms = (C.c_double * n)()
+    cnt = (C.c_uint64 * n)()
+    _check("csa_profile_collect", lib().csa_profile_collect(ms, cnt))
+    return {lib().csa_profile_kernel_name(k).decode(): (ms[k], cnt[k]) for k in range(n)}
+
+
+# ----------------------------------------------------------------- pack --
+def csa_pack_weights(p: CsaParams, W: dict, stream=None) -> torch.Tensor:
+    """Pack compressor weights ([d][width] each, act dtype) and fp32 biases
+    ([m][width]) into the library's layout; returns the packed uint8 buffer."""
+    d = W["Wkv_a"].shape[0]
+    dev = W["Wkv_a"].device
+    nbytes = lib().csa_packed_weight_bytes(C.byref(p), d)
+    if nbytes == 0:
+        raise CsaError("csa_packed_weight_bytes", 2, "invalid params")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    g = W.get
+    st = lib().csa_pack_weights(C.byref(p), d, _p(g("Wkv_a")), _p(g("Wkv_b")), _p(g("Wz_a")),
+                                _p(g("Wz_b")), _p(g("WIkv_a")), _p(g("WIkv_b")),
+                                _p(g("WIz_a")), _p(g("WIz_b")), _p(g("B_a")), _p(g("B_b")),
+                                _p(g("BI_a")), _p(g("BI_b")), _p(packed), _stream(stream))
+    _check("csa_pack_weights", st)
+    return packed
+
+
+# ------------------------------------------------------------- compress --
+def compress_workspace_bytes(p: CsaParams, B, T, d) -> int:
+    return lib().csa_compress_workspace_bytes(C.byref(p), B, T, d)
+
+
+def csa_compress(p: CsaParams, H, packed, ckv, ckv_scale, kI, win, win_scale,
+                 workspace=None, stream=None):
+    B, T, d = H.shape
+    ws, wsb = _ws(compress_workspace_bytes(p, B, T, d), H.device, workspace)
+    st = lib().csa_compress(C.byref(p), B, T, d, _p(H), _p(packed), _p(ckv), _p(ckv_scale),
+                            _p(kI), _p(win), _p(win_scale), _p(ws), wsb, _stream(stream))
+    _check("csa_compress", st)
+
+
+def hca_compress(p: CsaParams, H, packed, ckv, ckv_scale, win, win_scale,
+                 workspace=None, stream=None):
+    B, T, d = H.shape
+    ws, wsb = _ws(compress_workspace_bytes(p, B, T, d), H.device, workspace)
+    st = lib().hca_compress(C.byref(p), B, T, d, _p(H), _p(packed), _p(ckv), _p(ckv_scale),
+                            _p(win), _p(win_scale), _p(ws), wsb, _stream(stream))
+    _check("hca_compress", st)
+
+
+# --------------------------------------------------------- index / top-k --
+def index_topk_workspace_bytes(p: CsaParams, B, Q, N) -> int:
+    return lib().csa_index_topk_workspace_bytes(C.byref(p), B, Q, N)
+
+
+def csa_index_topk(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out=None,
+                   workspace=None, stream=None):
+    """q_pos [B*Q], qI [B*Q][n_hI][c_I], w [B*Q][n_hI], kI [B][N][c_I] ->
+    idx_out [B*Q][topk] (and score_out [B*Q][topk])."""
+    B, N = kI.shape[0], kI.shape[1]
+    Q = qI.shape[0] // B
+    ws, wsb = _ws(index_topk_workspace_bytes(p, B, Q, N), qI.device, workspace)
+    st = lib().csa_index_topk(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI), N,
+                              _p(idx_out), _p(score_out), _p(ws), wsb, _stream(stream))
+    _check("csa_index_topk", st)
+
+
+# ---------------------------------------------------------------- attend --
+def attend_workspace_bytes(p: CsaParams, B, Q, N) -> int:
+    return lib().csa_attend_workspace_bytes(C.byref(p), B, Q, N)
+
+
+def csa_attend(p: CsaParams, q_pos, q, idx, ckv, ckv_scale, win, win_scale, win_pos0,
+               sink, out, workspace=None, stream=None):
+    """q [B*Q][n_h][c], idx [B*Q][topk], ckv [B][N][row], win [B][W][row] ->
+    out [B*Q][n_h][c]."""
+    B, N = ckv.shape[0], ckv.shape[1]
+    Q = q.shape[0] // B
+    W = win.shape[1] if win is not None else 0
+    ws, wsb = _ws(attend_workspace_bytes(p, B, Q, N), q.device, workspace)
+    st = lib().csa_attend(C.byref(p), B, Q, _p(q_pos), _p(q), _p(idx), _p(ckv), _p(ckv_scale),
+                          N, _p(win), _p(win_scale), W, _p(win_pos0), _p(sink), _p(out),
+                          _p(ws), wsb, _stream(stream))
+    _check("csa_attend", st)
+
+
+def hca_attend(p: CsaParams, q_pos, q, ckv, ckv_scale, win, win_scale, win_pos0, sink,
+               out, workspace=None, stream=None):
+    B, N = ckv.shape[0], ckv.shape[1]
+    Q = q.shape[0] // B
+    W = win.shape[1] if win is not None else 0
+    ws, wsb = _ws(attend_workspace_bytes(p, B, Q, N), q.device, workspace)
+    st = lib().hca_attend(C.byref(p), B, Q, _p(q_pos), _p(q), _p(ckv), _p(ckv_scale), N,
+                          _p(win), _p(win_scale), W, _p(win_pos0), _p(sink), _p(out),
+                          _p(ws), wsb, _stream(stream))
+    _check("hca_attend", st)

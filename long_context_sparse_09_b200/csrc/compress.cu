@@ -1,0 +1,337 @@
+// compress.cu -- CSA / HCA KV compression ("DeepSeekV4技术报告阅读笔记" eq. 9-12
+// and 20-23; RMSNorm and partial RoPE of section 2.5.1-2.5.2; the FP8/BF16
+// entry format of "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" section 2.5).
+//
+// Path: (1) projection GEMM P = H * Wpacked^T into an fp32 workspace
+// [B*T][ncols] (columns C^a | C^b | Z^a | Z^b | indexer C^a | C^b | Z^a | Z^b),
+// (2) one CTA per entry folds its 2m rows with a per-channel softmax, applies
+// RMSNorm + RoPE and stores the entry (bf16 / fp32 / FP8-mixed) and its
+// indexer key, (3) one CTA per token writes the window row.
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+static int esize(int dt) { return dt == CSA_F32 ? 4 : 2; }
+
+PackLayout pack_layout(const csa_params& p, int d) {
+  PackLayout L;
+  const int c = p.c, ci = p.c_I;
+  if (p.overlap) {
+    L.col_Ca = 0; L.col_Cb = c; L.col_Za = 2 * c; L.col_Zb = 3 * c;
+    L.col_CIa = 4 * c; L.col_CIb = 4 * c + ci;
+    L.col_ZIa = 4 * c + 2 * ci; L.col_ZIb = 4 * c + 3 * ci;
+    L.ncols = 4 * c + 4 * ci;
+    L.nb = 2 * c + 2 * ci;
+    L.b_Ba = 0; L.b_Bb = c; L.b_BIa = 2 * c; L.b_BIb = 2 * c + ci;
+  } else {
+    L.col_Ca = 0; L.col_Za = c;
+    L.ncols = 2 * c;
+    L.nb = c;
+    L.b_Ba = 0;
+  }
+  L.bias_off = align_up((size_t)L.ncols * d * esize(p.act), 256);
+  L.total = L.bias_off + align_up((size_t)p.m * L.nb * 4, 256);
+  return L;
+}
+
+// ------------------------------------------------------------------ pack --
+// dst[(col0 + j) * d + k] = W[k * width + j]  (a 32x32-tiled transpose)
+template <typename T>
+__global__ void pack_transpose(const T* __restrict__ W, int d, int width,
+                               T* __restrict__ dst, int col0) {
+  __shared__ T tile[32][33];
+  const int k0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    int k = k0 + r, j = j0 + threadIdx.x;
+    if (k < d && j < width) tile[r][threadIdx.x] = W[(size_t)k * width + j];
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    int j = j0 + r, k = k0 + threadIdx.x;
+    if (k < d && j < width) dst[(size_t)(col0 + j) * d + k] = tile[threadIdx.x][r];
+  }
+}
+
+__global__ void pack_bias(const float* __restrict__ Bsrc, int m, int width,
+                          float* __restrict__ dst, int nb, int col0) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < m * width) {
+    int r = i / width, j = i % width;
+    dst[(size_t)r * nb + col0 + j] = Bsrc[i];
+  }
+}
+
+csa_status launch_pack(const csa_params& p, int d, const void* const W[8],
+                       const float* const Bias[4], void* packed, cudaStream_t st) {
+  PackLayout L = pack_layout(p, d);
+  const int cols[8] = {L.col_Ca, L.col_Cb, L.col_Za, L.col_Zb,
+                       L.col_CIa, L.col_CIb, L.col_ZIa, L.col_ZIb};
+  const int widths[8] = {p.c, p.c, p.c, p.c, p.c_I, p.c_I, p.c_I, p.c_I};
+  // argument order: Wkv_a, Wkv_b, Wz_a, Wz_b, WIkv_a, WIkv_b, WIz_a, WIz_b
+  for (int t = 0; t < 8; ++t) {
+    int col = cols[t];
+    if (col < 0) continue;
+    int width = widths[t];
+    dim3 grid((width + 31) / 32, (d + 31) / 32), block(32, 8);
+    if (p.act == CSA_F32)
+      CSA_LAUNCH(KK_PACK, st, pack_transpose<float><<<grid, block, 0, st>>>(
+                                  (const float*)W[t], d, width, (float*)packed, col));
+    else
+      CSA_LAUNCH(KK_PACK, st, pack_transpose<__nv_bfloat16><<<grid, block, 0, st>>>(
+                                  (const __nv_bfloat16*)W[t], d, width,
+                                  (__nv_bfloat16*)packed, col));
+  }
+  float* bias = (float*)((char*)packed + L.bias_off);
+  const int bcols[4] = {L.b_Ba, L.b_Bb, L.b_BIa, L.b_BIb};
+  const int bw[4] = {p.c, p.c, p.c_I, p.c_I};
+  for (int t = 0; t < 4; ++t) {
+    if (bcols[t] < 0) continue;
+    int n = p.m * bw[t];
+    CSA_LAUNCH(KK_PACK, st, pack_bias<<<(n + 255) / 256, 256, 0, st>>>(
+                                Bias[t], p.m, bw[t], bias, L.nb, bcols[t]));
+  }
+  return last_launch_status();
+}
+
+// ------------------------------------------------------------------ GEMM --
+// C[M][N] (fp32) = A[M][K] * Bm[N][K]^T, fp32 accumulation in k order.
+// 64x64 tile per 256-thread CTA, 4x4 outputs per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) gemm_nt_simt(const T* __restrict__ A,
+                                                    const T* __restrict__ Bm,
+                                                    float* __restrict__ C, int M,
+                                                    int N, int K) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      int r = i >> 4, kk = i & 15;
+      int gk = k0 + kk;
+      int gm = m0 + r, gn = n0 + r;
+      As[kk][r] = (gm < M && gk < K) ? to_f32(A[(size_t)gm * K + gk]) : 0.f;
+      Bs[kk][r] = (gn < N && gk < K) ? to_f32(Bm[(size_t)gn * K + gk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int gn = n0 + tx * 4 + j;
+      if (gn < N) C[(size_t)gm * N + gn] = acc[i][j];
+    }
+  }
+}
+
+// ------------------------------------------------------------ fold / store --
+// One channel of entry i: softmax over the a rows m*i..m*i+m-1 (logit Z^a +
+// B^a) and, when overlapping and i > 0, the b rows m*(i-1)..m*i-1 (Z^b + B^b);
+// returns sum S * C over the same rows.
+__device__ float fold_channel(const float* __restrict__ Pb, int ncols, int m,
+                              int i, bool use_b, int cCa, int cZa, int cCb,
+                              int cZb, const float* __restrict__ bias, int nb,
+                              int bA, int bB, int ch) {
+  float mx = -INFINITY;
+  for (int r = 0; r < m; ++r) {
+    float z = Pb[(size_t)(m * i + r) * ncols + cZa + ch] + bias[r * nb + bA + ch];
+    mx = fmaxf(mx, z);
+  }
+  if (use_b)
+    for (int r = 0; r < m; ++r) {
+      float z = Pb[(size_t)(m * (i - 1) + r) * ncols + cZb + ch] + bias[r * nb + bB + ch];
+      mx = fmaxf(mx, z);
+    }
+  float den = 0.f, num = 0.f;
+  for (int r = 0; r < m; ++r) {
+    size_t row = (size_t)(m * i + r) * ncols;
+    float e = expf(Pb[row + cZa + ch] + bias[r * nb + bA + ch] - mx);
+    den += e;
+    num = fmaf(e, Pb[row + cCa + ch], num);
+  }
+  if (use_b)
+    for (int r = 0; r < m; ++r) {
+      size_t row = (size_t)(m * (i - 1) + r) * ncols;
+      float e = expf(Pb[row + cZb + ch] + bias[r * nb + bB + ch] - mx);
+      den += e;
+      num = fmaf(e, Pb[row + cCb + ch], num);
+    }
+  return num / den;
+}
+
+// RMSNorm (unit gain) and RoPE at `pos` of the row held in shared xs[c].
+__device__ void norm_rope_shared(float* xs, int c, int rd, float eps, double pos,
+                                 double base, float* red) {
+  float ss = 0.f;
+  for (int ch = threadIdx.x; ch < c; ch += blockDim.x) ss = fmaf(xs[ch], xs[ch], ss);
+  ss = block_reduce<false>(ss, red);
+  float inv = 1.0f / sqrtf(ss / (float)c + eps);
+  __syncthreads();
+  for (int ch = threadIdx.x; ch < c; ch += blockDim.x) xs[ch] *= inv;
+  __syncthreads();
+  for (int pp = threadIdx.x; pp < rd / 2; pp += blockDim.x) {
+    float cs, sn;
+    rope_cs(pos, pp, rd, base, &cs, &sn);
+    int j = c - rd + 2 * pp;
+    float x0 = xs[j], x1 = xs[j + 1];
+    xs[j] = x0 * cs - x1 * sn;
+    xs[j + 1] = x0 * sn + x1 * cs;
+  }
+  __syncthreads();
+}
+
+// Store the row xs[c] in KV format kKV (0 f32, 1 bf16, 2 fp8-mixed).
+template <int kKV>
+__device__ void store_kv_row(const float* xs, int c, int rd, void* dst,
+                             float* dst_scale, float* red) {
+  if (kKV == CSA_F32) {
+    for (int ch = threadIdx.x; ch < c; ch += blockDim.x) ((float*)dst)[ch] = xs[ch];
+  } else if (kKV == CSA_BF16) {
+    for (int ch = threadIdx.x; ch < c; ch += blockDim.x)
+      ((__nv_bfloat16*)dst)[ch] = __float2bfloat16_rn(xs[ch]);
+  } else {
+    const int nf = c - rd;
+    float amax = 0.f;
+    for (int ch = threadIdx.x; ch < nf; ch += blockDim.x) amax = fmaxf(amax, fabsf(xs[ch]));
+    amax = block_reduce<true>(amax, red);
+    float s = amax > 0.f ? amax / 448.0f : 1.0f;
+    uint8_t* codes = (uint8_t*)dst;
+    for (int ch = threadIdx.x; ch < nf; ch += blockDim.x) codes[ch] = f32_to_e4m3(xs[ch] / s);
+    __nv_bfloat16* rope = (__nv_bfloat16*)(codes + nf);
+    for (int ch = nf + threadIdx.x; ch < c; ch += blockDim.x)
+      rope[ch - nf] = __float2bfloat16_rn(xs[ch]);
+    if (threadIdx.x == 0) *dst_scale = s;
+  }
+}
+
+__host__ __device__ inline size_t kv_row_bytes(int kv, int c, int rd) {
+  return kv == CSA_F32 ? (size_t)4 * c : kv == CSA_BF16 ? (size_t)2 * c : (size_t)(c - rd) + 2 * rd;
+}
+
+template <typename TA, int kKV>
+__global__ void __launch_bounds__(256) fold_entries(
+    const float* __restrict__ P, int ncols, const float* __restrict__ bias, int nb,
+    PackLayout L, int B, int T, int nE, int m, int overlap, int c, int rd,
+    int cI, float eps, double base, void* __restrict__ ckv,
+    float* __restrict__ ckv_scale, TA* __restrict__ kI) {
+  extern __shared__ float xs[];  // c floats
+  __shared__ float red[32];
+  const int b = blockIdx.x / nE, i = blockIdx.x % nE;
+  const float* Pb = P + (size_t)b * T * ncols;
+  const bool use_b = overlap && i > 0;
+  for (int ch = threadIdx.x; ch < c; ch += blockDim.x)
+    xs[ch] = fold_channel(Pb, ncols, m, i, use_b, L.col_Ca, L.col_Za, L.col_Cb,
+                          L.col_Zb, bias, nb, L.b_Ba, L.b_Bb, ch);
+  __syncthreads();
+  norm_rope_shared(xs, c, rd, eps, (double)m * i, base, red);
+  const size_t rowb = kv_row_bytes(kKV, c, rd);
+  const size_t e = (size_t)b * nE + i;
+  store_kv_row<kKV>(xs, c, rd, (char*)ckv + e * rowb,
+                    ckv_scale ? ckv_scale + e : nullptr, red);
+  if (kI != nullptr)
+    for (int ch = threadIdx.x; ch < cI; ch += blockDim.x)
+      kI[e * cI + ch] = from_f32<TA>(fold_channel(Pb, ncols, m, i, use_b, L.col_CIa,
+                                                  L.col_ZIa, L.col_CIb, L.col_ZIb, bias,
+                                                  nb, L.b_BIa, L.b_BIb, ch));
+}
+
+template <int kKV>
+__global__ void __launch_bounds__(256) window_rows(const float* __restrict__ P,
+                                                  int ncols, int colC, int T, int c,
+                                                  int rd, float eps, double base,
+                                                  void* __restrict__ win,
+                                                  float* __restrict__ win_scale) {
+  extern __shared__ float xs[];
+  __shared__ float red[32];
+  const size_t row = blockIdx.x;  // b*T + j
+  const int j = (int)(row % T);
+  for (int ch = threadIdx.x; ch < c; ch += blockDim.x) xs[ch] = P[row * ncols + colC + ch];
+  __syncthreads();
+  norm_rope_shared(xs, c, rd, eps, (double)j, base, red);
+  const size_t rowb = kv_row_bytes(kKV, c, rd);
+  store_kv_row<kKV>(xs, c, rd, (char*)win + row * rowb,
+                    win_scale ? win_scale + row : nullptr, red);
+}
+
+size_t compress_ws_bytes(const csa_params& p, int B, int T, int d) {
+  PackLayout L = pack_layout(p, d);
+  return align_up((size_t)B * T * L.ncols * sizeof(float), 256);
+}
+
+template <typename TA, int kKV>
+static void launch_fold(const csa_params& p, const PackLayout& L, const float* P,
+                        const float* bias, int B, int T, int nE, void* ckv,
+                        float* ckv_scale, void* kI, void* win, float* win_scale,
+                        cudaStream_t st) {
+  size_t smem = (size_t)p.c * sizeof(float);
+  if (nE > 0) {
+    CSA_LAUNCH(KK_FOLD, st, fold_entries<TA, kKV><<<B * nE, 256, smem, st>>>(
+        P, L.ncols, bias, L.nb, L, B, T, nE, p.m, p.overlap, p.c, p.rope_dims, p.c_I,
+        p.rms_eps, (double)p.rope_base, ckv, ckv_scale, (TA*)kI));
+  }
+  if (win != nullptr) {
+    CSA_LAUNCH(KK_WINDOW, st, window_rows<kKV><<<B * T, 256, smem, st>>>(
+        P, L.ncols, L.col_Ca, T, p.c, p.rope_dims, p.rms_eps, (double)p.rope_base, win,
+        win_scale));
+  }
+}
+
+csa_status launch_compress(const csa_params& p, int B, int T, int d,
+                           const void* H, const void* packed, void* ckv,
+                           float* ckv_scale, void* kI, void* win,
+                           float* win_scale, void* ws, cudaStream_t st) {
+  PackLayout L = pack_layout(p, d);
+  const int M = B * T;
+  float* P = (float*)ws;
+  dim3 grid((L.ncols + 63) / 64, (M + 63) / 64);
+  if (p.act == CSA_F32)
+    CSA_LAUNCH(KK_GEMM, st, gemm_nt_simt<float><<<grid, 256, 0, st>>>(
+        (const float*)H, (const float*)packed, P, M, L.ncols, d));
+  else
+    CSA_LAUNCH(KK_GEMM, st, gemm_nt_simt<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16*)H, (const __nv_bfloat16*)packed, P, M, L.ncols, d));
+  const float* bias = (const float*)((const char*)packed + L.bias_off);
+  const int nE = T / p.m;
+  if (p.act == CSA_F32) {
+    if (p.kv == CSA_F32)
+      launch_fold<float, CSA_F32>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    else if (p.kv == CSA_BF16)
+      launch_fold<float, CSA_BF16>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    else
+      launch_fold<float, CSA_KV_FP8MIX>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+  } else {
+    if (p.kv == CSA_F32)
+      launch_fold<__nv_bfloat16, CSA_F32>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    else if (p.kv == CSA_BF16)
+      launch_fold<__nv_bfloat16, CSA_BF16>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    else
+      launch_fold<__nv_bfloat16, CSA_KV_FP8MIX>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+  }
+  return last_launch_status();
+}
+
+}  // namespace csa

@@ -1,0 +1,50 @@
+// kernels.h -- host-side launchers of the CSA / HCA kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+// Packed compressor weights: [ncols][d] act dtype (K-major rows, one per GEMM
+// output column), then fp32 biases [m][nb] at bias_off.
+struct PackLayout {
+  int ncols = 0;
+  int col_Ca = -1, col_Cb = -1, col_Za = -1, col_Zb = -1;
+  int col_CIa = -1, col_CIb = -1, col_ZIa = -1, col_ZIb = -1;
+  int nb = 0;
+  int b_Ba = -1, b_Bb = -1, b_BIa = -1, b_BIb = -1;
+  size_t bias_off = 0;
+  size_t total = 0;
+};
+PackLayout pack_layout(const csa_params& p, int d);
+
+csa_status launch_pack(const csa_params& p, int d, const void* const W[8],
+                       const float* const Bias[4], void* packed, cudaStream_t st);
+
+size_t compress_ws_bytes(const csa_params& p, int B, int T, int d);
+csa_status launch_compress(const csa_params& p, int B, int T, int d,
+                           const void* H, const void* packed, void* ckv,
+                           float* ckv_scale, void* kI, void* win,
+                           float* win_scale, void* ws, cudaStream_t st);
+
+size_t index_topk_ws_bytes(const csa_params& p, int B, int Q, int N);
+csa_status launch_index_topk(const csa_params& p, int B, int Q,
+                             const int32_t* q_pos, const void* qI,
+                             const float* w, const void* kI, int N,
+                             int32_t* idx_out, float* score_out, void* ws,
+                             cudaStream_t st);
+
+size_t attend_ws_bytes(const csa_params& p, int B, int Q, int N, bool dense);
+csa_status launch_attend(const csa_params& p, bool dense, int B, int Q,
+                         const int32_t* q_pos, const void* q,
+                         const int32_t* idx, const void* ckv,
+                         const float* ckv_scale, int N, const void* win,
+                         const float* win_scale, int W,
+                         const int32_t* win_pos0, const float* sink, void* out,
+                         void* ws, cudaStream_t st);
+
+}  // namespace csa

@@ -1,0 +1,109 @@
+"""Helpers shared by the GPU parity tests: buffer allocation in the library's
+layouts, conversion of stored values to float64, and the comparison rules.
+
+Comparison rules (what "parity" means here):
+* fp outputs: bf16 / FP8 paths: max-abs <= 2e-2 and rel-L2 <= 5e-3 against
+  the fp64 oracle; fp32 path: max-abs <= 1e-5.
+* indexer scores: |gpu - oracle| <= tol, tol derived from fp32 accumulation
+  of c_I products per head and n_hI heads: 4 (c_I + n_hI) 2^-24
+  (sum_h |w_h| |q_h|) . |K_s| (factor 4 of margin over the first-order bound).
+* top-k sets: equal, except that an index selected by only one side must have
+  an oracle score within the two sides' tolerance of the oracle's k-th
+  score (a tie at fp32 resolution); output ascending, -1 padded, visible.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from oracle import pipeline as P
+
+DEV = "cuda"
+U32 = 2.0 ** -24
+
+
+def row_bytes(wl) -> int:
+    if wl.kv == "f32":
+        return 4 * wl.c
+    if wl.kv == "bf16":
+        return 2 * wl.c
+    return (wl.c - wl.rope_dims) + 2 * wl.rope_dims
+
+
+def alloc_kv(wl, lead: tuple, rows: int, device=DEV):
+    """Empty cache rows in the workload's KV format: (rec, scale or None)."""
+    if wl.kv == "f32":
+        return torch.empty(lead + (rows, wl.c), dtype=torch.float32, device=device), None
+    if wl.kv == "bf16":
+        return torch.empty(lead + (rows, wl.c), dtype=torch.bfloat16, device=device), None
+    rec = torch.empty(lead + (rows, row_bytes(wl)), dtype=torch.uint8, device=device)
+    return rec, torch.empty(lead + (rows,), dtype=torch.float32, device=device)
+
+
+def kv_values(wl, rec, scale) -> np.ndarray:
+    return P.cache_values(rec, scale, wl.kv, wl.c, wl.rope_dims)
+
+
+def act_dtype(wl):
+    return torch.float32 if wl.act == "f32" else torch.bfloat16
+
+
+def to_dev(d: dict) -> dict:
+    return {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in d.items()}
+
+
+def assert_close(got, ref, fmt: str, what: str = ""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    if fmt == "f32":
+        assert err.max() <= 1e-5, f"{what}: max-abs {err.max():.3g} > 1e-5"
+    else:
+        rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+        assert err.max() <= 2e-2, f"{what}: max-abs {err.max():.3g} > 2e-2"
+        assert rel <= 5e-3, f"{what}: rel-L2 {rel:.3g} > 5e-3"
+
+
+def score_tolerance(qI, w, kI) -> np.ndarray:
+    """Per (query, entry) bound on the fp32 accumulation error of eq. 16."""
+    qI = np.abs(np.asarray(qI, dtype=np.float64))
+    w = np.abs(np.asarray(w, dtype=np.float64))
+    K = np.abs(np.asarray(kI, dtype=np.float64))
+    n_hI, c_I = qI.shape[1], qI.shape[2]
+    comb = np.einsum("qh,qhe->qe", w, qI)
+    return 4.0 * (c_I + n_hI) * U32 * (comb @ K.T) + 1e-30
+
+
+def check_topk(idx_gpu, score_gpu, scores_ref, nv, k, tol, what=""):
+    """Check GPU idx/scores of several queries against oracle scores."""
+    idx_gpu = np.asarray(idx_gpu)
+    for q in range(idx_gpu.shape[0]):
+        n = int(nv[q])
+        keep = min(k, n)
+        row = idx_gpu[q]
+        sel = row[:keep]
+        assert np.all(row[keep:] == -1), f"{what} q{q}: padding"
+        assert np.all(np.diff(sel) > 0), f"{what} q{q}: not ascending/unique"
+        assert keep == 0 or (sel[0] >= 0 and sel[-1] < n), f"{what} q{q}: out of range"
+        if score_gpu is not None and keep:
+            sg = np.asarray(score_gpu[q][:keep], dtype=np.float64)
+            bad = np.abs(sg - scores_ref[q, sel]) > tol[q, sel]
+            assert not bad.any(), f"{what} q{q}: score mismatch at {sel[bad][:5]}"
+        if keep == 0:
+            continue
+        ref_idx, kth = oracle.topk(scores_ref[q: q + 1], np.array([n], np.int32), k)
+        ref_sel = ref_idx[0][:keep]
+        only_g = np.setdiff1d(sel, ref_sel)
+        only_o = np.setdiff1d(ref_sel, sel)
+        assert len(only_g) == len(only_o)
+        if len(only_g):
+            # a swap needs gpu(s_g) >= gpu(s_o) while oracle(s_g) <= kth <=
+            # oracle(s_o): both lie within tol(s_g) + tol(s_o) of kth
+            diff = np.concatenate([only_g, only_o])
+            band = 2.0 * tol[q, diff].max()
+            for s in diff:
+                assert abs(scores_ref[q, s] - kth[0]) <= band, (
+                    f"{what} q{q}: index {s} differs beyond the fp32 tie band")
