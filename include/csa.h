@@ -155,6 +155,29 @@ csa_status csa_index_topk(const csa_params* p, int B, int Q,
                           float* score_out, void* workspace, size_t ws_bytes,
                           csa_stream_t stream);
 
+/* csa_index_topk_noalloc: csa_index_topk for callers that cannot allocate
+ * device memory or pass a workspace -- e.g. plugins of a host framework that
+ * owns all device memory, or latency-critical loops where an allocation would
+ * synchronise the device.  The pages have no counterpart: this is a library
+ * convenience, not part of the method.
+ *   Same arguments and results as csa_index_topk, without the workspace.
+ *   The scratch is one fixed 16 MiB device array inside the library (enough
+ *   for B*Q*N <= 4,194,304 scores); it occupies that memory on every GPU
+ *   that loads the library until the process exits.  A request that needs
+ *   more returns CSA_ERR_WORKSPACE before anything is launched.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call on a device shares the same array: calls whose kernels can
+ *   overlap on the GPU (different streams without ordering between them)
+ *   race on it and give undefined results.  Nothing in it needs to start at
+ *   zero; it keeps the last call's contents.
+ *   Calls no cudaMalloc, cudaFree or other allocating routine. */
+csa_status csa_index_topk_noalloc(const csa_params* p, int B, int Q,
+                                  const int32_t* q_pos, const void* qI,
+                                  const float* w, const void* kI, int N,
+                                  int32_t* idx_out, float* score_out,
+                                  csa_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * csa_attend: shared-KV multi-query attention of each query over its
  * selected entries and its last n_win tokens, in ONE softmax whose

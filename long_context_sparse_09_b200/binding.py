@@ -62,6 +62,7 @@ _SIGS = {
     "hca_compress": (C.c_int, [_P, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "csa_index_topk_noalloc": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
     "csa_attend_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_attend": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp,
                              _vp, _vp, _sz, _vp]),
@@ -198,6 +199,17 @@ def csa_index_topk(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out=None,
     st = lib().csa_index_topk(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI), N,
                               _p(idx_out), _p(score_out), _p(ws), wsb, _stream(stream))
     _check("csa_index_topk", st)
+
+
+def csa_index_topk_noalloc(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out=None,
+                           stream=None):
+    """csa_index_topk with the library's fixed scratch instead of a
+    workspace (for callers that cannot allocate device memory)."""
+    B, N = kI.shape[0], kI.shape[1]
+    Q = qI.shape[0] // B
+    st = lib().csa_index_topk_noalloc(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI), N,
+                                      _p(idx_out), _p(score_out), _stream(stream))
+    _check("csa_index_topk_noalloc", st)
 
 
 # ---------------------------------------------------------------- attend --
