@@ -48,9 +48,10 @@ void prof_end(int slot, cudaStream_t st) {
   if (slot < (int)g_prof_recs.size()) cudaEventRecord(g_prof_recs[slot].b, st);
 }
 
-static const char* kKindNames[KK_COUNT] = {"pack_weights", "compress_gemm", "compress_fold",
-                                           "compress_window", "index_scores", "topk_select",
-                                           "attend", "attend_combine"};
+static const char* kKindNames[KK_COUNT] = {
+    "pack_weights", "compress_gemm", "compress_fold", "compress_window", "index_scores",
+    "topk_radix", "attend", "attend_combine", "index_plan", "topk_hist", "topk_select",
+    "topk_final"};
 
 unsigned int* device_error_word() {
   // cudaGetSymbolAddress is per device; cache one address per device index.

@@ -1,0 +1,363 @@
+// index_tc.cu -- Lightning-Indexer scores on the 5th-generation tensor cores
+// ("DeepSeekV4技术报告阅读笔记" eq. 16; "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文"
+// section 2.2).
+//
+// One product per (entry tile, query group): D[128 entries][G*n_hI] =
+// K^I_tile[128][c_I] * Q_group[G*n_hI][c_I]^T, bf16 in, fp32 in TMEM.  The
+// entries are the MMA's M dimension so that each TMEM lane -- one epilogue
+// thread -- holds one entry's dot products with every head of the group's
+// queries; ReLU, the head weights w and the sum over heads then run in
+// registers with no cross-thread reduction.
+//
+// Warp roles (per CTA): warp 0 issues TMA loads of K^I tiles (and of the
+// query group's q^I when it changes), warp 1 allocates TMEM and issues the
+// MMAs, the remaining warps drain TMEM, apply the score epilogue and store
+// fp32 scores.  K^I tiles go through a ring of smem stages, accumulators
+// through two TMEM buffers, so loads, MMAs and epilogues overlap.  Every
+// wait is bounded; a timeout sets CSA_DEV_TIMEOUT and the CTA winds down.
+//
+// Work: the flat list of (query group, entry tile) pairs over each group's
+// visible tiles (a plan kernel computes per-group tile counts and their
+// prefix sum on the device), split evenly over a persistent grid.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace csa {
+
+using namespace sm100;
+
+struct IdxTcArgs {
+  const int32_t* q_pos;
+  const float* w;
+  const int* prefix;  // [ngroups + 1] exclusive prefix of tiles per group
+  float* scores;      // [R][N]
+  unsigned* err;
+  int Q, N, m, nhI, ngroups;
+};
+
+constexpr int kTileM = 128;
+constexpr int kKBlockBytes = kTileM * 128;  // 128 rows x 64 bf16
+
+template <int G, int KB, int S, int NE>
+struct IdxTcCfg {
+  static constexpr int kStageBytes = KB * kKBlockBytes;
+  static constexpr int kThreads = 64 + 32 * NE;
+};
+
+// Per-group visible tile counts and their exclusive prefix (one CTA).
+__global__ void __launch_bounds__(1024) index_plan(const int32_t* __restrict__ q_pos, int G,
+                                                   int ngroups, int m, int N,
+                                                   int* __restrict__ prefix) {
+  __shared__ unsigned sh[33];
+  unsigned running = 0;
+  for (int base = 0; base < ngroups; base += blockDim.x) {
+    const int g = base + threadIdx.x;
+    unsigned tiles = 0;
+    if (g < ngroups) {
+      int nv = 0;
+      for (int i = 0; i < G; ++i) nv = max(nv, n_visible(q_pos[g * G + i], m, N));
+      tiles = (unsigned)((nv + kTileM - 1) / kTileM);
+    }
+    unsigned total;
+    unsigned ex = block_exclusive_scan(tiles, sh, &total);
+    if (g < ngroups) prefix[g] = (int)(running + ex);
+    running += total;
+  }
+  if (threadIdx.x == 0) prefix[ngroups] = (int)running;
+}
+
+// Walk of a CTA over its slice of the flat (group, tile) list.
+struct TileCursor {
+  int g, t, left;
+  __device__ void init(const int* prefix, int ngroups, int start, int count) {
+    int lo = 0, hi = ngroups;
+    while (lo < hi) {  // last g with prefix[g] <= start
+      int mid = (lo + hi + 1) >> 1;
+      if (__ldg(prefix + mid) <= start) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    t = start - __ldg(prefix + g);
+    left = count;
+  }
+  __device__ int tiles(const int* prefix) const { return __ldg(prefix + g + 1) - __ldg(prefix + g); }
+  __device__ bool first(int pos_in_cta) const { return t == 0 || pos_in_cta == 0; }
+  __device__ bool last(const int* prefix) const { return left == 1 || t + 1 == tiles(prefix); }
+  __device__ void next(const int* prefix, int ngroups) {
+    --left;
+    if (++t >= tiles(prefix)) {
+      t = 0;
+      do { ++g; } while (g < ngroups && __ldg(prefix + g + 1) == __ldg(prefix + g));
+    }
+  }
+};
+
+template <int G, int KB, int S, int NE>
+__global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
+    index_scores_tc(const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmQ, IdxTcArgs a) {
+  using Cfg = IdxTcCfg<G, KB, S, NE>;
+  const int NROWS = G * a.nhI;  // MMA N: the group's query heads
+  const int NCOL = NROWS;       // TMEM columns per accumulator
+  const int qslot_bytes = KB * NROWS * 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* kst = smem;                                  // S stages
+  uint8_t* qsl = kst + S * Cfg::kStageBytes;            // 2 query slots
+  uint64_t* bars = (uint64_t*)(qsl + 2 * qslot_bytes);  // barriers
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + S;
+  uint64_t* qfull = bars + 2 * S;
+  uint64_t* qempty = qfull + 2;
+  uint64_t* tfull = qempty + 2;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tbase_sm = (uint32_t*)(tempty + 2);
+  volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int ncols_alloc = 32;
+  while (ncols_alloc < 2 * NCOL) ncols_alloc <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 1);
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], NE);
+    }
+    *abort_sm = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tbase_sm, ncols_alloc);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmQ);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tbase_sm;
+
+  const int total = __ldg(a.prefix + a.ngroups);
+  const int start = (int)((long long)total * blockIdx.x / gridDim.x);
+  const int count = (int)((long long)total * (blockIdx.x + 1) / gridDim.x) - start;
+
+  if (count > 0) {
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------- producer --
+      TileCursor cur;
+      cur.init(a.prefix, a.ngroups, start, count);
+      int kn = 0, qn = 0;
+      for (int i = 0; i < count; ++i) {
+        if (cur.first(i)) {
+          const int slot = qn & 1;
+          if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_sm)) break;
+          mbar_expect_tx(&qfull[slot], (uint32_t)qslot_bytes);
+          uint8_t* dst = qsl + slot * qslot_bytes;
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(dst + kb * NROWS * 128, &tmQ, &qfull[slot], kb * 64,
+                        cur.g * G * a.nhI);
+          ++qn;
+        }
+        const int s = kn % S;
+        if (!mbar_wait(&kempty[s], ((kn / S) & 1) ^ 1, abort_sm)) break;
+        mbar_expect_tx(&kfull[s], (uint32_t)Cfg::kStageBytes);
+        const int b = (cur.g * G) / a.Q;
+        const int row = b * a.N + cur.t * kTileM;
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_2d(kst + s * Cfg::kStageBytes + kb * kKBlockBytes, &tmK, &kfull[s], kb * 64,
+                      row);
+        ++kn;
+        cur.next(a.prefix, a.ngroups);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA --
+      TileCursor cur;
+      cur.init(a.prefix, a.ngroups, start, count);
+      const uint32_t idesc = idesc_bf16(kTileM, NROWS);
+      int kn = 0, qn = 0, an = 0;
+      for (int i = 0; i < count; ++i) {
+        const bool first = cur.first(i), last = cur.last(a.prefix);
+        const int slot = qn & 1;
+        if (first && !mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_sm)) break;
+        const int s = kn % S;
+        if (!mbar_wait(&kfull[s], (kn / S) & 1, abort_sm)) break;
+        const int acc = an & 1;
+        if (!mbar_wait(&tempty[acc], ((an >> 1) & 1) ^ 1, abort_sm)) break;
+        tc_fence_after();
+        const uint32_t abase = smem_u32(kst + s * Cfg::kStageBytes);
+        const uint32_t bbase = smem_u32(qsl + slot * qslot_bytes);
+        const uint32_t d = tbase + acc * NCOL;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_bf16(d, sdesc_k_sw128(abase + kb * kKBlockBytes + j * 32),
+                     sdesc_k_sw128(bbase + kb * NROWS * 128 + j * 32), idesc,
+                     (kb | j) != 0);
+        mma_commit(&kempty[s]);
+        mma_commit(&tfull[acc]);
+        if (last) {
+          mma_commit(&qempty[slot]);
+          ++qn;
+        }
+        ++kn;
+        ++an;
+        cur.next(a.prefix, a.ngroups);
+      }
+    } else if (warp >= 2) {
+      // ------------------------------------------------------- epilogue --
+      const int e = warp - 2;
+      const int quad = warp & 3;         // TMEM lane quadrant of this warp
+      const int nq_mine = NE == 4 ? G : G / 2;
+      const int q0 = NE == 4 ? 0 : (e >> 2) * (G / 2);
+      TileCursor cur;
+      cur.init(a.prefix, a.ngroups, start, count);
+      int an = 0;
+      for (int i = 0; i < count; ++i) {
+        const int acc = an & 1;
+        if (!mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm)) break;
+        tc_fence_after();
+        const int s = cur.t * kTileM + quad * 32 + lane;
+        float sc[G];
+#pragma unroll
+        for (int qi = 0; qi < G; ++qi) sc[qi] = 0.f;
+        const uint32_t trow = tbase + ((uint32_t)(quad * 32) << 16) + acc * NCOL;
+        for (int qq = 0; qq < nq_mine; ++qq) {
+          const int qi = q0 + qq;
+          const float* wr = a.w + (size_t)(cur.g * G + qi) * a.nhI;
+          float acc_s = 0.f;
+          for (int c0 = 0; c0 < a.nhI; c0 += 16) {
+            float v[16];
+            tmem_ld16(trow + qi * a.nhI + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc_s = fmaf(__ldg(wr + c0 + j), fmaxf(v[j], 0.f), acc_s);
+          }
+          sc[qq] = acc_s;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        for (int qq = 0; qq < nq_mine; ++qq) {
+          const int r = cur.g * G + q0 + qq;
+          const int nv = n_visible(__ldg(a.q_pos + r), a.m, a.N);
+          if (s < nv) a.scores[(size_t)r * a.N + s] = sc[qq];
+        }
+        ++an;
+        cur.next(a.prefix, a.ngroups);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_sm) {
+    if (threadIdx.x == 0) atomicOr(a.err, CSA_DEV_TIMEOUT);
+    // let tensor-core work already issued drain before TMEM is released
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+  }
+  if (warp == 1) tmem_dealloc(tbase, ncols_alloc);
+}
+
+// ------------------------------------------------------------------ host --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), boxes of 64 x box_rows with
+// the 128-byte swizzle.
+static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool index_tc_supported(const csa_params& p) {
+  return p.act == CSA_BF16 && (p.c_I == 64 || p.c_I == 128) && p.n_hI % 16 == 0 &&
+         p.n_hI <= 64 && encode_fn() != nullptr;
+}
+
+int index_tc_group(const csa_params& p, int Q) {
+  int G = 1;
+  for (int g : {4, 2})
+    if (Q % g == 0 && g * p.n_hI <= 256) { G = g; break; }
+  return G;
+}
+
+size_t index_tc_plan_bytes(int ngroups) { return align_up((size_t)(ngroups + 1) * 4, 256); }
+
+template <int G, int KB, int S, int NE>
+static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
+                              const IdxTcArgs& a, cudaStream_t st) {
+  using Cfg = IdxTcCfg<G, KB, S, NE>;
+  const int NROWS = G * a.nhI;
+  size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + 2 * (size_t)KB * NROWS * 128 + 256;
+  auto kern = index_scores_tc<G, KB, S, NE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
+  int dev = 0, sms = 0, occ = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
+  if (occ < 1) return CSA_ERR_UNSUPPORTED;
+  const int grid = sms * occ;
+  CSA_LAUNCH(KK_SCORES, st, kern<<<grid, Cfg::kThreads, smem, st>>>(tmK, tmQ, a));
+  return last_launch_status();
+}
+
+csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32_t* q_pos,
+                                  const void* qI, const float* w, const void* kI, int N,
+                                  float* scores, int* plan, cudaStream_t st) {
+  const int R = B * Q;
+  const int G = index_tc_group(p, Q);
+  const int ngroups = R / G;
+  CSA_LAUNCH(KK_PLAN, st, index_plan<<<1, 1024, 0, st>>>(q_pos, G, ngroups, p.m, N, plan));
+  if (N == 0) return last_launch_status();
+  CUtensorMap tmK, tmQ;
+  if (!make_tmap_bf16(&tmK, kI, (uint64_t)B * N, p.c_I, kTileM)) return CSA_ERR_CUDA;
+  if (!make_tmap_bf16(&tmQ, qI, (uint64_t)R * p.n_hI, p.c_I, G * p.n_hI)) return CSA_ERR_CUDA;
+  IdxTcArgs a{q_pos, w, plan, scores, device_error_word(), Q, N, p.m, p.n_hI, ngroups};
+  if (a.err == nullptr) return CSA_ERR_CUDA;
+  const bool k2 = p.c_I == 128;
+  if (G == 1) return k2 ? launch_tc_t<1, 2, 5, 4>(tmK, tmQ, a, st) : launch_tc_t<1, 1, 8, 4>(tmK, tmQ, a, st);
+  if (G == 2) return k2 ? launch_tc_t<2, 2, 4, 4>(tmK, tmQ, a, st) : launch_tc_t<2, 1, 6, 4>(tmK, tmQ, a, st);
+  return k2 ? launch_tc_t<4, 2, 2, 8>(tmK, tmQ, a, st) : launch_tc_t<4, 1, 4, 8>(tmK, tmQ, a, st);
+}
+
+}  // namespace csa

@@ -69,29 +69,21 @@ __global__ void __launch_bounds__(256) index_scores_simt(
 }
 
 // ------------------------------------------------------------ radix top-k --
-// One 1024-thread CTA per query.  Three digit passes (11, 11, 10 bits) over
-// the order-preserving keys find the k-th largest key K; the output takes
-// every entry with key > K and the lowest-index entries with key == K.
+// Block-wide exact top-k of one query's scores sc[0..nv) (nv > k), 1024
+// threads.  Three digit passes (11, 11, 10 bits) over the order-preserving
+// keys find the k-th largest key K; the output takes every entry with key > K
+// and the lowest-index entries with key == K, in ascending index order.
 constexpr int kTopkThreads = 1024;
 
-__global__ void __launch_bounds__(kTopkThreads) topk_radix(
-    const float* __restrict__ scores, int N, const int32_t* __restrict__ q_pos,
-    int m, int k, int32_t* __restrict__ idx_out, float* __restrict__ score_out) {
-  __shared__ unsigned hist[2048];
-  __shared__ unsigned scan_sh[33];
-  __shared__ unsigned s_digit, s_remaining;
-  const int r = blockIdx.x;
-  const int nv = n_visible(q_pos[r], m, N);
-  const float* sc = scores + (size_t)r * N;
-  int32_t* out = idx_out + (size_t)r * k;
-  float* sout = score_out ? score_out + (size_t)r * k : nullptr;
-  if (nv <= k) {
-    for (int j = threadIdx.x; j < k; j += blockDim.x) {
-      out[j] = j < nv ? j : -1;
-      if (sout) sout[j] = j < nv ? sc[j] : -INFINITY;
-    }
-    return;
-  }
+struct RadixShared {
+  unsigned hist[2048];
+  unsigned scan[33];
+  unsigned digit, remaining;
+};
+
+__device__ void radix_select_block(const float* __restrict__ sc, int nv, int k,
+                                   int32_t* __restrict__ out, float* __restrict__ sout,
+                                   RadixShared& sh) {
   unsigned prefix = 0, mask = 0;
   unsigned remaining = (unsigned)k;  // rank of the wanted key among those matching prefix
   const int shifts[3] = {21, 10, 0};
@@ -99,35 +91,32 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = shifts[pass];
     const unsigned dmask = (1u << widths[pass]) - 1u;
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sh.hist[i] = 0;
     __syncthreads();
     for (int s = threadIdx.x; s < nv; s += blockDim.x) {
       unsigned key = score_key(sc[s]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+      if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & dmask], 1u);
     }
     __syncthreads();
-    // suffix sums: thread t owns bins 2t and 2t+1; scan in descending order
-    const int t = threadIdx.x;
-    const int rt = kTopkThreads - 1 - t;  // rt-th thread holds bins 2rt, 2rt+1
-    unsigned h_hi = hist[2 * rt + 1], h_lo = hist[2 * rt];
+    // thread t owns bins 2rt, 2rt+1 with rt = 1023 - t, so the exclusive scan
+    // over t counts the keys in higher bins
+    const int rt = kTopkThreads - 1 - threadIdx.x;
+    unsigned h_hi = sh.hist[2 * rt + 1], h_lo = sh.hist[2 * rt];
     unsigned total;
-    unsigned above = block_exclusive_scan(h_hi + h_lo, scan_sh, &total);
-    // `above` = keys in bins > 2rt+1
+    unsigned above = block_exclusive_scan(h_hi + h_lo, sh.scan, &total);
     if (above < remaining && above + h_hi >= remaining) {
-      s_digit = 2 * rt + 1;
-      s_remaining = remaining - above;
+      sh.digit = 2 * rt + 1;
+      sh.remaining = remaining - above;
     } else if (above + h_hi < remaining && above + h_hi + h_lo >= remaining) {
-      s_digit = 2 * rt;
-      s_remaining = remaining - above - h_hi;
+      sh.digit = 2 * rt;
+      sh.remaining = remaining - above - h_hi;
     }
     __syncthreads();
-    prefix |= s_digit << shift;
+    prefix |= sh.digit << shift;
     mask |= dmask << shift;
-    remaining = s_remaining;
+    remaining = sh.remaining;
     __syncthreads();
   }
-  // prefix = K (exact key of the k-th largest); `remaining` keys equal to K
-  // are taken, lowest index first.
   const unsigned K = prefix;
   unsigned eq_before = 0, sel_before = 0;
   for (int base = 0; base < nv; base += blockDim.x) {
@@ -136,9 +125,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
     bool gt = s < nv && key > K;
     bool eq = s < nv && key == K;
     unsigned eq_tot, sel_tot;
-    unsigned eq_rank = block_exclusive_scan(eq ? 1u : 0u, scan_sh, &eq_tot);
+    unsigned eq_rank = block_exclusive_scan(eq ? 1u : 0u, sh.scan, &eq_tot);
     bool sel = gt || (eq && eq_before + eq_rank < remaining);
-    unsigned pos = block_exclusive_scan(sel ? 1u : 0u, scan_sh, &sel_tot);
+    unsigned pos = block_exclusive_scan(sel ? 1u : 0u, sh.scan, &sel_tot);
     if (sel) {
       out[sel_before + pos] = s;
       if (sout) sout[sel_before + pos] = sc[s];
@@ -148,8 +137,247 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
   }
 }
 
+__device__ __forceinline__ void write_all_visible(const float* sc, int nv, int k, int32_t* out,
+                                                  float* sout) {
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    out[j] = j < nv ? j : -1;
+    if (sout) sout[j] = j < nv ? sc[j] : -INFINITY;
+  }
+}
+
+// One CTA per query (used when there are many queries).
+__global__ void __launch_bounds__(kTopkThreads) topk_radix(
+    const float* __restrict__ scores, int N, const int32_t* __restrict__ q_pos,
+    int m, int k, int32_t* __restrict__ idx_out, float* __restrict__ score_out) {
+  __shared__ RadixShared sh;
+  const int r = blockIdx.x;
+  const int nv = n_visible(q_pos[r], m, N);
+  const float* sc = scores + (size_t)r * N;
+  int32_t* out = idx_out + (size_t)r * k;
+  float* sout = score_out ? score_out + (size_t)r * k : nullptr;
+  if (nv <= k) {
+    write_all_visible(sc, nv, k, out, sout);
+    return;
+  }
+  radix_select_block(sc, nv, k, out, sout, sh);
+}
+
+// ------------------------------------------------- multi-CTA top-k (few q) --
+// For a handful of queries with long visible ranges (decode): (1) every CTA
+// histograms the top 12 key bits of a chunk, (2) every CTA finds the bin T
+// that holds the k-th largest key, marks the entries of higher bins in a
+// bitmap and lists the entries of bin T as candidates, (3) one CTA per query
+// orders the candidates (key desc, index asc), marks the ones still needed
+// and compacts the bitmap into ascending indices.  If bin T overflows the
+// candidate list, (3) falls back to the exact block-wide radix select.
+constexpr int kBins = 4096;
+constexpr int kChunk = 8192;    // entries per CTA in (1) and (2)
+constexpr int kCandCap = 4096;  // candidates per query
+
+struct MultiTopkWs {
+  unsigned* ghist;     // [R][kBins]
+  unsigned* cand_cnt;  // [R]
+  unsigned* bitmap;    // [R][N32]
+  uint2* cand;         // [R][kCandCap] (key, index)
+};
+
+__global__ void __launch_bounds__(1024) topk_hist(const float* __restrict__ scores, int N,
+                                                  const int32_t* __restrict__ q_pos, int m,
+                                                  int k, unsigned* __restrict__ ghist) {
+  __shared__ unsigned h[kBins];
+  const int r = blockIdx.x;
+  const int nv = n_visible(q_pos[r], m, N);
+  if (nv <= k) return;
+  const int s0 = blockIdx.y * kChunk;
+  if (s0 >= nv) return;
+  const int s1 = min(nv, s0 + kChunk);
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const float* sc = scores + (size_t)r * N;
+  for (int s = s0 + threadIdx.x; s < s1; s += blockDim.x) atomicAdd(&h[score_key(sc[s]) >> 20], 1u);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x)
+    if (h[i]) atomicAdd(&ghist[(size_t)r * kBins + i], h[i]);
+}
+
+// Bin holding the k-th largest key and the number of keys in higher bins
+// (1024 threads, 4 bins each).
+__device__ void find_threshold_bin(const unsigned* __restrict__ gh, unsigned k, unsigned* scan,
+                                   int* T_out, unsigned* above_out, int* sT, unsigned* sAbove) {
+  const int rt = 1023 - (int)threadIdx.x;  // bins 4rt .. 4rt+3
+  unsigned c[4];
+  unsigned sum = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    c[j] = __ldcg(gh + 4 * rt + j);
+    sum += c[j];
+  }
+  unsigned total;
+  unsigned above = block_exclusive_scan(sum, scan, &total);
+#pragma unroll
+  for (int j = 3; j >= 0; --j) {
+    if (above < k && above + c[j] >= k) {
+      *sT = 4 * rt + j;
+      *sAbove = above;
+    }
+    above += c[j];
+  }
+  __syncthreads();
+  *T_out = *sT;
+  *above_out = *sAbove;
+}
+
+__global__ void __launch_bounds__(1024) topk_select(const float* __restrict__ scores, int N,
+                                                    const int32_t* __restrict__ q_pos, int m,
+                                                    int k, MultiTopkWs ws) {
+  __shared__ unsigned scan[33];
+  __shared__ int sT;
+  __shared__ unsigned sAbove;
+  const int r = blockIdx.x;
+  const int nv = n_visible(q_pos[r], m, N);
+  if (nv <= k) return;
+  const int s0 = blockIdx.y * kChunk;
+  if (s0 >= N) return;
+  int T;
+  unsigned above;
+  find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, scan, &T, &above, &sT, &sAbove);
+  const int N32 = (N + 31) >> 5;
+  const float* sc = scores + (size_t)r * N;
+  const int s1 = min(N, s0 + kChunk);
+  for (int base = s0; base < s1; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    const bool vis = s < nv && s < s1;
+    const unsigned key = vis ? score_key(sc[s]) : 0u;
+    const int bin = (int)(key >> 20);
+    const bool gt = vis && bin > T;
+    const bool eq = vis && bin == T;
+    const unsigned word = __ballot_sync(0xffffffffu, gt);
+    if ((threadIdx.x & 31) == 0 && (s >> 5) < N32 && s < s1) ws.bitmap[(size_t)r * N32 + (s >> 5)] = word;
+    if (eq) {
+      unsigned pos = atomicAdd(&ws.cand_cnt[r], 1u);
+      if (pos < kCandCap) ws.cand[(size_t)r * kCandCap + pos] = make_uint2(key, (unsigned)s);
+    }
+  }
+}
+
+__device__ __forceinline__ bool cand_before(uint2 x, uint2 y) {
+  return x.x > y.x || (x.x == y.x && x.y < y.y);
+}
+
+__global__ void __launch_bounds__(1024) topk_finalize(const float* __restrict__ scores, int N,
+                                                      const int32_t* __restrict__ q_pos, int m,
+                                                      int k, MultiTopkWs ws,
+                                                      int32_t* __restrict__ idx_out,
+                                                      float* __restrict__ score_out) {
+  __shared__ uint2 cand[kCandCap];
+  __shared__ RadixShared sh;
+  __shared__ int sT;
+  __shared__ unsigned sAbove;
+  const int r = blockIdx.x;
+  const int nv = n_visible(q_pos[r], m, N);
+  const float* sc = scores + (size_t)r * N;
+  int32_t* out = idx_out + (size_t)r * k;
+  float* sout = score_out ? score_out + (size_t)r * k : nullptr;
+  if (nv <= k) {
+    write_all_visible(sc, nv, k, out, sout);
+    return;
+  }
+  int T;
+  unsigned above;
+  find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, &sT, &sAbove);
+  const unsigned nc = __ldcg(ws.cand_cnt + r);
+  if (nc > (unsigned)kCandCap) {  // bin T too crowded: exact block-wide select
+    radix_select_block(sc, nv, k, out, sout, sh);
+    return;
+  }
+  const unsigned need = (unsigned)k - above;
+  int P = 1;
+  while (P < (int)nc) P <<= 1;
+  for (int i = threadIdx.x; i < P; i += blockDim.x)
+    cand[i] = i < (int)nc ? __ldcg(ws.cand + (size_t)r * kCandCap + i) : make_uint2(0u, 0x7fffffffu);
+  __syncthreads();
+  // bitonic sort into (key descending, index ascending)
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
+        const int lo = 2 * stride * (i / stride) + (i % stride);
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint2 x = cand[lo], y = cand[hi];
+        if (up ? cand_before(y, x) : cand_before(x, y)) {
+          cand[lo] = y;
+          cand[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int N32 = (N + 31) >> 5;
+  unsigned* bm = ws.bitmap + (size_t)r * N32;
+  for (unsigned i = threadIdx.x; i < need; i += blockDim.x) {
+    const unsigned s = cand[i].y;
+    atomicOr(bm + (s >> 5), 1u << (s & 31));
+  }
+  __threadfence();
+  __syncthreads();
+  // ordered compaction of the bitmap
+  const int per = (N32 + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * per, w1 = min(N32, w0 + per);
+  unsigned cnt = 0;
+  for (int wi = w0; wi < w1; ++wi) cnt += __popc(__ldcg(bm + wi));
+  unsigned tot;
+  unsigned pos = block_exclusive_scan(cnt, sh.scan, &tot);
+  for (int wi = w0; wi < w1; ++wi) {
+    unsigned word = __ldcg(bm + wi);
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      const int s = wi * 32 + bit;
+      if (pos < (unsigned)k) {
+        out[pos] = s;
+        if (sout) sout[pos] = sc[s];
+      }
+      ++pos;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host --
+bool index_tc_supported(const csa_params& p);
+int index_tc_group(const csa_params& p, int Q);
+size_t index_tc_plan_bytes(int ngroups);
+csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32_t* q_pos,
+                                  const void* qI, const float* w, const void* kI, int N,
+                                  float* scores, int* plan, cudaStream_t st);
+
+static bool use_multi_topk(int R, int N) { return R <= 64 && N >= 4096; }
+
+struct IdxWsLayout {
+  size_t scores = 0, plan = 0, ghist = 0, cand_cnt = 0, bitmap = 0, cand = 0, total = 0;
+};
+
+static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
+  IdxWsLayout L;
+  const size_t R = (size_t)B * Q;
+  size_t off = align_up(R * N * sizeof(float), 256);
+  L.plan = off;
+  off += align_up((R + 1) * sizeof(int), 256);
+  if (use_multi_topk((int)R, N)) {
+    L.ghist = off;
+    off += R * kBins * 4;
+    L.cand_cnt = off;
+    off = align_up(off + R * 4, 256);
+    L.bitmap = off;
+    off += align_up(R * ((N + 31) / 32) * 4, 256);
+    L.cand = off;
+    off += align_up(R * kCandCap * sizeof(uint2), 256);
+  }
+  L.total = off;
+  return L;
+}
+
 size_t index_topk_ws_bytes(const csa_params& p, int B, int Q, int N) {
-  return align_up((size_t)B * Q * N * sizeof(float), 256);
+  return idx_ws_layout(p, B, Q, N).total;
 }
 
 template <typename T>
@@ -183,13 +411,36 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
                              const float* w, const void* kI, int N,
                              int32_t* idx_out, float* score_out, void* ws,
                              cudaStream_t st) {
-  float* scores = (float*)ws;
-  if (p.act == CSA_F32)
+  const IdxWsLayout L = idx_ws_layout(p, B, Q, N);
+  const int R = B * Q;
+  char* base = (char*)ws;
+  float* scores = (float*)base;
+  if (index_tc_supported(p)) {
+    csa_status s = launch_index_scores_tc(p, B, Q, q_pos, qI, w, kI, N, scores,
+                                          (int*)(base + L.plan), st);
+    if (s != CSA_OK) return s;
+  } else if (p.act == CSA_F32) {
     launch_scores<float>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
-  else
+  } else {
     launch_scores<__nv_bfloat16>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
-  CSA_LAUNCH(KK_TOPK, st, topk_radix<<<B * Q, kTopkThreads, 0, st>>>(
-                              scores, N, q_pos, p.m, p.topk, idx_out, score_out));
+  }
+  if (use_multi_topk(R, N)) {
+    MultiTopkWs m{(unsigned*)(base + L.ghist), (unsigned*)(base + L.cand_cnt),
+                  (unsigned*)(base + L.bitmap), (uint2*)(base + L.cand)};
+    // ghist and cand_cnt are adjacent: one memset clears both
+    if (cudaMemsetAsync(m.ghist, 0, L.bitmap - L.ghist, st) != cudaSuccess) return CSA_ERR_CUDA;
+    dim3 grid(R, (N + kChunk - 1) / kChunk);
+    CSA_LAUNCH(KK_TOPK_HIST, st, topk_hist<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m, p.topk,
+                                                                  m.ghist));
+    CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m,
+                                                                      p.topk, m));
+    CSA_LAUNCH(KK_TOPK_FINAL, st, topk_finalize<<<R, 1024, 0, st>>>(scores, N, q_pos, p.m,
+                                                                    p.topk, m, idx_out,
+                                                                    score_out));
+  } else {
+    CSA_LAUNCH(KK_TOPK, st, topk_radix<<<R, kTopkThreads, 0, st>>>(scores, N, q_pos, p.m,
+                                                                   p.topk, idx_out, score_out));
+  }
   return last_launch_status();
 }
 

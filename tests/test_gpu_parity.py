@@ -41,6 +41,10 @@ INDEX_CASES = [
     ("bf16_ragged", "bf16", 2, 3, 3001, 64, 128, 512, "decode"),
     ("bf16_causal", "bf16", 1, 300, 300, 64, 128, 32, "prefill"),
     ("bf16_few_visible", "bf16", 3, 4, 200, 8, 64, 128, "prefill"),
+    ("bf16_h16_groups", "bf16", 2, 8, 900, 16, 64, 40, "prefill"),
+    ("bf16_h32_decode", "bf16", 5, 2, 2500, 32, 64, 64, "decode"),
+    ("bf16_multi_cta_topk", "bf16", 3, 1, 50000, 64, 128, 1024, "decode"),
+    ("bf16_multi_cta_ragged", "bf16", 2, 2, 9001, 64, 128, 300, "prefill"),
 ]
 
 
@@ -72,14 +76,16 @@ def test_index_topk_parity(case):
         check_topk(idx[rows].cpu().numpy(), sco[rows].cpu().numpy(), sref, nv, k, tol, name)
 
 
-def test_index_topk_all_ties_take_lowest_indices():
-    """w = 0: every score is 0, the selection is 0..k-1 (lower index wins)."""
-    wl = BASE.with_(n_hI=8, c_I=64, topk=100)
+@pytest.mark.parametrize("nh,N", [(8, 1000), (64, 20000)])
+def test_index_topk_all_ties_take_lowest_indices(nh, N):
+    """w = 0: every score is 0, the selection is 0..k-1 (lower index wins);
+    the long case overflows the multi-CTA candidate list on purpose."""
+    wl = BASE.with_(n_hI=nh, c_I=64, topk=100)
     p = bd.params_for(wl)
-    qI = torch.randn(2, 8, 64).to(torch.bfloat16).to(DEV)
-    w = torch.zeros(2, 8, device=DEV)
-    kI = torch.randn(2, 1000, 64).to(torch.bfloat16).to(DEV)
-    pos = torch.full((2,), 4000, dtype=torch.int32, device=DEV)
+    qI = torch.randn(2, nh, 64).to(torch.bfloat16).to(DEV)
+    w = torch.zeros(2, nh, device=DEV)
+    kI = torch.randn(2, N, 64).to(torch.bfloat16).to(DEV)
+    pos = torch.full((2,), 4 * N, dtype=torch.int32, device=DEV)
     idx = torch.empty(2, 100, dtype=torch.int32, device=DEV)
     bd.csa_index_topk(p, pos, qI, w, kI, idx)
     assert torch.equal(idx.cpu(), torch.arange(100, dtype=torch.int32).repeat(2, 1))
