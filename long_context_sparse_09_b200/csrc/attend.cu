@@ -290,8 +290,21 @@ __global__ void attend_combine(AttnArgs a) {
 
 static int head_block(int n_h) { return n_h >= 16 ? 16 : n_h; }
 
+bool attend_tc_supported(const csa_params& p);
+void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps);
+csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
+                            const int32_t* q_pos, const void* q, const int32_t* idx,
+                            const void* ckv, const float* ckv_scale, int N, const void* win,
+                            const float* win_scale, int W, const int32_t* win_pos0,
+                            const float* sink, void* out, float* ws_o, float* ws_ml,
+                            int nsplit, int kps, cudaStream_t st);
+
 static void split_plan(const csa_params& p, int R, int N, bool dense, int* nsplit,
                        int* kps) {
+  if (attend_tc_supported(p)) {
+    attend_tc_plan(p, R, N, dense, nsplit, kps);
+    return;
+  }
   const int HB = head_block(p.n_h);
   const int base_ctas = R * (p.n_h / HB);
   const int nk_max = (dense ? N : p.topk) + p.n_win;
@@ -362,6 +375,14 @@ csa_status launch_attend(const csa_params& p, bool dense, int B, int Q,
   if (a.nsplit > 1) {
     a.ws_o = (float*)ws;
     a.ws_ml = (float*)((char*)ws + align_up((size_t)a.nsplit * R * p.n_h * p.c * 4, 256));
+  }
+  if (attend_tc_supported(p)) {
+    csa_status s = launch_attend_tc(p, dense, B, Q, q_pos, q, idx, ckv, ckv_scale, N, win,
+                                    win_scale, W, win_pos0, sink, out, a.ws_o, a.ws_ml,
+                                    a.nsplit, a.keys_per_split, st);
+    if (s != CSA_OK || a.nsplit <= 1) return s;
+    CSA_LAUNCH(KK_COMBINE, st, attend_combine<__nv_bfloat16><<<dim3(R, a.n_h), 128, 0, st>>>(a));
+    return last_launch_status();
   }
   if (p.act == CSA_F32) {
     if (p.kv == CSA_F32) return launch_attn_c<float, CSA_F32>(a, R, st);

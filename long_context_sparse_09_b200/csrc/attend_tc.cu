@@ -1,0 +1,578 @@
+// attend_tc.cu -- shared-KV MQA with window and sink on the 5th-generation
+// tensor cores ("DeepSeekV4技术报告阅读笔记" eq. 19 / 26 / 27, sections
+// 2.5.2-2.5.3; "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" sections 2.4-2.5).
+//
+// A CTA owns (query, block of 64 heads, slice of the query's key list).  The
+// 64 heads are the MMA's M dimension: S = Q K^T (M = 64 heads, N = 64 keys,
+// K = 512 dims) and O += P V (M = 64 heads, N = dims, K = 64 keys).  An M = 64
+// accumulator fills half of every 32-lane TMEM sub-partition, so O (64 x 512
+// fp32) lives as two halves -- dims 0-255 in the upper half-lanes, dims
+// 256-511 in the lower half-lanes, 256 columns -- and the two S buffers of a
+// double-buffered key tile sit in the remaining columns, one per half.  Each
+// softmax thread therefore owns one head's row: the max, exp and sum are
+// in-thread.  The running max is kept "lazily": O is rescaled only when a
+// tile raises it by more than 8 (e^8 headroom in fp32).
+//
+// One smem key tile [64 keys][512] bf16 in the 128-byte swizzle layout is
+// both the K-major B operand of Q K^T and the MN-major B operand of P V.
+// Keys are gathered (top-k indices, window rows) by four loader warps with
+// 16-byte loads; FP8-mixed rows are widened to bf16 exactly (E4M3 codes are
+// bf16 values) and their per-row scale is applied in fp32: logit =
+// scale_j * (q . codes_j) + q_rope . rope_j, and P V uses p_j * scale_j for
+// the FP8 dims and p_j for the RoPE dims.
+//
+// Warps: 0-3 gather keys, 4 loads Q by TMA / owns TMEM / issues MMAs, 5-8 run
+// the softmax and the epilogue (sink, normalisation, R_{-t0}, store).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace csa {
+
+using namespace sm100;
+
+struct AttnTcArgs {
+  const int32_t* q_pos;
+  const int32_t* idx;
+  const uint8_t* ckv;
+  const float* ckv_scale;
+  const uint8_t* win;
+  const float* win_scale;
+  const int32_t* win_pos0;
+  const float* sink;
+  __nv_bfloat16* out;
+  float* ws_o;
+  float* ws_ml;
+  unsigned* err;
+  int Q, N, W, n_h, m, topk, n_win, nsplit, keys_per_split, dense, R, hblocks;
+  float scale;
+  double base;
+};
+
+constexpr int kAtKeys = 64;       // keys per tile
+constexpr int kAtThreads = 288;   // 9 warps
+constexpr int kQBytes = 64 * 1024;
+constexpr int kKBytes = 64 * 1024;
+constexpr int kPBytes = 8 * 1024;
+constexpr float kLazyRescale = 8.0f;
+
+template <bool FP8>
+struct AtLayout {
+  static constexpr int NP = FP8 ? 2 : 1;  // P buffers per tile parity
+  static constexpr int q = 0;
+  static constexpr int k = kQBytes;
+  static constexpr int p = k + 2 * kKBytes;
+  static constexpr int meta = p + 2 * NP * kPBytes;
+  static constexpr int bars = meta + 1024;
+  static constexpr int total = bars + 256;
+};
+
+__device__ __forceinline__ uint4 zero4() { return make_uint4(0u, 0u, 0u, 0u); }
+
+__device__ __forceinline__ void st_shared16(uint8_t* p, uint4 v) {
+  *reinterpret_cast<uint4*>(p) = v;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 16 E4M3 codes -> 16 bf16 (exact), as two 16-byte chunks
+__device__ __forceinline__ void widen_e4m3(uint4 raw, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t x = w[i];
+    o[2 * i] = pack_bf16(e4m3_to_f32(x & 0xFF), e4m3_to_f32((x >> 8) & 0xFF));
+    o[2 * i + 1] = pack_bf16(e4m3_to_f32((x >> 16) & 0xFF), e4m3_to_f32(x >> 24));
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kAtThreads, 1)
+    attend_tc(const __grid_constant__ CUtensorMap tmQ, AttnTcArgs a) {
+  using L = AtLayout<FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = sm + L::q;
+  uint8_t* sK = sm + L::k;
+  uint8_t* sP = sm + L::p;
+  float* meta_scale = (float*)(sm + L::meta);         // [2][64]
+  int* meta_valid = (int*)(sm + L::meta + 512);       // [2][64]
+  uint64_t* bars = (uint64_t*)(sm + L::bars);
+  uint64_t* qfull = bars;
+  uint64_t* kfull = bars + 1;
+  uint64_t* kempty = bars + 3;
+  uint64_t* sfull = bars + 5;
+  uint64_t* sfree = bars + 7;
+  uint64_t* pfull = bars + 9;
+  uint64_t* pvdone = bars + 11;
+  uint32_t* tbase_sm = (uint32_t*)(bars + 13);
+  volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
+  __shared__ const uint8_t* row_sm[kAtKeys];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x;
+  const int per_r = a.hblocks * a.nsplit;
+  const int r = item / per_r;
+  const int hb = (item % per_r) / a.nsplit;
+  const int sp = item % a.nsplit;
+  const int b = r / a.Q;
+  const int t0 = a.q_pos[r];
+  const int nv = n_visible(t0, a.m, a.N);
+  const int lo = t0 - a.n_win + 1 > 0 ? t0 - a.n_win + 1 : 0;
+  const int nwin_q = (a.n_win > 0 && t0 >= 0) ? t0 - lo + 1 : 0;
+  const int n_main = a.dense ? nv : a.topk;
+  const int nk = n_main + nwin_q;
+  const int j_begin = sp * a.keys_per_split;
+  const int j_end = min(nk, j_begin + a.keys_per_split);
+  const int ntiles = j_end > j_begin ? (j_end - j_begin + kAtKeys - 1) / kAtKeys : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kfull[i], 128);
+      mbar_init(&kempty[i], 1);
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sfree[i], 4);
+      mbar_init(&pfull[i], 4);
+      mbar_init(&pvdone[i], 1);
+    }
+    *abort_sm = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tbase_sm, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tbase_sm;
+  const size_t rb = FP8 ? 576 : 1024;  // stored row bytes
+
+  if (ntiles > 0) {
+    if (warp < 4) {
+      // ------------------------------------------------------ key gather --
+      const int t = threadIdx.x;
+      const uint8_t* ckv = a.ckv + (size_t)b * a.N * rb;
+      const uint8_t* win = a.win + (size_t)b * a.W * rb;
+      const int wp0 = a.win ? a.win_pos0[b] : 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i & 1;
+        if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
+        if (t < kAtKeys) {
+          const int j = j_begin + i * kAtKeys + t;
+          int valid = 0;
+          const uint8_t* row = nullptr;
+          float sc = 1.f;
+          if (j < j_end) {
+            if (j < n_main) {
+              const int e = a.dense ? j : a.idx[(size_t)r * a.topk + j];
+              if (e >= 0) {
+                if (e < nv) {
+                  valid = 1;
+                  row = ckv + (size_t)e * rb;
+                  if (FP8) sc = a.ckv_scale[(size_t)b * a.N + e];
+                } else {
+                  atomicOr(a.err, CSA_DEV_BAD_INDEX);
+                }
+              }
+            } else {
+              const int wr = lo + (j - n_main) - wp0;
+              if (a.win != nullptr && wr >= 0 && wr < a.W) {
+                valid = 1;
+                row = win + (size_t)wr * rb;
+                if (FP8) sc = a.win_scale[(size_t)b * a.W + wr];
+              } else {
+                atomicOr(a.err, CSA_DEV_BAD_WINDOW);
+              }
+            }
+          }
+          row_sm[t] = valid ? row : nullptr;
+          meta_valid[s * 64 + t] = valid;
+          meta_scale[s * 64 + t] = sc;
+        }
+        named_bar(1, 128);
+        uint8_t* dstK = sK + s * kKBytes;
+        if (!FP8) {
+#pragma unroll 1
+          for (int it0 = 0; it0 < 32; it0 += 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int idx = (it0 + u) * 128 + t;
+              const int key = idx >> 6, ch = idx & 63;
+              const uint8_t* src = row_sm[key];
+              v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int idx = (it0 + u) * 128 + t;
+              const int key = idx >> 6, ch = idx & 63;
+              const int kb = ch >> 3, c = ch & 7;
+              st_shared16(dstK + kb * 8192 + key * 128 + ((c ^ (key & 7)) << 4), v[u]);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int it0 = 0; it0 < 18; it0 += 6) {
+            uint4 v[6];
+#pragma unroll
+            for (int u = 0; u < 6; ++u) {
+              const int idx = (it0 + u) * 128 + t;
+              const int key = idx / 36, ch = idx % 36;
+              const uint8_t* src = row_sm[key];
+              v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
+            }
+#pragma unroll
+            for (int u = 0; u < 6; ++u) {
+              const int idx = (it0 + u) * 128 + t;
+              const int key = idx / 36, ch = idx % 36;
+              uint8_t* rowp = dstK + key * 128;
+              const int sw = key & 7;
+              if (ch < 28) {
+                uint4 lo4, hi4;
+                widen_e4m3(v[u], lo4, hi4);
+                const int d0 = 2 * ch;  // destination chunk of dims 16ch..16ch+7
+                const int kb = d0 >> 3, c0 = d0 & 7;
+                st_shared16(rowp + kb * 8192 + ((c0 ^ sw) << 4), lo4);
+                st_shared16(rowp + kb * 8192 + (((c0 + 1) ^ sw) << 4), hi4);
+              } else {
+                const int c = ch - 28;  // dims 448 + 8c .. : K-block 7
+                st_shared16(rowp + 7 * 8192 + ((c ^ sw) << 4), v[u]);
+              }
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&kfull[s]);
+        named_bar(1, 128);  // row_sm is rewritten by the next tile
+      }
+    } else if (warp == 4) {
+      // ------------------------------------------------------------- MMA --
+      if (lane == 0) {
+        mbar_expect_tx(qfull, kQBytes);
+        for (int kb = 0; kb < 8; ++kb)
+          tma_load_2d(sQ + kb * 8192, &tmQ, qfull, kb * 64, r * a.n_h + hb * 64);
+        const uint32_t idesc_qk = idesc_bf16(64, 64, false);
+        bool ok = mbar_wait(qfull, 0, abort_sm);
+        for (int i = 0; ok && i < ntiles; ++i) {
+          const int s = i & 1, bb = i & 1;
+          if (!mbar_wait(&kfull[s], (i >> 1) & 1, abort_sm)) break;
+          if (!mbar_wait(&sfree[bb], ((i >> 1) & 1) ^ 1, abort_sm)) break;
+          tc_fence_after();
+          const uint32_t sacc = tbase + ((uint32_t)(16 * bb) << 16) + 256;
+          const uint32_t qb = smem_u32(sQ), kbase = smem_u32(sK + s * kKBytes);
+#pragma unroll
+          for (int kb = 0; kb < 8; ++kb) {
+            const bool rope_blk = FP8 && kb == 7;
+            const uint32_t d = rope_blk ? sacc + 64 : sacc;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const bool first = j == 0 && (kb == 0 || rope_blk);
+              mma_bf16(d, sdesc_k_sw128(qb + kb * 8192 + j * 32),
+                       sdesc_k_sw128(kbase + kb * 8192 + j * 32), idesc_qk, first ? 0u : 1u);
+            }
+          }
+          mma_commit(&sfull[bb]);
+          if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort_sm)) break;
+          tc_fence_after();
+          const uint32_t pb = smem_u32(sP + bb * L::NP * kPBytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t acc = (i > 0 || j > 0) ? 1u : 0u;
+            const uint32_t vb = kbase + j * 2048;  // 16 keys of the tile
+            if (!FP8) {
+              mma_bf16(tbase, sdesc_k_sw128(pb + j * 32), sdesc_mn_sw128(vb, 8192, 1024),
+                       idesc_bf16(64, 256, true), acc);
+              mma_bf16(tbase + (16u << 16), sdesc_k_sw128(pb + j * 32),
+                       sdesc_mn_sw128(vb + 4 * 8192, 8192, 1024), idesc_bf16(64, 256, true), acc);
+            } else {
+              const uint32_t ps = pb, p1 = pb + kPBytes;  // p*scale, p
+              mma_bf16(tbase, sdesc_k_sw128(ps + j * 32), sdesc_mn_sw128(vb, 8192, 1024),
+                       idesc_bf16(64, 256, true), acc);
+              mma_bf16(tbase + (16u << 16), sdesc_k_sw128(ps + j * 32),
+                       sdesc_mn_sw128(vb + 4 * 8192, 8192, 1024), idesc_bf16(64, 192, true), acc);
+              mma_bf16(tbase + (16u << 16) + 192, sdesc_k_sw128(p1 + j * 32),
+                       sdesc_mn_sw128(vb + 7 * 8192, 8192, 1024), idesc_bf16(64, 64, true), acc);
+            }
+          }
+          mma_commit(&kempty[s]);
+          mma_commit(&pvdone[bb]);
+        }
+      }
+    } else {
+      // ------------------------------------------------- softmax / output --
+      const int quad = warp & 3;
+      const int half = lane >> 4;
+      const int hl = quad * 16 + (lane & 15);  // head within the block
+      const int head = hb * 64 + hl;
+      const uint32_t trow = tbase + ((uint32_t)(quad * 32) << 16);
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int i = 0; i < ntiles; ++i) {
+        const int bb = i & 1, s = i & 1;
+        const bool mine = half == bb;
+        if (!mbar_wait(&sfull[bb], (i >> 1) & 1, abort_sm)) { ok = false; break; }
+        tc_fence_after();
+        float sv[64];
+        float rv[FP8 ? 64 : 1];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[16];
+          tmem_ld16(trow + 256 + c * 16, v);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) sv[c * 16 + u] = v[u];
+        }
+        if (FP8) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float v[16];
+            tmem_ld16(trow + 320 + c * 16, v);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) rv[FP8 ? c * 16 + u : 0] = v[u];
+          }
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfree[bb]);
+        float mt = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          float z = -INFINITY;
+          if (meta_valid[s * 64 + j]) {
+            z = FP8 ? a.scale * fmaf(meta_scale[s * 64 + j], sv[j], rv[FP8 ? j : 0])
+                    : a.scale * sv[j];
+          }
+          sv[j] = z;
+          mt = fmaxf(mt, z);
+        }
+        float alpha = 1.f;
+        int resc = 0;
+        float m_new = fmaxf(m_used, mt);
+        if (m_new > -INFINITY) {
+          if (m_used == -INFINITY) {
+            m_used = m_new;
+          } else if (m_new > m_used + kLazyRescale) {
+            alpha = expf(m_used - m_new);
+            m_used = m_new;
+            resc = 1;
+          }
+        }
+        const int src = mine ? lane : (lane ^ 16);
+        m_used = __shfl_sync(0xffffffffu, m_used, src);
+        alpha = __shfl_sync(0xffffffffu, alpha, src);
+        resc = __shfl_sync(0xffffffffu, resc, src);
+        if (__any_sync(0xffffffffu, resc)) {
+          // O must not be in flight: wait for the previous tile's P V
+          if (!mbar_wait(&pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_sm)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t orow = trow + ((uint32_t)(16 * half) << 16);
+          for (int c0 = 0; c0 < 256; c0 += 16) {
+            float v[16];
+            tmem_ld16(orow + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] *= alpha;
+            tmem_st16(orow + c0, v);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        float lsum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float p = (m_used == -INFINITY || sv[j] == -INFINITY) ? 0.f : expf(sv[j] - m_used);
+          lsum += p;
+          sv[j] = p;
+        }
+        l = l * alpha + lsum;
+        l = __shfl_sync(0xffffffffu, l, src);
+        // P buffer bb was read by the P V of tile i-2
+        if (i >= 2 && !mbar_wait(&pvdone[bb], ((i - 2) >> 1) & 1, abort_sm)) { ok = false; break; }
+        if (mine) {
+          uint8_t* prow = sP + bb * L::NP * kPBytes + hl * 128;
+          const float* scl = meta_scale + s * 64;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int off = ((c ^ (hl & 7)) << 4);
+            const float* x = sv + 8 * c;
+            const uint4 w1 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                        pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+            if (FP8) {
+              const float* y = scl + 8 * c;
+              const uint4 ws = make_uint4(pack_bf16(x[0] * y[0], x[1] * y[1]),
+                                          pack_bf16(x[2] * y[2], x[3] * y[3]),
+                                          pack_bf16(x[4] * y[4], x[5] * y[5]),
+                                          pack_bf16(x[6] * y[6], x[7] * y[7]));
+              st_shared16(prow + off, ws);
+              st_shared16(prow + kPBytes + off, w1);
+            } else {
+              st_shared16(prow + off, w1);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pfull[bb]);
+      }
+      // ---------------------------------------------------------- output --
+      if (ok && mbar_wait(&pvdone[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_sm)) {
+        tc_fence_after();
+        const uint32_t orow = trow + ((uint32_t)(16 * half) << 16);
+        const bool store = head < a.n_h;
+        const int dim0 = half * 256;
+        if (a.nsplit == 1) {
+          const float zs = store ? a.sink[head] : 0.f;
+          const float M = fmaxf(m_used, zs);
+          const float em = m_used == -INFINITY ? 0.f : expf(m_used - M);
+          const float den = l * em + expf(zs - M);
+          const float f = em / den;
+          __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + (store ? head : 0)) * 512 + dim0;
+          for (int c0 = 0; c0 < 256; c0 += 16) {
+            float v[16];
+            tmem_ld16(orow + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] *= f;
+            if (dim0 + c0 >= 448) {  // RoPE dims: apply R_{-t0}
+#pragma unroll
+              for (int u = 0; u < 16; u += 2) {
+                float cs, sn;
+                rope_cs(-(double)t0, (dim0 + c0 + u - 448) >> 1, 64, a.base, &cs, &sn);
+                const float x0 = v[u], x1 = v[u + 1];
+                v[u] = x0 * cs - x1 * sn;
+                v[u + 1] = x0 * sn + x1 * cs;
+              }
+            }
+            if (store) {
+              *reinterpret_cast<uint4*>(dst + c0) =
+                  make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                             pack_bf16(v[6], v[7]));
+              *reinterpret_cast<uint4*>(dst + c0 + 8) =
+                  make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                             pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+            }
+          }
+        } else {
+          const size_t slot = ((size_t)sp * a.R + r) * a.n_h + (store ? head : 0);
+          float* dst = a.ws_o + slot * 512 + dim0;
+          for (int c0 = 0; c0 < 256; c0 += 16) {
+            float v[16];
+            tmem_ld16(orow + c0, v);
+            tmem_wait_ld();
+            if (store)
+#pragma unroll
+              for (int u = 0; u < 16; u += 4)
+                *reinterpret_cast<float4*>(dst + c0 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+          }
+          if (store && half == 0) {
+            a.ws_ml[slot * 2] = m_used;
+            a.ws_ml[slot * 2 + 1] = l;
+          }
+        }
+      }
+    }
+  }
+  if (ntiles == 0 && warp >= 5) {
+    // no keys in this slice: all weight on the sink (or an empty partial)
+    const int quad = warp & 3, half = lane >> 4;
+    const int head = hb * 64 + quad * 16 + (lane & 15);
+    if (head < a.n_h) {
+      if (a.nsplit == 1) {
+        __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + head) * 512 + half * 256;
+        for (int c0 = 0; c0 < 256; c0 += 8) *reinterpret_cast<uint4*>(dst + c0) = zero4();
+      } else {
+        const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
+        float* dst = a.ws_o + slot * 512 + half * 256;
+        for (int c0 = 0; c0 < 256; c0 += 4)
+          *reinterpret_cast<float4*>(dst + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (half == 0) {
+          a.ws_ml[slot * 2] = -INFINITY;
+          a.ws_ml[slot * 2 + 1] = 0.f;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_sm) {
+    if (threadIdx.x == 0) atomicOr(a.err, CSA_DEV_TIMEOUT);
+    const uint64_t t0w = globaltimer();
+    while (globaltimer() - t0w < 200000ull) __nanosleep(1000);
+  }
+  if (warp == 4) tmem_dealloc(tbase, 512);
+}
+
+// ------------------------------------------------------------------ host --
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+bool tma_available();
+
+bool attend_tc_supported(const csa_params& p) {
+  return p.act == CSA_BF16 && (p.kv == CSA_BF16 || p.kv == CSA_KV_FP8MIX) && p.c == 512 &&
+         p.rope_dims == 64 && p.n_h % 16 == 0 && (p.n_h <= 64 || p.n_h % 64 == 0) &&
+         tma_available();
+}
+
+void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps) {
+  const int hbn = (p.n_h + 63) / 64;
+  const int base = R * hbn;
+  const int nk_max = (dense ? N : p.topk) + p.n_win;
+  int s = (148 + base - 1) / base;
+  const int max_s = (nk_max + kAtKeys - 1) / kAtKeys;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  int k = (nk_max + s - 1) / s;
+  k = (k + kAtKeys - 1) / kAtKeys * kAtKeys;
+  if (k < kAtKeys) k = kAtKeys;
+  *kps = k;
+  *nsplit = nk_max > 0 ? (nk_max + k - 1) / k : 1;
+}
+
+csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
+                            const int32_t* q_pos, const void* q, const int32_t* idx,
+                            const void* ckv, const float* ckv_scale, int N, const void* win,
+                            const float* win_scale, int W, const int32_t* win_pos0,
+                            const float* sink, void* out, float* ws_o, float* ws_ml,
+                            int nsplit, int kps, cudaStream_t st) {
+  const int R = B * Q;
+  const int hbn = (p.n_h + 63) / 64;
+  CUtensorMap tmQ;
+  if (!make_tmap_bf16(&tmQ, q, (uint64_t)R * p.n_h, 512, 64)) return CSA_ERR_CUDA;
+  AttnTcArgs a{};
+  a.q_pos = q_pos; a.idx = idx; a.ckv = (const uint8_t*)ckv; a.ckv_scale = ckv_scale;
+  a.win = (const uint8_t*)win; a.win_scale = win_scale; a.win_pos0 = win_pos0; a.sink = sink;
+  a.out = (__nv_bfloat16*)out; a.ws_o = ws_o; a.ws_ml = ws_ml; a.err = device_error_word();
+  a.Q = Q; a.N = N; a.W = W; a.n_h = p.n_h; a.m = p.m; a.topk = p.topk; a.n_win = p.n_win;
+  a.nsplit = nsplit; a.keys_per_split = kps; a.dense = dense ? 1 : 0; a.R = R; a.hblocks = hbn;
+  a.scale = p.softmax_scale; a.base = (double)p.rope_base;
+  if (a.err == nullptr) return CSA_ERR_CUDA;
+  const long long items = (long long)R * hbn * nsplit;
+  if (p.kv == CSA_KV_FP8MIX) {
+    const int smem = AtLayout<true>::total + 1024;
+    if (cudaFuncSetAttribute(attend_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return CSA_ERR_CUDA;
+    CSA_LAUNCH(KK_ATTN, st, attend_tc<true><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, a));
+  } else {
+    const int smem = AtLayout<false>::total + 1024;
+    if (cudaFuncSetAttribute(attend_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return CSA_ERR_CUDA;
+    CSA_LAUNCH(KK_ATTN, st, attend_tc<false><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, a));
+  }
+  return last_launch_status();
+}
+
+}  // namespace csa

@@ -293,7 +293,7 @@ static EncodeTiledFn encode_fn() {
 
 // 2-D bf16 tensor [rows][cols] (cols contiguous), boxes of 64 x box_rows with
 // the 128-byte swizzle.
-static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -306,6 +306,8 @@ static bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+bool tma_available() { return encode_fn() != nullptr; }
 
 bool index_tc_supported(const csa_params& p) {
   return p.act == CSA_BF16 && (p.c_I == 64 || p.c_I == 128) && p.n_hI % 16 == 0 &&
