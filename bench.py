@@ -247,6 +247,10 @@ def run_ours(args, world, rank, local):
         build.build_library()
     _barrier(world)
     wl = WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(B=args.batch)
+    if args.context:
+        wl = wl.with_(T=args.context)
     dev = torch.device(f"cuda:{local}")
     torch.manual_seed(0)
     if wl.mode != "decode":
@@ -257,28 +261,41 @@ def run_ours(args, world, rank, local):
         step.run()
     torch.cuda.synchronize()
     assert bd.device_status() == 0, "device error word set during warm-up"
+    # The timed step is a CUDA-graph replay of the library calls (launch
+    # overhead out of the way); the graph carries the per-kernel event pairs
+    # of the library's profiler, read back after the timed replays.
+    bd.profile_enable(True)
+    step.run()
+    torch.cuda.synchronize()
+    bd.profile_collect()  # warms the event pool so capture creates no events
+    l0 = bd.kernel_launches()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step.run()
+    launches_per_step = bd.kernel_launches() - l0
+    bd.profile_enable(False)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
     clocks = ClockSampler(dev)
     time.sleep(0.15)
     _barrier(world)
     torch.cuda.synchronize()
-    bd.profile_enable(True)
-    bd.profile_collect()
-    l0 = bd.kernel_launches()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step.run()
+        graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     _barrier(world)
-    launches = bd.kernel_launches() - l0
-    prof = bd.profile_collect()
-    bd.profile_enable(False)
+    prof = bd.profile_collect()  # per-kernel device time of the last replay
     clk = clocks.stop()
+    launches = launches_per_step * args.steps
     ms = e0.elapsed_time(e1) / args.steps
     ms = _max_over_ranks(ms, world)
     units = step.units() * world
     value = units / (ms / 1e3)
+    assert bd.device_status() == 0, "device error word set during the timed steps"
 
     # end to end through the public API: pinned host inputs -> device, step,
     # result -> pinned host, every step
@@ -307,7 +324,7 @@ def run_ours(args, world, rank, local):
     assert bd.device_status() == 0, "device error word set during the timed steps"
 
     kind, nbytes, src, bound = step.dominant()
-    kms, kcnt = prof.get(kind, (0.0, 0))
+    kms, kcnt = prof.get(kind, (0.0, 0))  # one replay: kcnt launches of the kernel
     hbm, tfl, peak_src = _peaks()
     roof = None
     if kcnt:
@@ -319,7 +336,7 @@ def run_ours(args, world, rank, local):
                 "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": kind,
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
                 "peak_source": peak_src}
-    kernels = {k: {"ms_per_step": round(v[0] / args.steps, 5), "launches": v[1],
+    kernels = {k: {"ms_per_step": round(v[0], 5), "launches": v[1],
                    "share": round(v[0] / max(sum(x[0] for x in prof.values()), 1e-12), 4)}
                for k, v in prof.items() if v[1]}
 
@@ -344,6 +361,7 @@ def run_ours(args, world, rank, local):
                     "unit": "query-tok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 5)},
             "gpu_launches": launches,
+            "timing": "CUDA-graph replay of the step; per-kernel times from the last replay",
             "roofline": roof,
             "kernels": kernels,
             "cpu_baseline": cpu,
@@ -389,11 +407,13 @@ def run_reference(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (profiling)")
+    ap.add_argument("--context", type=int, default=0, help="override context length (profiling)")
     args = ap.parse_args()
     world, rank, local = _dist()
     try:

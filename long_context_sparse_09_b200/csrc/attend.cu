@@ -256,32 +256,61 @@ __global__ void attend_simt(AttnArgs a) {
 }
 
 // Fixed-order combine of the splits, sink, normalisation, R_{-t0}, store.
+// One CTA per (query, head): the split weights exp(m_s - M) are formed once
+// in shared memory, then each thread sums its 4 dims over the splits with
+// the loads issued back to back.
 template <typename T>
-__global__ void attend_combine(AttnArgs a) {
+__global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
+  __shared__ float wsp[256];
+  __shared__ float s_den;
   const int r = blockIdx.x, head = blockIdx.y;
   const size_t R = gridDim.x;
   const int c = a.c;
+  const int S = a.nsplit;
   const float zs = a.sink[head];
-  float M = zs;
-  for (int s = 0; s < a.nsplit; ++s)
-    M = fmaxf(M, a.ws_ml[(((size_t)s * R + r) * a.n_h + head) * 2]);
-  float den = expf(zs - M);
-  for (int s = 0; s < a.nsplit; ++s) {
-    size_t slot = ((size_t)s * R + r) * a.n_h + head;
-    den += a.ws_ml[slot * 2 + 1] * expf(a.ws_ml[slot * 2] - M);
+  // split maxima and sums (S <= 256)
+  float mloc = -INFINITY;
+  for (int s = threadIdx.x; s < S; s += blockDim.x)
+    mloc = fmaxf(mloc, a.ws_ml[(((size_t)s * R + r) * a.n_h + head) * 2]);
+  __shared__ float red[32];
+  const float M = fmaxf(block_reduce<true>(mloc, red), zs);
+  float dloc = 0.f;
+  for (int s = threadIdx.x; s < S; s += blockDim.x) {
+    const size_t slot = ((size_t)s * R + r) * a.n_h + head;
+    const float wgt = expf(a.ws_ml[slot * 2] - M);
+    wsp[s] = wgt;
+    dloc += a.ws_ml[slot * 2 + 1] * wgt;
   }
+  const float dsum = block_reduce<false>(dloc, red);
+  if (threadIdx.x == 0) s_den = dsum + expf(zs - M);
+  __syncthreads();
+  const float inv = 1.0f / s_den;
   const int t0 = a.q_pos[r];
   T* dst = reinterpret_cast<T*>(a.out) + ((size_t)r * a.n_h + head) * c;
+  const size_t stride = R * a.n_h * (size_t)c / 4;  // float4 stride between splits
   for (int e = 4 * threadIdx.x; e < c; e += 4 * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(a.ws_o + ((size_t)r * a.n_h + head) * c) + e / 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < a.nsplit; ++s) {
-      size_t slot = ((size_t)s * R + r) * a.n_h + head;
-      float f = expf(a.ws_ml[slot * 2] - M);
-      float4 v = reinterpret_cast<const float4*>(a.ws_o + slot * c)[e / 4];
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float4 v0 = src[(size_t)s * stride], v1 = src[(size_t)(s + 1) * stride];
+      float4 v2 = src[(size_t)(s + 2) * stride], v3 = src[(size_t)(s + 3) * stride];
+      const float f0 = wsp[s], f1 = wsp[s + 1], f2 = wsp[s + 2], f3 = wsp[s + 3];
+      acc.x = fmaf(f0, v0.x, acc.x); acc.y = fmaf(f0, v0.y, acc.y);
+      acc.z = fmaf(f0, v0.z, acc.z); acc.w = fmaf(f0, v0.w, acc.w);
+      acc.x = fmaf(f1, v1.x, acc.x); acc.y = fmaf(f1, v1.y, acc.y);
+      acc.z = fmaf(f1, v1.z, acc.z); acc.w = fmaf(f1, v1.w, acc.w);
+      acc.x = fmaf(f2, v2.x, acc.x); acc.y = fmaf(f2, v2.y, acc.y);
+      acc.z = fmaf(f2, v2.z, acc.z); acc.w = fmaf(f2, v2.w, acc.w);
+      acc.x = fmaf(f3, v3.x, acc.x); acc.y = fmaf(f3, v3.y, acc.y);
+      acc.z = fmaf(f3, v3.z, acc.z); acc.w = fmaf(f3, v3.w, acc.w);
+    }
+    for (; s < S; ++s) {
+      const float4 v = src[(size_t)s * stride];
+      const float f = wsp[s];
       acc.x = fmaf(f, v.x, acc.x); acc.y = fmaf(f, v.y, acc.y);
       acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
     }
-    float inv = 1.0f / den;
     acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
     derotate4(acc, e, c, a.rd, t0, a.base);
     store4<T>(dst + e, acc);
@@ -311,6 +340,7 @@ static void split_plan(const csa_params& p, int R, int N, bool dense, int* nspli
   const int want = 148 * 4;
   int s = 1;
   if (base_ctas < want) s = (want + base_ctas - 1) / base_ctas;
+  if (s > 256) s = 256;  // the combine keeps <= 256 split weights in shared memory
   int max_s = (nk_max + kKT - 1) / kKT;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
@@ -321,6 +351,7 @@ static void split_plan(const csa_params& p, int R, int N, bool dense, int* nspli
   if (*nsplit < 1) *nsplit = 1;
   *kps = k;
 }
+
 
 size_t attend_ws_bytes(const csa_params& p, int B, int Q, int N, bool dense) {
   int ns, kps;

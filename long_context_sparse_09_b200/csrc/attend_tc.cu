@@ -25,6 +25,8 @@
 // the softmax and the epilogue (sink, normalisation, R_{-t0}, store).
 #include <cuda.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -47,16 +49,27 @@ struct AttnTcArgs {
   float* ws_ml;
   unsigned* err;
   int Q, N, W, n_h, m, topk, n_win, nsplit, keys_per_split, dense, R, hblocks;
-  float scale;
+  int R_rows_c, R_rows_w;  // total rows of the cache / window tensors (out of range)
+  float scale2;  // softmax scale times log2(e): the softmax runs in base 2
   double base;
 };
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kMasked = -1e30f;  // logit of an absent key (exp2 -> 0)
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 constexpr int kAtKeys = 64;       // keys per tile
 constexpr int kAtThreads = 288;   // 9 warps
 constexpr int kQBytes = 64 * 1024;
 constexpr int kKBytes = 64 * 1024;
 constexpr int kPBytes = 8 * 1024;
-constexpr float kLazyRescale = 8.0f;
+constexpr float kLazyRescale = 8.0f;  // log2 units: rescale when the max grows 256x
 
 template <bool FP8>
 struct AtLayout {
@@ -94,17 +107,24 @@ __device__ __forceinline__ void widen_e4m3(uint4 raw, uint4& lo, uint4& hi) {
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// Key-row tensor maps (bf16 caches): boxes of 64 columns x 64 rows for
+// contiguous key runs, and of 64 x 1 rows for gathers of selected rows.
+struct KeyMaps {
+  CUtensorMap c_box, c_row, w_box, w_row;
+};
+
 template <bool FP8>
 __global__ void __launch_bounds__(kAtThreads, 1)
-    attend_tc(const __grid_constant__ CUtensorMap tmQ, AttnTcArgs a) {
+    attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KeyMaps km,
+              AttnTcArgs a) {
   using L = AtLayout<FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = sm + L::q;
   uint8_t* sK = sm + L::k;
   uint8_t* sP = sm + L::p;
-  float* meta_scale = (float*)(sm + L::meta);         // [2][64]
-  int* meta_valid = (int*)(sm + L::meta + 512);       // [2][64]
+  float* meta_scale = (float*)(sm + L::meta);                       // [2][64]
+  unsigned long long* meta_mask = (unsigned long long*)(sm + L::meta + 512);  // [2]
   uint64_t* bars = (uint64_t*)(sm + L::bars);
   uint64_t* qfull = bars;
   uint64_t* kfull = bars + 1;
@@ -137,7 +157,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kfull[i], 128);
+      mbar_init(&kfull[i], FP8 ? 128 : 1);
       mbar_init(&kempty[i], 1);
       mbar_init(&sfull[i], 1);
       mbar_init(&sfree[i], 4);
@@ -158,8 +178,100 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const size_t rb = FP8 ? 576 : 1024;  // stored row bytes
 
   if (ntiles > 0) {
-    if (warp < 4) {
-      // ------------------------------------------------------ key gather --
+    if (!FP8 && warp == 0) {
+      // --------------------------------------------- key loads by TMA (bf16) --
+      // Contiguous runs (HCA entries, window rows) come in as 64-row boxes;
+      // selected rows as 4-row gathers; a tile that straddles the entry and
+      // window lists, or a 4-key group of mixed origin, takes one-row loads.
+      // Absent keys read an in-range row (the sequence's first), masked out.
+      const int wp0 = a.win ? a.win_pos0[b] : 0;
+      const int crow_oob = min(b * a.N, a.R_rows_c - 1), wrow_oob = min(b * a.W, a.R_rows_w - 1);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i & 1;
+        if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
+        const int j0 = j_begin + i * kAtKeys;
+        int row[2], inwin[2], valid[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int j = j0 + lane + 32 * h2;
+          row[h2] = crow_oob;
+          inwin[h2] = 0;
+          valid[h2] = 0;
+          if (j < j_end) {
+            if (j < n_main) {
+              const int e = a.dense ? j : a.idx[(size_t)r * a.topk + j];
+              if (e >= 0) {
+                if (e < nv) {
+                  valid[h2] = 1;
+                  row[h2] = b * a.N + e;
+                } else {
+                  atomicOr(a.err, CSA_DEV_BAD_INDEX);
+                }
+              }
+            } else {
+              inwin[h2] = 1;
+              row[h2] = wrow_oob;
+              const int wr = lo + (j - n_main) - wp0;
+              if (a.win != nullptr && wr >= 0 && wr < a.W) {
+                valid[h2] = 1;
+                row[h2] = b * a.W + wr;
+              } else {
+                atomicOr(a.err, CSA_DEV_BAD_WINDOW);
+              }
+            }
+          } else if (j >= n_main) {
+            inwin[h2] = 1;
+            row[h2] = wrow_oob;
+          }
+          meta_scale[s * 64 + lane + 32 * h2] = 1.f;
+        }
+        const unsigned m0 = __ballot_sync(0xffffffffu, valid[0]);
+        const unsigned m1 = __ballot_sync(0xffffffffu, valid[1]);
+        if (lane == 0) meta_mask[s] = ((unsigned long long)m1 << 32) | m0;
+        const unsigned w0 = __ballot_sync(0xffffffffu, inwin[0]);
+        const unsigned w1 = __ballot_sync(0xffffffffu, inwin[1]);
+        uint8_t* dstK = sK + s * kKBytes;
+        if (lane == 0) mbar_expect_tx(&kfull[s], kKBytes);
+        __syncwarp();
+        const bool all_entry = (w0 | w1) == 0u, all_win = (w0 & w1) == 0xffffffffu;
+        if (a.dense && all_entry) {  // contiguous entries s = j0 .. j0+63
+          if (lane < 8)
+            tma_load_2d(dstK + lane * 8192, &km.c_box, &kfull[s], lane * 64, b * a.N + j0);
+        } else if (all_win) {  // contiguous window rows
+          const int wr0 = b * a.W + lo + (j0 - n_main) - wp0;
+          if (lane < 8) tma_load_2d(dstK + lane * 8192, &km.w_box, &kfull[s], lane * 64, wr0);
+        } else {
+          // lane l: 4-key group g = l & 15, K-blocks 4*(l >> 4) .. +3
+          const int g = lane & 15;
+          int gr[4], gw = 0;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int k = 4 * g + u;
+            const int r0 = __shfl_sync(0xffffffffu, row[0], k & 31);
+            const int r1 = __shfl_sync(0xffffffffu, row[1], k & 31);
+            gr[u] = k < 32 ? r0 : r1;
+          }
+          const unsigned wbits = (w0 >> (4 * (g & 7))) & 0xFu;  // keys 4g..4g+3 (g < 8)
+          const unsigned wbits_hi = (w1 >> (4 * (g & 7))) & 0xFu;
+          gw = g < 8 ? (int)wbits : (int)wbits_hi;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int kb = 4 * (lane >> 4) + q4;
+            uint8_t* dst = dstK + kb * 8192 + g * 4 * 128;
+            if (gw == 0)
+              tma_gather4(dst, &km.c_row, &kfull[s], kb * 64, gr[0], gr[1], gr[2], gr[3]);
+            else if (gw == 0xF)
+              tma_gather4(dst, &km.w_row, &kfull[s], kb * 64, gr[0], gr[1], gr[2], gr[3]);
+            else
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                tma_load_2d(dst + u * 128, ((gw >> u) & 1) ? &km.w_row : &km.c_row, &kfull[s],
+                            kb * 64, gr[u]);
+          }
+        }
+      }
+    } else if (FP8 && warp < 4) {
+      // ------------------------------------------- key gather (FP8-mixed) --
       const int t = threadIdx.x;
       const uint8_t* ckv = a.ckv + (size_t)b * a.N * rb;
       const uint8_t* win = a.win + (size_t)b * a.W * rb;
@@ -179,7 +291,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 if (e < nv) {
                   valid = 1;
                   row = ckv + (size_t)e * rb;
-                  if (FP8) sc = a.ckv_scale[(size_t)b * a.N + e];
+                  sc = a.ckv_scale[(size_t)b * a.N + e];
                 } else {
                   atomicOr(a.err, CSA_DEV_BAD_INDEX);
                 }
@@ -189,66 +301,44 @@ __global__ void __launch_bounds__(kAtThreads, 1)
               if (a.win != nullptr && wr >= 0 && wr < a.W) {
                 valid = 1;
                 row = win + (size_t)wr * rb;
-                if (FP8) sc = a.win_scale[(size_t)b * a.W + wr];
+                sc = a.win_scale[(size_t)b * a.W + wr];
               } else {
                 atomicOr(a.err, CSA_DEV_BAD_WINDOW);
               }
             }
           }
           row_sm[t] = valid ? row : nullptr;
-          meta_valid[s * 64 + t] = valid;
           meta_scale[s * 64 + t] = sc;
+          const unsigned bits = __ballot_sync(0xffffffffu, valid);
+          if ((t & 31) == 0) reinterpret_cast<unsigned*>(&meta_mask[s])[t >> 5] = bits;
         }
         named_bar(1, 128);
         uint8_t* dstK = sK + s * kKBytes;
-        if (!FP8) {
-#pragma unroll 1
-          for (int it0 = 0; it0 < 32; it0 += 8) {
-            uint4 v[8];
+        // all 18 loads in flight, then widen and store
+        uint4 v[18];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int idx = (it0 + u) * 128 + t;
-              const int key = idx >> 6, ch = idx & 63;
-              const uint8_t* src = row_sm[key];
-              v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
-            }
+        for (int u = 0; u < 18; ++u) {
+          const int idx = u * 128 + t;
+          const int key = idx / 36, ch = idx % 36;
+          const uint8_t* src = row_sm[key];
+          v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
+        }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int idx = (it0 + u) * 128 + t;
-              const int key = idx >> 6, ch = idx & 63;
-              const int kb = ch >> 3, c = ch & 7;
-              st_shared16(dstK + kb * 8192 + key * 128 + ((c ^ (key & 7)) << 4), v[u]);
-            }
-          }
-        } else {
-#pragma unroll 1
-          for (int it0 = 0; it0 < 18; it0 += 6) {
-            uint4 v[6];
-#pragma unroll
-            for (int u = 0; u < 6; ++u) {
-              const int idx = (it0 + u) * 128 + t;
-              const int key = idx / 36, ch = idx % 36;
-              const uint8_t* src = row_sm[key];
-              v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
-            }
-#pragma unroll
-            for (int u = 0; u < 6; ++u) {
-              const int idx = (it0 + u) * 128 + t;
-              const int key = idx / 36, ch = idx % 36;
-              uint8_t* rowp = dstK + key * 128;
-              const int sw = key & 7;
-              if (ch < 28) {
-                uint4 lo4, hi4;
-                widen_e4m3(v[u], lo4, hi4);
-                const int d0 = 2 * ch;  // destination chunk of dims 16ch..16ch+7
-                const int kb = d0 >> 3, c0 = d0 & 7;
-                st_shared16(rowp + kb * 8192 + ((c0 ^ sw) << 4), lo4);
-                st_shared16(rowp + kb * 8192 + (((c0 + 1) ^ sw) << 4), hi4);
-              } else {
-                const int c = ch - 28;  // dims 448 + 8c .. : K-block 7
-                st_shared16(rowp + 7 * 8192 + ((c ^ sw) << 4), v[u]);
-              }
-            }
+        for (int u = 0; u < 18; ++u) {
+          const int idx = u * 128 + t;
+          const int key = idx / 36, ch = idx % 36;
+          uint8_t* rowp = dstK + key * 128;
+          const int sw = key & 7;
+          if (ch < 28) {
+            uint4 lo4, hi4;
+            widen_e4m3(v[u], lo4, hi4);
+            const int d0 = 2 * ch;  // destination chunk of dims 16ch..16ch+7
+            const int kb = d0 >> 3, c0 = d0 & 7;
+            st_shared16(rowp + kb * 8192 + ((c0 ^ sw) << 4), lo4);
+            st_shared16(rowp + kb * 8192 + (((c0 + 1) ^ sw) << 4), hi4);
+          } else {
+            const int c = ch - 28;  // dims 448 + 8c .. : K-block 7
+            st_shared16(rowp + 7 * 8192 + ((c ^ sw) << 4), v[u]);
           }
         }
         fence_proxy_async_smem();
@@ -262,14 +352,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         for (int kb = 0; kb < 8; ++kb)
           tma_load_2d(sQ + kb * 8192, &tmQ, qfull, kb * 64, r * a.n_h + hb * 64);
         const uint32_t idesc_qk = idesc_bf16(64, 64, false);
+        const uint32_t qb = smem_u32(sQ);
         bool ok = mbar_wait(qfull, 0, abort_sm);
-        for (int i = 0; ok && i < ntiles; ++i) {
+        // S(i) = Q K(i)^T into S buffer i&1 (waits for the tile and the buffer)
+        auto issue_qk = [&](int i) -> bool {
           const int s = i & 1, bb = i & 1;
-          if (!mbar_wait(&kfull[s], (i >> 1) & 1, abort_sm)) break;
-          if (!mbar_wait(&sfree[bb], ((i >> 1) & 1) ^ 1, abort_sm)) break;
+          if (!mbar_wait(&kfull[s], (i >> 1) & 1, abort_sm)) return false;
+          fence_proxy_async_smem();  // cp.async-written tile -> tensor-core reads
+          if (!mbar_wait(&sfree[bb], ((i >> 1) & 1) ^ 1, abort_sm)) return false;
           tc_fence_after();
           const uint32_t sacc = tbase + ((uint32_t)(16 * bb) << 16) + 256;
-          const uint32_t qb = smem_u32(sQ), kbase = smem_u32(sK + s * kKBytes);
+          const uint32_t kbase = smem_u32(sK + s * kKBytes);
 #pragma unroll
           for (int kb = 0; kb < 8; ++kb) {
             const bool rope_blk = FP8 && kb == 7;
@@ -282,8 +375,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
           }
           mma_commit(&sfull[bb]);
+          return true;
+        };
+        if (ok) ok = issue_qk(0);
+        for (int i = 0; ok && i < ntiles; ++i) {
+          const int s = i & 1, bb = i & 1;
+          if (i + 1 < ntiles && !issue_qk(i + 1)) break;  // overlaps softmax(i)
           if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort_sm)) break;
           tc_fence_after();
+          const uint32_t kbase = smem_u32(sK + s * kKBytes);
           const uint32_t pb = smem_u32(sP + bb * L::NP * kPBytes);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -308,14 +408,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           mma_commit(&pvdone[bb]);
         }
       }
-    } else {
+    } else if (warp >= 5) {
       // ------------------------------------------------- softmax / output --
       const int quad = warp & 3;
       const int half = lane >> 4;
       const int hl = quad * 16 + (lane & 15);  // head within the block
       const int head = hb * 64 + hl;
       const uint32_t trow = tbase + ((uint32_t)(quad * 32) << 16);
-      float m_used = -INFINITY, l = 0.f;
+      float m_used = kMasked, l = 0.f;  // running max (base 2) and sum
       bool ok = true;
       for (int i = 0; i < ntiles; ++i) {
         const int bb = i & 1, s = i & 1;
@@ -323,7 +423,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (!mbar_wait(&sfull[bb], (i >> 1) & 1, abort_sm)) { ok = false; break; }
         tc_fence_after();
         float sv[64];
-        float rv[FP8 ? 64 : 1];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float v[16];
@@ -331,39 +430,40 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) sv[c * 16 + u] = v[u];
         }
-        if (FP8) {
+        if (FP8) {  // logit = scale_j * (q . codes_j) + q_rope . rope_j, 16 keys at a time
+          tmem_wait_ld();
+          const float* scl0 = meta_scale + s * 64;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             float v[16];
             tmem_ld16(trow + 320 + c * 16, v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 16; ++u) rv[FP8 ? c * 16 + u : 0] = v[u];
+            for (int u = 0; u < 16; ++u) sv[c * 16 + u] = fmaf(scl0[c * 16 + u], sv[c * 16 + u], v[u]);
           }
         }
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sfree[bb]);
-        float mt = -INFINITY;
+        // logits in base-2 units; absent keys get a huge negative logit
+        const unsigned long long vmask = meta_mask[s];
+        const float* scl = meta_scale + s * 64;
+        float mt = kMasked;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          float z = -INFINITY;
-          if (meta_valid[s * 64 + j]) {
-            z = FP8 ? a.scale * fmaf(meta_scale[s * 64 + j], sv[j], rv[FP8 ? j : 0])
-                    : a.scale * sv[j];
-          }
+          const float z = ((vmask >> j) & 1ull) ? a.scale2 * sv[j] : kMasked;
           sv[j] = z;
           mt = fmaxf(mt, z);
         }
         float alpha = 1.f;
         int resc = 0;
-        float m_new = fmaxf(m_used, mt);
-        if (m_new > -INFINITY) {
-          if (m_used == -INFINITY) {
-            m_used = m_new;
-          } else if (m_new > m_used + kLazyRescale) {
-            alpha = expf(m_used - m_new);
-            m_used = m_new;
+        if (mt > 0.5f * kMasked) {  // the tile has a present key
+          if (m_used == kMasked) {
+            m_used = mt;
+          } else if (mt > m_used + kLazyRescale) {
+            alpha = fast_exp2(m_used - mt);
+            m_used = mt;
             resc = 1;
           }
         }
@@ -390,7 +490,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         float lsum = 0.f;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          const float p = (m_used == -INFINITY || sv[j] == -INFINITY) ? 0.f : expf(sv[j] - m_used);
+          const float p = sv[j] > 0.5f * kMasked ? fast_exp2(sv[j] - m_used) : 0.f;
           lsum += p;
           sv[j] = p;
         }
@@ -400,7 +500,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (i >= 2 && !mbar_wait(&pvdone[bb], ((i - 2) >> 1) & 1, abort_sm)) { ok = false; break; }
         if (mine) {
           uint8_t* prow = sP + bb * L::NP * kPBytes + hl * 128;
-          const float* scl = meta_scale + s * 64;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const int off = ((c ^ (hl & 7)) << 4);
@@ -430,22 +529,31 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const uint32_t orow = trow + ((uint32_t)(16 * half) << 16);
         const bool store = head < a.n_h;
         const int dim0 = half * 256;
+        const bool any = m_used > 0.5f * kMasked;
+        float f = 1.f;
         if (a.nsplit == 1) {
-          const float zs = store ? a.sink[head] : 0.f;
-          const float M = fmaxf(m_used, zs);
-          const float em = m_used == -INFINITY ? 0.f : expf(m_used - M);
-          const float den = l * em + expf(zs - M);
-          const float f = em / den;
-          __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + (store ? head : 0)) * 512 + dim0;
-          for (int c0 = 0; c0 < 256; c0 += 16) {
-            float v[16];
-            tmem_ld16(orow + c0, v);
-            tmem_wait_ld();
+          const float zs = store ? a.sink[head] * kLog2e : 0.f;
+          const float M = fmaxf(any ? m_used : zs, zs);
+          const float em = any ? fast_exp2(m_used - M) : 0.f;
+          f = em / (l * em + fast_exp2(zs - M));
+        }
+        for (int c0 = 0; c0 < 256; c0 += 64) {
+          float v[64];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] *= f;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float w16[16];
+            tmem_ld16(orow + c0 + q4 * 16, w16);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[q4 * 16 + u] = w16[u];
+          }
+          tmem_wait_ld();
+          if (!store) continue;
+          if (a.nsplit == 1) {
+#pragma unroll
+            for (int u = 0; u < 64; ++u) v[u] *= f;
             if (dim0 + c0 >= 448) {  // RoPE dims: apply R_{-t0}
 #pragma unroll
-              for (int u = 0; u < 16; u += 2) {
+              for (int u = 0; u < 64; u += 2) {
                 float cs, sn;
                 rope_cs(-(double)t0, (dim0 + c0 + u - 448) >> 1, 64, a.base, &cs, &sn);
                 const float x0 = v[u], x1 = v[u + 1];
@@ -453,31 +561,24 @@ __global__ void __launch_bounds__(kAtThreads, 1)
                 v[u + 1] = x0 * sn + x1 * cs;
               }
             }
-            if (store) {
-              *reinterpret_cast<uint4*>(dst + c0) =
-                  make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                             pack_bf16(v[6], v[7]));
-              *reinterpret_cast<uint4*>(dst + c0 + 8) =
-                  make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
-                             pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
-            }
-          }
-        } else {
-          const size_t slot = ((size_t)sp * a.R + r) * a.n_h + (store ? head : 0);
-          float* dst = a.ws_o + slot * 512 + dim0;
-          for (int c0 = 0; c0 < 256; c0 += 16) {
-            float v[16];
-            tmem_ld16(orow + c0, v);
-            tmem_wait_ld();
-            if (store)
+            __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + head) * 512 + dim0 + c0;
 #pragma unroll
-              for (int u = 0; u < 16; u += 4)
-                *reinterpret_cast<float4*>(dst + c0 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+            for (int u = 0; u < 64; u += 8)
+              *reinterpret_cast<uint4*>(dst + u) =
+                  make_uint4(pack_bf16(v[u], v[u + 1]), pack_bf16(v[u + 2], v[u + 3]),
+                             pack_bf16(v[u + 4], v[u + 5]), pack_bf16(v[u + 6], v[u + 7]));
+          } else {
+            const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
+            float* dst = a.ws_o + slot * 512 + dim0 + c0;
+#pragma unroll
+            for (int u = 0; u < 64; u += 4)
+              *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
           }
-          if (store && half == 0) {
-            a.ws_ml[slot * 2] = m_used;
-            a.ws_ml[slot * 2 + 1] = l;
-          }
+        }
+        if (store && a.nsplit > 1 && half == 0) {  // natural-log max for the combine
+          const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
+          a.ws_ml[slot * 2] = any ? m_used * kLn2 : -INFINITY;
+          a.ws_ml[slot * 2 + 1] = l;
         }
       }
     }
@@ -530,6 +631,7 @@ void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, 
   const int base = R * hbn;
   const int nk_max = (dense ? N : p.topk) + p.n_win;
   int s = (148 + base - 1) / base;
+  if (s > 256) s = 256;
   const int max_s = (nk_max + kAtKeys - 1) / kAtKeys;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
@@ -556,21 +658,41 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
   a.out = (__nv_bfloat16*)out; a.ws_o = ws_o; a.ws_ml = ws_ml; a.err = device_error_word();
   a.Q = Q; a.N = N; a.W = W; a.n_h = p.n_h; a.m = p.m; a.topk = p.topk; a.n_win = p.n_win;
   a.nsplit = nsplit; a.keys_per_split = kps; a.dense = dense ? 1 : 0; a.R = R; a.hblocks = hbn;
-  a.scale = p.softmax_scale; a.base = (double)p.rope_base;
+  a.scale2 = p.softmax_scale * kLog2e; a.base = (double)p.rope_base;
   if (a.err == nullptr) return CSA_ERR_CUDA;
   const long long items = (long long)R * hbn * nsplit;
+  KeyMaps km;
+  memset(&km, 0, sizeof(km));
+  a.R_rows_c = B * N;
+  a.R_rows_w = B * W;
+  if (p.kv == CSA_BF16) {
+    // a tensor map needs at least one row: an empty cache / window borrows
+    // the other's memory (its rows are never used)
+    const void* cbase = N > 0 ? ckv : win;
+    const void* wbase = (W > 0 && win) ? win : ckv;
+    const uint64_t crows = N > 0 ? (uint64_t)B * N : (uint64_t)B * W;
+    const uint64_t wrows = (W > 0 && win) ? (uint64_t)B * W : (uint64_t)B * N;
+    if (crows == 0 || wrows == 0) return CSA_ERR_UNSUPPORTED;
+    if (!make_tmap_bf16(&km.c_box, cbase, crows, 512, 64) ||
+        !make_tmap_bf16(&km.c_row, cbase, crows, 512, 1) ||
+        !make_tmap_bf16(&km.w_box, wbase, wrows, 512, 64) ||
+        !make_tmap_bf16(&km.w_row, wbase, wrows, 512, 1))
+      return CSA_ERR_CUDA;
+    a.R_rows_c = (int)crows;
+    a.R_rows_w = (int)wrows;
+  }
   if (p.kv == CSA_KV_FP8MIX) {
     const int smem = AtLayout<true>::total + 1024;
     if (cudaFuncSetAttribute(attend_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return CSA_ERR_CUDA;
-    CSA_LAUNCH(KK_ATTN, st, attend_tc<true><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, a));
+    CSA_LAUNCH(KK_ATTN, st, attend_tc<true><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, km, a));
   } else {
     const int smem = AtLayout<false>::total + 1024;
     if (cudaFuncSetAttribute(attend_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return CSA_ERR_CUDA;
-    CSA_LAUNCH(KK_ATTN, st, attend_tc<false><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, a));
+    CSA_LAUNCH(KK_ATTN, st, attend_tc<false><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, km, a));
   }
   return last_launch_status();
 }

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/csa.h"
+#include "csa.h"
 
 namespace csa {
 

@@ -26,6 +26,16 @@ static std::atomic<bool> g_prof_on{false};
 static std::vector<ProfRec> g_prof_recs;
 static std::vector<ProfRec> g_prof_free;
 
+// Events recorded while `st` is being captured into a CUDA graph must be
+// external event nodes to be recorded at each replay.
+static void prof_record(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, st);
+}
+
 int prof_begin(int kind, cudaStream_t st) {
   if (!g_prof_on.load(std::memory_order_relaxed)) return -1;
   std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -37,7 +47,7 @@ int prof_begin(int kind, cudaStream_t st) {
   } else if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) {
     return -1;
   }
-  cudaEventRecord(r.a, st);
+  prof_record(r.a, st);
   g_prof_recs.push_back(r);
   return (int)g_prof_recs.size() - 1;
 }
@@ -45,7 +55,7 @@ int prof_begin(int kind, cudaStream_t st) {
 void prof_end(int slot, cudaStream_t st) {
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  if (slot < (int)g_prof_recs.size()) cudaEventRecord(g_prof_recs[slot].b, st);
+  if (slot < (int)g_prof_recs.size()) prof_record(g_prof_recs[slot].b, st);
 }
 
 static const char* kKindNames[KK_COUNT] = {

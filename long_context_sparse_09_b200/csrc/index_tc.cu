@@ -21,6 +21,8 @@
 // prefix sum on the device), split evenly over a persistent grid.
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -35,8 +37,11 @@ struct IdxTcArgs {
   const int* prefix;  // [ngroups + 1] exclusive prefix of tiles per group
   float* scores;      // [R][N]
   unsigned* err;
+  unsigned* ghist;    // [R][4096] key histograms for the top-k (G == 1), or null
   int Q, N, m, nhI, ngroups;
 };
+
+constexpr int kHistBins = 4096;  // top 12 bits of the order-preserving score key
 
 constexpr int kTileM = 128;
 constexpr int kKBlockBytes = kTileM * 128;  // 128 rows x 64 bf16
@@ -47,11 +52,18 @@ struct IdxTcCfg {
   static constexpr int kThreads = 64 + 32 * NE;
 };
 
-// Per-group visible tile counts and their exclusive prefix (one CTA).
+// Per-group visible tile counts and their exclusive prefix (CTA 0), and
+// zeroing of the top-k bookkeeping words (every CTA, a strided share).
 __global__ void __launch_bounds__(1024) index_plan(const int32_t* __restrict__ q_pos, int G,
                                                    int ngroups, int m, int N,
-                                                   int* __restrict__ prefix) {
+                                                   int* __restrict__ prefix,
+                                                   unsigned* __restrict__ zero_words,
+                                                   size_t nzero) {
   __shared__ unsigned sh[33];
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nzero;
+       i += (size_t)gridDim.x * blockDim.x)
+    zero_words[i] = 0u;
+  if (blockIdx.x != 0) return;
   unsigned running = 0;
   for (int base = 0; base < ngroups; base += blockDim.x) {
     const int g = base + threadIdx.x;
@@ -116,6 +128,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint32_t* tbase_sm = (uint32_t*)(tempty + 2);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
+  unsigned* shist = (unsigned*)((uint8_t*)bars + 256);  // [kHistBins] when G == 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int ncols_alloc = 32;
@@ -221,10 +234,28 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
       const int quad = warp & 3;         // TMEM lane quadrant of this warp
       const int nq_mine = NE == 4 ? G : G / 2;
       const int q0 = NE == 4 ? 0 : (e >> 2) * (G / 2);
+      const bool hist = G == 1 && a.ghist != nullptr;
+      const int et = threadIdx.x - 64;  // 0 .. 32*NE-1
+      if (hist) {
+        for (int i = et; i < kHistBins; i += 32 * NE) shist[i] = 0u;
+        named_bar(2, 32 * NE);
+      }
       TileCursor cur;
       cur.init(a.prefix, a.ngroups, start, count);
-      int an = 0;
+      int an = 0, hist_r = cur.g;
       for (int i = 0; i < count; ++i) {
+        if (hist && cur.g != hist_r) {  // query changed: flush its histogram
+          named_bar(2, 32 * NE);
+          for (int bin = et; bin < kHistBins; bin += 32 * NE) {
+            const unsigned c = shist[bin];
+            if (c) {
+              atomicAdd(&a.ghist[(size_t)hist_r * kHistBins + bin], c);
+              shist[bin] = 0u;
+            }
+          }
+          named_bar(2, 32 * NE);
+          hist_r = cur.g;
+        }
         const int acc = an & 1;
         if (!mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm)) break;
         tc_fence_after();
@@ -252,10 +283,20 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
         for (int qq = 0; qq < nq_mine; ++qq) {
           const int r = cur.g * G + q0 + qq;
           const int nv = n_visible(__ldg(a.q_pos + r), a.m, a.N);
-          if (s < nv) a.scores[(size_t)r * a.N + s] = sc[qq];
+          if (s < nv) {
+            a.scores[(size_t)r * a.N + s] = sc[qq];
+            if (hist) atomicAdd(&shist[score_key(sc[qq]) >> 20], 1u);
+          }
         }
         ++an;
         cur.next(a.prefix, a.ngroups);
+      }
+      if (hist) {  // flush the last query's histogram
+        named_bar(2, 32 * NE);
+        for (int bin = et; bin < kHistBins; bin += 32 * NE) {
+          const unsigned c = shist[bin];
+          if (c) atomicAdd(&a.ghist[(size_t)hist_r * kHistBins + bin], c);
+        }
       }
     }
   }
@@ -328,7 +369,8 @@ static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
                               const IdxTcArgs& a, cudaStream_t st) {
   using Cfg = IdxTcCfg<G, KB, S, NE>;
   const int NROWS = G * a.nhI;
-  size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + 2 * (size_t)KB * NROWS * 128 + 256;
+  size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + 2 * (size_t)KB * NROWS * 128 + 256 +
+                (G == 1 ? kHistBins * 4 : 0);
   auto kern = index_scores_tc<G, KB, S, NE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -345,17 +387,23 @@ static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
 
 csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32_t* q_pos,
                                   const void* qI, const float* w, const void* kI, int N,
-                                  float* scores, int* plan, cudaStream_t st) {
+                                  float* scores, int* plan, unsigned* zero_words, size_t nzero,
+                                  unsigned* ghist, bool* hist_done, cudaStream_t st) {
   const int R = B * Q;
   const int G = index_tc_group(p, Q);
   const int ngroups = R / G;
-  CSA_LAUNCH(KK_PLAN, st, index_plan<<<1, 1024, 0, st>>>(q_pos, G, ngroups, p.m, N, plan));
+  const unsigned zblocks = (unsigned)std::min<size_t>(64, (nzero + 16383) / 16384 + 1);
+  CSA_LAUNCH(KK_PLAN, st, index_plan<<<zblocks, 1024, 0, st>>>(q_pos, G, ngroups, p.m, N, plan,
+                                                               zero_words, nzero));
+  *hist_done = false;
   if (N == 0) return last_launch_status();
   CUtensorMap tmK, tmQ;
   if (!make_tmap_bf16(&tmK, kI, (uint64_t)B * N, p.c_I, kTileM)) return CSA_ERR_CUDA;
   if (!make_tmap_bf16(&tmQ, qI, (uint64_t)R * p.n_hI, p.c_I, G * p.n_hI)) return CSA_ERR_CUDA;
-  IdxTcArgs a{q_pos, w, plan, scores, device_error_word(), Q, N, p.m, p.n_hI, ngroups};
+  IdxTcArgs a{q_pos, w, plan, scores, device_error_word(), G == 1 ? ghist : nullptr,
+              Q, N, p.m, p.n_hI, ngroups};
   if (a.err == nullptr) return CSA_ERR_CUDA;
+  *hist_done = a.ghist != nullptr;
   const bool k2 = p.c_I == 128;
   if (G == 1) return k2 ? launch_tc_t<1, 2, 5, 4>(tmK, tmQ, a, st) : launch_tc_t<1, 1, 8, 4>(tmK, tmQ, a, st);
   if (G == 2) return k2 ? launch_tc_t<2, 2, 4, 4>(tmK, tmQ, a, st) : launch_tc_t<2, 1, 6, 4>(tmK, tmQ, a, st);

@@ -177,6 +177,7 @@ constexpr int kCandCap = 4096;  // candidates per query
 struct MultiTopkWs {
   unsigned* ghist;     // [R][kBins]
   unsigned* cand_cnt;  // [R]
+  unsigned* done;      // [R] CTAs of the select pass that have finished
   unsigned* bitmap;    // [R][N32]
   uint2* cand;         // [R][kCandCap] (key, index)
 };
@@ -227,96 +228,96 @@ __device__ void find_threshold_bin(const unsigned* __restrict__ gh, unsigned k, 
   *above_out = *sAbove;
 }
 
-__global__ void __launch_bounds__(1024) topk_select(const float* __restrict__ scores, int N,
-                                                    const int32_t* __restrict__ q_pos, int m,
-                                                    int k, MultiTopkWs ws) {
-  __shared__ unsigned scan[33];
-  __shared__ int sT;
-  __shared__ unsigned sAbove;
-  const int r = blockIdx.x;
-  const int nv = n_visible(q_pos[r], m, N);
-  if (nv <= k) return;
-  const int s0 = blockIdx.y * kChunk;
-  if (s0 >= N) return;
-  int T;
-  unsigned above;
-  find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, scan, &T, &above, &sT, &sAbove);
-  const int N32 = (N + 31) >> 5;
-  const float* sc = scores + (size_t)r * N;
-  const int s1 = min(N, s0 + kChunk);
-  for (int base = s0; base < s1; base += blockDim.x) {
-    const int s = base + threadIdx.x;
-    const bool vis = s < nv && s < s1;
-    const unsigned key = vis ? score_key(sc[s]) : 0u;
-    const int bin = (int)(key >> 20);
-    const bool gt = vis && bin > T;
-    const bool eq = vis && bin == T;
-    const unsigned word = __ballot_sync(0xffffffffu, gt);
-    if ((threadIdx.x & 31) == 0 && (s >> 5) < N32 && s < s1) ws.bitmap[(size_t)r * N32 + (s >> 5)] = word;
-    if (eq) {
-      unsigned pos = atomicAdd(&ws.cand_cnt[r], 1u);
-      if (pos < kCandCap) ws.cand[(size_t)r * kCandCap + pos] = make_uint2(key, (unsigned)s);
-    }
-  }
-}
+constexpr int kLocalCap = 2048;  // candidates one select CTA may hold locally
 
-__device__ __forceinline__ bool cand_before(uint2 x, uint2 y) {
-  return x.x > y.x || (x.x == y.x && x.y < y.y);
-}
-
-__global__ void __launch_bounds__(1024) topk_finalize(const float* __restrict__ scores, int N,
-                                                      const int32_t* __restrict__ q_pos, int m,
-                                                      int k, MultiTopkWs ws,
-                                                      int32_t* __restrict__ idx_out,
-                                                      float* __restrict__ score_out) {
-  __shared__ uint2 cand[kCandCap];
-  __shared__ RadixShared sh;
-  __shared__ int sT;
-  __shared__ unsigned sAbove;
-  const int r = blockIdx.x;
-  const int nv = n_visible(q_pos[r], m, N);
-  const float* sc = scores + (size_t)r * N;
-  int32_t* out = idx_out + (size_t)r * k;
-  float* sout = score_out ? score_out + (size_t)r * k : nullptr;
+// Exact completion of one query's selection (one CTA): a two-pass radix
+// select over the low 20 key bits of the bin-T candidates (all share the top
+// 12), equal keys resolved towards the lower index, the chosen ones marked
+// in the bitmap, then the bitmap compacted in index order.
+__device__ void finalize_query(const float* __restrict__ sc, int nv, int N, int k, int r,
+                               const MultiTopkWs& ws, int32_t* __restrict__ out,
+                               float* __restrict__ sout, uint2* cand, RadixShared& sh,
+                               int* sT, unsigned* sAbove) {
+  __shared__ unsigned s_eq_n;
+  __shared__ int s_fallback;
   if (nv <= k) {
     write_all_visible(sc, nv, k, out, sout);
     return;
   }
   int T;
   unsigned above;
-  find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, &sT, &sAbove);
+  find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, sT, sAbove);
   const unsigned nc = __ldcg(ws.cand_cnt + r);
   if (nc > (unsigned)kCandCap) {  // bin T too crowded: exact block-wide select
     radix_select_block(sc, nv, k, out, sout, sh);
     return;
   }
-  const unsigned need = (unsigned)k - above;
-  int P = 1;
-  while (P < (int)nc) P <<= 1;
-  for (int i = threadIdx.x; i < P; i += blockDim.x)
-    cand[i] = i < (int)nc ? __ldcg(ws.cand + (size_t)r * kCandCap + i) : make_uint2(0u, 0x7fffffffu);
-  __syncthreads();
-  // bitonic sort into (key descending, index ascending)
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
-        const int lo = 2 * stride * (i / stride) + (i % stride);
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const uint2 x = cand[lo], y = cand[hi];
-        if (up ? cand_before(y, x) : cand_before(x, y)) {
-          cand[lo] = y;
-          cand[hi] = x;
-        }
-      }
-      __syncthreads();
+  for (int i = threadIdx.x; i < (int)nc; i += blockDim.x)
+    cand[i] = __ldcg(ws.cand + (size_t)r * kCandCap + i);
+  // radix select of the need-th largest key among the candidates
+  unsigned remaining = (unsigned)k - above;  // 1 <= remaining <= nc
+  unsigned prefix = (unsigned)T << 20, mask = 0xFFF00000u;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sh.hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
+      const unsigned key = cand[i].x;
+      if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 1023u], 1u);
     }
+    __syncthreads();
+    // thread t owns bin 1023 - t (1024 threads): exclusive scan counts higher bins
+    const int bin = 1023 - (int)threadIdx.x;
+    const unsigned hcount = sh.hist[bin];
+    unsigned tot;
+    const unsigned higher = block_exclusive_scan(hcount, sh.scan, &tot);
+    if (higher < remaining && higher + hcount >= remaining) {
+      sh.digit = (unsigned)bin;
+      sh.remaining = remaining - higher;
+    }
+    __syncthreads();
+    prefix |= sh.digit << shift;
+    mask |= 1023u << shift;
+    remaining = sh.remaining;
+    __syncthreads();
   }
+  const unsigned K = prefix;  // exact key of the k-th largest score
+  // equal keys: the `remaining` lowest indices win
+  if (threadIdx.x == 0) { s_eq_n = 0; s_fallback = 0; }
+  __syncthreads();
   const int N32 = (N + 31) >> 5;
   unsigned* bm = ws.bitmap + (size_t)r * N32;
-  for (unsigned i = threadIdx.x; i < need; i += blockDim.x) {
-    const unsigned s = cand[i].y;
-    atomicOr(bm + (s >> 5), 1u << (s & 31));
+  for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
+    const uint2 c = cand[i];
+    if (c.x > K) {
+      atomicOr(bm + (c.y >> 5), 1u << (c.y & 31));
+    } else if (c.x == K) {
+      const unsigned p = atomicAdd(&s_eq_n, 1u);
+      if (p < 2048) sh.hist[p] = c.y;  // reuse the histogram as an index list
+    }
+  }
+  __syncthreads();
+  const unsigned neq = s_eq_n;
+  if (neq > 2048) {
+    s_fallback = 1;
+  } else if (neq == remaining) {
+    for (unsigned i = threadIdx.x; i < neq; i += blockDim.x) {
+      const unsigned s = sh.hist[i];
+      atomicOr(bm + (s >> 5), 1u << (s & 31));
+    }
+  } else {
+    // rank each equal-key index among the others (neq is small)
+    for (unsigned i = threadIdx.x; i < neq; i += blockDim.x) {
+      const unsigned s = sh.hist[i];
+      unsigned rank = 0;
+      for (unsigned j = 0; j < neq; ++j) rank += sh.hist[j] < s;
+      if (rank < remaining) atomicOr(bm + (s >> 5), 1u << (s & 31));
+    }
+  }
+  __syncthreads();
+  if (s_fallback) {  // a huge tie: exact block-wide select over all scores
+    radix_select_block(sc, nv, k, out, sout, sh);
+    return;
   }
   __threadfence();
   __syncthreads();
@@ -342,18 +343,82 @@ __global__ void __launch_bounds__(1024) topk_finalize(const float* __restrict__ 
   }
 }
 
+// Selection pass over a chunk of one query's scores; the last CTA of the
+// query to finish completes the query (threadfence + counter).
+__global__ void __launch_bounds__(1024) topk_select_final(
+    const float* __restrict__ scores, int N, const int32_t* __restrict__ q_pos, int m, int k,
+    MultiTopkWs ws, int32_t* __restrict__ idx_out, float* __restrict__ score_out) {
+  __shared__ uint2 cand[kCandCap];
+  __shared__ RadixShared sh;
+  __shared__ int sT;
+  __shared__ unsigned sAbove;
+  __shared__ int s_last;
+  __shared__ unsigned s_lcount, s_base;
+  const int r = blockIdx.x;
+  const int nv = n_visible(q_pos[r], m, N);
+  const float* sc = scores + (size_t)r * N;
+  const int s0 = blockIdx.y * kChunk;
+  if (threadIdx.x == 0) s_lcount = 0;
+  __syncthreads();
+  if (nv > k && s0 < N) {
+    int T;
+    unsigned above;
+    find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, &sT,
+                       &sAbove);
+    const int N32 = (N + 31) >> 5;
+    const int s1 = min(N, s0 + kChunk);
+    for (int base = s0; base < s1; base += blockDim.x) {
+      const int s = base + threadIdx.x;
+      const bool vis = s < nv && s < s1;
+      const unsigned key = vis ? score_key(sc[s]) : 0u;
+      const int bin = (int)(key >> 20);
+      const bool gt = vis && bin > T;
+      const bool eq = vis && bin == T;
+      const unsigned word = __ballot_sync(0xffffffffu, gt);
+      if ((threadIdx.x & 31) == 0 && (s >> 5) < N32 && s < s1)
+        ws.bitmap[(size_t)r * N32 + (s >> 5)] = word;
+      if (eq) {  // collect locally, publish with one global atomic per CTA
+        const unsigned pos = atomicAdd(&s_lcount, 1u);
+        if (pos < kLocalCap) cand[pos] = make_uint2(key, (unsigned)s);
+      }
+    }
+    __syncthreads();
+    const unsigned ln = s_lcount;
+    if (threadIdx.x == 0 && ln > 0)
+      s_base = atomicAdd(&ws.cand_cnt[r], ln > kLocalCap ? (unsigned)kCandCap + 1u : ln);
+    __syncthreads();
+    if (ln > 0 && ln <= kLocalCap)
+      for (unsigned i = threadIdx.x; i < ln; i += blockDim.x)
+        if (s_base + i < (unsigned)kCandCap) ws.cand[(size_t)r * kCandCap + s_base + i] = cand[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(&ws.done[r], 1u);
+    s_last = prev == gridDim.y - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  finalize_query(sc, nv, N, k, r, ws, idx_out + (size_t)r * k,
+                 score_out ? score_out + (size_t)r * k : nullptr, cand, sh, &sT, &sAbove);
+}
+
 // ------------------------------------------------------------------ host --
 bool index_tc_supported(const csa_params& p);
 int index_tc_group(const csa_params& p, int Q);
-size_t index_tc_plan_bytes(int ngroups);
 csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32_t* q_pos,
                                   const void* qI, const float* w, const void* kI, int N,
-                                  float* scores, int* plan, cudaStream_t st);
+                                  float* scores, int* plan, unsigned* zero_words, size_t nzero,
+                                  unsigned* ghist, bool* hist_done, cudaStream_t st);
+__global__ void index_plan(const int32_t* q_pos, int G, int ngroups, int m, int N, int* prefix,
+                           unsigned* zero_words, size_t nzero);
 
 static bool use_multi_topk(int R, int N) { return R <= 64 && N >= 4096; }
 
 struct IdxWsLayout {
-  size_t scores = 0, plan = 0, ghist = 0, cand_cnt = 0, bitmap = 0, cand = 0, total = 0;
+  size_t scores = 0, plan = 0, ghist = 0, cand_cnt = 0, done = 0, bitmap = 0, cand = 0,
+         total = 0;
 };
 
 static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
@@ -366,6 +431,8 @@ static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
     L.ghist = off;
     off += R * kBins * 4;
     L.cand_cnt = off;
+    off += R * 4;
+    L.done = off;
     off = align_up(off + R * 4, 256);
     L.bitmap = off;
     off += align_up(R * ((N + 31) / 32) * 4, 256);
@@ -415,28 +482,37 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
   const int R = B * Q;
   char* base = (char*)ws;
   float* scores = (float*)base;
-  if (index_tc_supported(p)) {
-    csa_status s = launch_index_scores_tc(p, B, Q, q_pos, qI, w, kI, N, scores,
-                                          (int*)(base + L.plan), st);
-    if (s != CSA_OK) return s;
-  } else if (p.act == CSA_F32) {
-    launch_scores<float>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
-  } else {
-    launch_scores<__nv_bfloat16>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
+  int* plan = (int*)(base + L.plan);
+  const bool multi = use_multi_topk(R, N);
+  MultiTopkWs mw{};
+  size_t nzero = 0;
+  if (multi) {
+    mw = MultiTopkWs{(unsigned*)(base + L.ghist), (unsigned*)(base + L.cand_cnt),
+                     (unsigned*)(base + L.done), (unsigned*)(base + L.bitmap),
+                     (uint2*)(base + L.cand)};
+    nzero = (L.bitmap - L.ghist) / 4;  // ghist, cand_cnt and done are contiguous
   }
-  if (use_multi_topk(R, N)) {
-    MultiTopkWs m{(unsigned*)(base + L.ghist), (unsigned*)(base + L.cand_cnt),
-                  (unsigned*)(base + L.bitmap), (uint2*)(base + L.cand)};
-    // ghist and cand_cnt are adjacent: one memset clears both
-    if (cudaMemsetAsync(m.ghist, 0, L.bitmap - L.ghist, st) != cudaSuccess) return CSA_ERR_CUDA;
+  bool hist_done = false;
+  if (index_tc_supported(p)) {
+    csa_status s = launch_index_scores_tc(p, B, Q, q_pos, qI, w, kI, N, scores, plan, mw.ghist,
+                                          nzero, multi ? mw.ghist : nullptr, &hist_done, st);
+    if (s != CSA_OK) return s;
+  } else {
+    if (multi)
+      CSA_LAUNCH(KK_PLAN, st, index_plan<<<1, 1024, 0, st>>>(q_pos, 1, 0, p.m, N, plan, mw.ghist,
+                                                             nzero));
+    if (p.act == CSA_F32)
+      launch_scores<float>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
+    else
+      launch_scores<__nv_bfloat16>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
+  }
+  if (multi) {
     dim3 grid(R, (N + kChunk - 1) / kChunk);
-    CSA_LAUNCH(KK_TOPK_HIST, st, topk_hist<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m, p.topk,
-                                                                  m.ghist));
-    CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m,
-                                                                      p.topk, m));
-    CSA_LAUNCH(KK_TOPK_FINAL, st, topk_finalize<<<R, 1024, 0, st>>>(scores, N, q_pos, p.m,
-                                                                    p.topk, m, idx_out,
-                                                                    score_out));
+    if (!hist_done)
+      CSA_LAUNCH(KK_TOPK_HIST, st, topk_hist<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m, p.topk,
+                                                                    mw.ghist));
+    CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select_final<<<grid, 1024, 0, st>>>(
+                                       scores, N, q_pos, p.m, p.topk, mw, idx_out, score_out));
   } else {
     CSA_LAUNCH(KK_TOPK, st, topk_radix<<<R, kTopkThreads, 0, st>>>(scores, N, q_pos, p.m,
                                                                    p.topk, idx_out, score_out));
