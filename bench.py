@@ -240,6 +240,67 @@ class DecodeStep:
         return nq, t_total, f"{nq} of the {wl.B} queries of one step (full context each)"
 
 
+class PrefillStep:
+    """One sequence of T tokens: compress (entries, indexer keys, window rows),
+    then index/top-k and attention for every token."""
+
+    def __init__(self, wl, device, seed_offset=0):
+        self.wl = wl
+        self.p = bd.params_for(wl)
+        wl_s = wl.with_(seed=wl.seed + seed_offset)
+        self.W = synth.weights(wl_s, device=device)
+        self.inp = synth.prefill_inputs(wl_s, device=device)
+        self.packed = bd.csa_pack_weights(self.p, self.W)
+        B, T = wl.B, wl.T
+        nE = T // wl.m
+        self.nE = nE
+        kvdt = torch.bfloat16 if wl.kv == "bf16" else torch.float32
+        self.ckv = torch.empty(B, nE, wl.c, dtype=kvdt, device=device)
+        self.win = torch.empty(B, T, wl.c, dtype=kvdt, device=device)
+        self.kI = torch.empty(B, nE, wl.c_I, dtype=kvdt, device=device)
+        self.idx = torch.empty(B * T, wl.topk, dtype=torch.int32, device=device)
+        self.out = torch.empty(B * T, wl.n_h, wl.c, dtype=kvdt, device=device)
+        self.win_pos0 = torch.zeros(B, dtype=torch.int32, device=device)
+        self.ws_c = torch.empty(bd.compress_workspace_bytes(self.p, B, T, wl.d), dtype=torch.uint8,
+                                device=device)
+        self.ws_i = torch.empty(bd.index_topk_workspace_bytes(self.p, B, T, nE), dtype=torch.uint8,
+                                device=device)
+        self.ws_a = torch.empty(max(bd.attend_workspace_bytes(self.p, B, T, nE), 1),
+                                dtype=torch.uint8, device=device)
+
+    def run(self, H=None, q=None, qI=None, w=None):
+        i = self.inp
+        H = i["H"] if H is None else H
+        bd.csa_compress(self.p, H, self.packed, self.ckv, None, self.kI, self.win, None,
+                        workspace=self.ws_c)
+        bd.csa_index_topk(self.p, i["q_pos"], i["qI"] if qI is None else qI,
+                          i["w"] if w is None else w, self.kI, self.idx, workspace=self.ws_i)
+        bd.csa_attend(self.p, i["q_pos"], i["q"] if q is None else q, self.idx, self.ckv, None,
+                      self.win, None, self.win_pos0, i["sink"], self.out, workspace=self.ws_a)
+
+    def step_inputs(self):
+        i = self.inp
+        return {k: i[k] for k in ("H", "q", "qI", "w", "q_pos")}
+
+    def units(self):
+        return self.wl.B * self.wl.T  # tokens per step
+
+    def flops(self):
+        """Algorithmic FLOPs of one step (compress GEMM + indexer + attention)."""
+        wl, T, m = self.wl, self.wl.T, self.wl.m
+        ncols = 4 * wl.c + 4 * wl.c_I
+        comp = 2.0 * T * wl.d * ncols
+        pairs = sum(min(self.nE, (t + 1) // m) for t in range(T))
+        index = 2.0 * pairs * wl.n_hI * wl.c_I
+        keys = sum(min(wl.topk, min(self.nE, (t + 1) // m)) + min(wl.n_win, t + 1) for t in range(T))
+        attn = 4.0 * keys * wl.n_h * wl.c
+        return comp, index, attn
+
+    def dominant(self):
+        comp, index, attn = self.flops()
+        return "attend", attn, "attend_tc.cu", "tensor"
+
+
 # -------------------------------------------------------------------- main --
 def run_ours(args, world, rank, local):
     from long_context_sparse_09_b200 import build
@@ -253,9 +314,7 @@ def run_ours(args, world, rank, local):
         wl = wl.with_(T=args.context)
     dev = torch.device(f"cuda:{local}")
     torch.manual_seed(0)
-    if wl.mode != "decode":
-        raise SystemExit("prefill benchmarking: use --workload with a decode workload for now")
-    step = DecodeStep(wl, dev, seed_offset=rank)
+    step = (DecodeStep if wl.mode == "decode" else PrefillStep)(wl, dev, seed_offset=rank)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         step.run()
@@ -308,7 +367,10 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         for k, v in host_in.items():
             dev_in[k].copy_(v, non_blocking=True)
-        step.run(q=dev_in["q"], qI=dev_in.get("qI"), w=dev_in.get("w"))
+        kw = {"q": dev_in["q"], "qI": dev_in.get("qI"), "w": dev_in.get("w")}
+        if "H" in dev_in:
+            kw["H"] = dev_in["H"]
+        step.run(**kw)
         host_out.copy_(step.out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -327,7 +389,7 @@ def run_ours(args, world, rank, local):
     kms, kcnt = prof.get(kind, (0.0, 0))  # one replay: kcnt launches of the kernel
     hbm, tfl, peak_src = _peaks()
     roof = None
-    if kcnt:
+    if kcnt and bound == "hbm":
         per_launch_ms = kms / kcnt
         achieved = nbytes / (per_launch_ms / 1e3) / 1e9
         tr = NCU_TRAFFIC.get(kind)
@@ -336,12 +398,22 @@ def run_ours(args, world, rank, local):
                 "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": kind,
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
                 "peak_source": peak_src}
+    elif kcnt:
+        per_launch_ms = kms / kcnt
+        achieved = nbytes / (per_launch_ms / 1e3) / 1e12
+        tr = NCU_TRAFFIC.get(kind)
+        traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tfl, "unit": "TFLOP/s",
+                "frac": round(achieved / tfl, 4), "traffic": traffic, "kernel": kind,
+                "algorithmic_flops_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
+                "peak_source": peak_src}
     kernels = {k: {"ms_per_step": round(v[0], 5), "launches": v[1],
                    "share": round(v[0] / max(sum(x[0] for x in prof.values()), 1e-12), 4)}
                for k, v in prof.items() if v[1]}
 
+    unit = "query-tok/s" if wl.mode == "decode" else "tok/s"
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(step, "cpu_baseline"):
         import oracle
         nq, secs, sample = step.cpu_baseline()
         cpu = {"value": round(nq / secs, 4), "unit": "query-tok/s", "cores": oracle.num_threads(),
@@ -349,16 +421,17 @@ def run_ours(args, world, rank, local):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "query-tok/s",
+            "metric": METRIC, "value": round(value, 2), "unit": unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.T,
-                       "entries_per_seq": step.N, "m": wl.m, "topk": wl.topk,
+                       "entries_per_seq": getattr(step, "N", getattr(step, "nE", 0)),
+                       "m": wl.m, "topk": wl.topk,
                        "n_h": wl.n_h, "c": wl.c, "kv_format": wl.kv, "n_win": wl.n_win,
                        "l2": "inputs larger than L2 (cache streamed every step)"},
             "e2e": {"value": round(step.units() * world / (e2e_ms / 1e3), 2),
-                    "unit": "query-tok/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 5)},
             "gpu_launches": launches,
             "timing": "CUDA-graph replay of the step; per-kernel times from the last replay",

@@ -630,10 +630,11 @@ void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, 
   const int hbn = (p.n_h + 63) / 64;
   const int base = R * hbn;
   const int nk_max = (dense ? N : p.topk) + p.n_win;
-  int s = (148 + base - 1) / base;
+  // at most one wave of CTAs (148 SMs, one CTA each)
+  const int ntiles = (nk_max + kAtKeys - 1) / kAtKeys;
+  int s = base >= 148 ? 1 : 148 / base;
+  if (s > ntiles) s = ntiles;
   if (s > 256) s = 256;
-  const int max_s = (nk_max + kAtKeys - 1) / kAtKeys;
-  if (s > max_s) s = max_s;
   if (s < 1) s = 1;
   int k = (nk_max + s - 1) / s;
   k = (k + kAtKeys - 1) / kAtKeys * kAtKeys;

@@ -277,6 +277,10 @@ __global__ void __launch_bounds__(256) window_rows(const float* __restrict__ P,
                     win_scale ? win_scale + row : nullptr, red);
 }
 
+bool gemm_tc_supported(int M, int N, int K);
+csa_status launch_gemm_tc(const void* A, const void* B, float* C, int M, int N, int K,
+                          cudaStream_t st);
+
 size_t compress_ws_bytes(const csa_params& p, int B, int T, int d) {
   PackLayout L = pack_layout(p, d);
   return align_up((size_t)B * T * L.ncols * sizeof(float), 256);
@@ -308,7 +312,10 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
   const int M = B * T;
   float* P = (float*)ws;
   dim3 grid((L.ncols + 63) / 64, (M + 63) / 64);
-  if (p.act == CSA_F32)
+  if (p.act == CSA_BF16 && gemm_tc_supported(M, L.ncols, d)) {
+    csa_status s = launch_gemm_tc(H, packed, P, M, L.ncols, d, st);
+    if (s != CSA_OK) return s;
+  } else if (p.act == CSA_F32)
     CSA_LAUNCH(KK_GEMM, st, gemm_nt_simt<float><<<grid, 256, 0, st>>>(
         (const float*)H, (const float*)packed, P, M, L.ncols, d));
   else

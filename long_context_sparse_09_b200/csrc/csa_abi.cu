@@ -253,7 +253,7 @@ csa_status csa_index_topk(const csa_params* p, int B, int Q, const int32_t* q_po
   if (B <= 0 || Q <= 0 || N < 0) return CSA_ERR_SHAPE;
   if (p->c_I % 8 != 0 || p->n_hI > 64) return CSA_ERR_UNSUPPORTED;
   if (!q_pos || !qI || !w || !idx_out || (N > 0 && !kI)) return CSA_ERR_ARG;
-  if (!aligned16(qI) || (kI && !aligned16(kI))) return CSA_ERR_ALIGN;
+  if (!aligned16(qI) || (kI && !aligned16(kI)) || !aligned16(w)) return CSA_ERR_ALIGN;
   const size_t need = index_topk_ws_bytes(*p, B, Q, N);
   if (need > 0 && (workspace == nullptr || ws_bytes < need)) return CSA_ERR_WORKSPACE;
   return launch_index_topk(*p, B, Q, q_pos, qI, w, kI, N, idx_out, score_out, workspace,

@@ -44,9 +44,10 @@ struct IdxTcArgs {
 constexpr int kHistBins = 4096;  // top 12 bits of the order-preserving score key
 
 constexpr int kTileM = 128;
+constexpr int kMaxAcc = 8;  // TMEM accumulator ring depth (bounded by 512 columns)
 constexpr int kKBlockBytes = kTileM * 128;  // 128 rows x 64 bf16
 
-template <int G, int KB, int S, int NE>
+template <int G, int KB, int S, int NE, int NQ = 2>
 struct IdxTcCfg {
   static constexpr int kStageBytes = KB * kKBlockBytes;
   static constexpr int kThreads = 64 + 32 * NE;
@@ -106,11 +107,11 @@ struct TileCursor {
   }
 };
 
-template <int G, int KB, int S, int NE>
-__global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
+template <int G, int KB, int S, int NE, int NQ>
+__global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
     index_scores_tc(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmQ, IdxTcArgs a) {
-  using Cfg = IdxTcCfg<G, KB, S, NE>;
+  using Cfg = IdxTcCfg<G, KB, S, NE, NQ>;
   const int NROWS = G * a.nhI;  // MMA N: the group's query heads
   const int NCOL = NROWS;       // TMEM columns per accumulator
   const int qslot_bytes = KB * NROWS * 128;
@@ -118,21 +119,24 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* kst = smem;                                  // S stages
-  uint8_t* qsl = kst + S * Cfg::kStageBytes;            // 2 query slots
-  uint64_t* bars = (uint64_t*)(qsl + 2 * qslot_bytes);  // barriers
+  uint8_t* qsl = kst + S * Cfg::kStageBytes;            // NQ query slots
+  uint64_t* bars = (uint64_t*)(qsl + NQ * qslot_bytes);  // barriers
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + S;
   uint64_t* qfull = bars + 2 * S;
   uint64_t* qempty = qfull + 2;
   uint64_t* tfull = qempty + 2;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tbase_sm = (uint32_t*)(tempty + 2);
+  uint64_t* tempty = tfull + kMaxAcc;
+  uint32_t* tbase_sm = (uint32_t*)(tempty + kMaxAcc);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
-  unsigned* shist = (unsigned*)((uint8_t*)bars + 256);  // [kHistBins] when G == 1
+  unsigned* shist = (unsigned*)((uint8_t*)bars + 512);  // [kHistBins] when G == 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int ncols_alloc = 32;
-  while (ncols_alloc < 2 * NCOL) ncols_alloc <<= 1;
+  // as many TMEM accumulators as fit (up to 8): more products in flight
+  // hide the latency of each tile's chain of dependent MMAs
+  int nacc = 512 / NCOL;
+  if (nacc > kMaxAcc) nacc = kMaxAcc;
+  const int ncols_alloc = 512;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -142,6 +146,8 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qfull[i], 1);
       mbar_init(&qempty[i], 1);
+    }
+    for (int i = 0; i < kMaxAcc; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], NE);
     }
@@ -173,8 +179,8 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
       int kn = 0, qn = 0;
       for (int i = 0; i < count; ++i) {
         if (cur.first(i)) {
-          const int slot = qn & 1;
-          if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_sm)) break;
+          const int slot = qn % NQ;
+          if (!mbar_wait(&qempty[slot], ((qn / NQ) & 1) ^ 1, abort_sm)) break;
           mbar_expect_tx(&qfull[slot], (uint32_t)qslot_bytes);
           uint8_t* dst = qsl + slot * qslot_bytes;
           for (int kb = 0; kb < KB; ++kb)
@@ -201,12 +207,12 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
       int kn = 0, qn = 0, an = 0;
       for (int i = 0; i < count; ++i) {
         const bool first = cur.first(i), last = cur.last(a.prefix);
-        const int slot = qn & 1;
-        if (first && !mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_sm)) break;
+        const int slot = qn % NQ;
+        if (first && !mbar_wait(&qfull[slot], (qn / NQ) & 1, abort_sm)) break;
         const int s = kn % S;
         if (!mbar_wait(&kfull[s], (kn / S) & 1, abort_sm)) break;
-        const int acc = an & 1;
-        if (!mbar_wait(&tempty[acc], ((an >> 1) & 1) ^ 1, abort_sm)) break;
+        const int acc = an % nacc;
+        if (!mbar_wait(&tempty[acc], ((an / nacc) & 1) ^ 1, abort_sm)) break;
         tc_fence_after();
         const uint32_t abase = smem_u32(kst + s * Cfg::kStageBytes);
         const uint32_t bbase = smem_u32(qsl + slot * qslot_bytes);
@@ -243,6 +249,8 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
       TileCursor cur;
       cur.init(a.prefix, a.ngroups, start, count);
       int an = 0, hist_r = cur.g;
+      float wreg[G == 1 ? 64 : 1];
+      int w_r = -1;
       for (int i = 0; i < count; ++i) {
         if (hist && cur.g != hist_r) {  // query changed: flush its histogram
           named_bar(2, 32 * NE);
@@ -256,26 +264,66 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE>::kThreads, 1)
           named_bar(2, 32 * NE);
           hist_r = cur.g;
         }
-        const int acc = an & 1;
-        if (!mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm)) break;
+        const int acc = an % nacc;
+        if (!mbar_wait(&tfull[acc], (an / nacc) & 1, abort_sm)) break;
         tc_fence_after();
         const int s = cur.t * kTileM + quad * 32 + lane;
         float sc[G];
 #pragma unroll
         for (int qi = 0; qi < G; ++qi) sc[qi] = 0.f;
         const uint32_t trow = tbase + ((uint32_t)(quad * 32) << 16) + acc * NCOL;
+        if (G == 1 && a.nhI == 64) {
+          // one query per group: its 64 head weights stay in registers
+          if (cur.g != w_r) {
+            const float4* w4 = reinterpret_cast<const float4*>(a.w + (size_t)cur.g * 64);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float4 t = __ldg(w4 + j);
+              wreg[4 * j] = t.x; wreg[4 * j + 1] = t.y; wreg[4 * j + 2] = t.z; wreg[4 * j + 3] = t.w;
+            }
+            w_r = cur.g;
+          }
+          float v[4][16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(trow + q4 * 16, v[q4]);
+          tmem_wait_ld();
+          float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              part[q4] = fmaf(wreg[16 * q4 + j], fmaxf(v[q4][j], 0.f), part[q4]);
+          sc[0] = (part[0] + part[1]) + (part[2] + part[3]);
+        } else {
         for (int qq = 0; qq < nq_mine; ++qq) {
           const int qi = q0 + qq;
           const float* wr = a.w + (size_t)(cur.g * G + qi) * a.nhI;
-          float acc_s = 0.f;
-          for (int c0 = 0; c0 < a.nhI; c0 += 16) {
-            float v[16];
-            tmem_ld16(trow + qi * a.nhI + c0, v);
+          // four independent partial sums over the heads (16 heads per
+          // TMEM load); all loads of a 64-head block issued before one wait
+          float part[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int c0 = 0; c0 < a.nhI; c0 += 64) {
+            const int nb = min(64, a.nhI - c0) / 16;
+            float v[4][16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              if (q4 < nb) tmem_ld16(trow + qi * a.nhI + c0 + q4 * 16, v[q4]);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc_s = fmaf(__ldg(wr + c0 + j), fmaxf(v[j], 0.f), acc_s);
+            for (int q4 = 0; q4 < 4; ++q4) {
+              if (q4 >= nb) continue;
+              const float4* w4 = reinterpret_cast<const float4*>(wr + c0 + q4 * 16);
+#pragma unroll
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 ww = __ldg(w4 + j4);
+                part[q4] = fmaf(ww.x, fmaxf(v[q4][4 * j4 + 0], 0.f), part[q4]);
+                part[q4] = fmaf(ww.y, fmaxf(v[q4][4 * j4 + 1], 0.f), part[q4]);
+                part[q4] = fmaf(ww.z, fmaxf(v[q4][4 * j4 + 2], 0.f), part[q4]);
+                part[q4] = fmaf(ww.w, fmaxf(v[q4][4 * j4 + 3], 0.f), part[q4]);
+              }
+            }
           }
-          sc[qq] = acc_s;
+          sc[qq] = (part[0] + part[1]) + (part[2] + part[3]);
+        }
         }
         tc_fence_before();
         __syncwarp();
@@ -364,14 +412,14 @@ int index_tc_group(const csa_params& p, int Q) {
 
 size_t index_tc_plan_bytes(int ngroups) { return align_up((size_t)(ngroups + 1) * 4, 256); }
 
-template <int G, int KB, int S, int NE>
+template <int G, int KB, int S, int NE, int NQ = 2>
 static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
                               const IdxTcArgs& a, cudaStream_t st) {
-  using Cfg = IdxTcCfg<G, KB, S, NE>;
+  using Cfg = IdxTcCfg<G, KB, S, NE, NQ>;
   const int NROWS = G * a.nhI;
-  size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + 2 * (size_t)KB * NROWS * 128 + 256 +
+  size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + NQ * (size_t)KB * NROWS * 128 + 512 +
                 (G == 1 ? kHistBins * 4 : 0);
-  auto kern = index_scores_tc<G, KB, S, NE>;
+  auto kern = index_scores_tc<G, KB, S, NE, NQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
@@ -405,7 +453,7 @@ csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32
   if (a.err == nullptr) return CSA_ERR_CUDA;
   *hist_done = a.ghist != nullptr;
   const bool k2 = p.c_I == 128;
-  if (G == 1) return k2 ? launch_tc_t<1, 2, 5, 4>(tmK, tmQ, a, st) : launch_tc_t<1, 1, 8, 4>(tmK, tmQ, a, st);
+  if (G == 1) return k2 ? launch_tc_t<1, 2, 6, 4, 1>(tmK, tmQ, a, st) : launch_tc_t<1, 1, 8, 4>(tmK, tmQ, a, st);
   if (G == 2) return k2 ? launch_tc_t<2, 2, 4, 4>(tmK, tmQ, a, st) : launch_tc_t<2, 1, 6, 4>(tmK, tmQ, a, st);
   return k2 ? launch_tc_t<4, 2, 2, 8>(tmK, tmQ, a, st) : launch_tc_t<4, 1, 4, 8>(tmK, tmQ, a, st);
 }
