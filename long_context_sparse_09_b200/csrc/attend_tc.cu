@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kfull[i], FP8 ? 128 : 1);
+      mbar_init(&kfull[i], 128);
       mbar_init(&kempty[i], 1);
       mbar_init(&sfull[i], 1);
       mbar_init(&sfree[i], 4);
@@ -178,97 +178,96 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const size_t rb = FP8 ? 576 : 1024;  // stored row bytes
 
   if (ntiles > 0) {
-    if (!FP8 && warp == 0) {
-      // --------------------------------------------- key loads by TMA (bf16) --
-      // Contiguous runs (HCA entries, window rows) come in as 64-row boxes;
-      // selected rows as 4-row gathers; a tile that straddles the entry and
-      // window lists, or a 4-key group of mixed origin, takes one-row loads.
-      // Absent keys read an in-range row (the sequence's first), masked out.
+    if (!FP8 && warp < 4) {
+      // ----------------------------------------------------- key loads (bf16) --
+      // Contiguous 64-key runs (HCA entries, window rows) come in as TMA
+      // boxes; selected rows are gathered with 16-byte loads, 16 in flight
+      // per thread, and stored into the swizzled tile.
+      const int t = threadIdx.x;
+      __shared__ int s_mode, s_row0;
       const int wp0 = a.win ? a.win_pos0[b] : 0;
-      const int crow_oob = min(b * a.N, a.R_rows_c - 1), wrow_oob = min(b * a.W, a.R_rows_w - 1);
+      const uint8_t* ckv = a.ckv + (size_t)b * a.N * rb;
+      const uint8_t* win = a.win + (size_t)b * a.W * rb;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i & 1;
         if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
         const int j0 = j_begin + i * kAtKeys;
-        int row[2], inwin[2], valid[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int j = j0 + lane + 32 * h2;
-          row[h2] = crow_oob;
-          inwin[h2] = 0;
-          valid[h2] = 0;
+        if (t < kAtKeys) {
+          const int j = j0 + t;
+          int valid = 0;
+          const int inwin = j >= n_main;
+          const uint8_t* row = nullptr;
           if (j < j_end) {
             if (j < n_main) {
               const int e = a.dense ? j : a.idx[(size_t)r * a.topk + j];
               if (e >= 0) {
                 if (e < nv) {
-                  valid[h2] = 1;
-                  row[h2] = b * a.N + e;
+                  valid = 1;
+                  row = ckv + (size_t)e * rb;
                 } else {
                   atomicOr(a.err, CSA_DEV_BAD_INDEX);
                 }
               }
             } else {
-              inwin[h2] = 1;
-              row[h2] = wrow_oob;
               const int wr = lo + (j - n_main) - wp0;
               if (a.win != nullptr && wr >= 0 && wr < a.W) {
-                valid[h2] = 1;
-                row[h2] = b * a.W + wr;
+                valid = 1;
+                row = win + (size_t)wr * rb;
               } else {
                 atomicOr(a.err, CSA_DEV_BAD_WINDOW);
               }
             }
-          } else if (j >= n_main) {
-            inwin[h2] = 1;
-            row[h2] = wrow_oob;
           }
-          meta_scale[s * 64 + lane + 32 * h2] = 1.f;
+          row_sm[t] = row;
+          meta_scale[s * 64 + t] = 1.f;
+          const unsigned vb = __ballot_sync(0xffffffffu, valid);
+          if ((t & 31) == 0) reinterpret_cast<unsigned*>(&meta_mask[s])[t >> 5] = vb;
+          (void)inwin;
         }
-        const unsigned m0 = __ballot_sync(0xffffffffu, valid[0]);
-        const unsigned m1 = __ballot_sync(0xffffffffu, valid[1]);
-        if (lane == 0) meta_mask[s] = ((unsigned long long)m1 << 32) | m0;
-        const unsigned w0 = __ballot_sync(0xffffffffu, inwin[0]);
-        const unsigned w1 = __ballot_sync(0xffffffffu, inwin[1]);
+        named_bar(1, 128);
+        if (t == 0) {
+          // whole tile contiguous in one tensor? (entries: dense; window)
+          bool ent = true, wnd = true;
+          for (int u = 0; u < kAtKeys; ++u) {
+            const int j = j0 + u;
+            if (j >= n_main) ent = false; else wnd = false;
+          }
+          s_mode = (a.dense && ent) ? 1 : (wnd ? 2 : 0);
+          s_row0 = s_mode == 1 ? b * a.N + j0 : b * a.W + lo + (j0 - n_main) - wp0;
+        }
+        named_bar(1, 128);
         uint8_t* dstK = sK + s * kKBytes;
-        if (lane == 0) mbar_expect_tx(&kfull[s], kKBytes);
-        __syncwarp();
-        const bool all_entry = (w0 | w1) == 0u, all_win = (w0 & w1) == 0xffffffffu;
-        if (a.dense && all_entry) {  // contiguous entries s = j0 .. j0+63
-          if (lane < 8)
-            tma_load_2d(dstK + lane * 8192, &km.c_box, &kfull[s], lane * 64, b * a.N + j0);
-        } else if (all_win) {  // contiguous window rows
-          const int wr0 = b * a.W + lo + (j0 - n_main) - wp0;
-          if (lane < 8) tma_load_2d(dstK + lane * 8192, &km.w_box, &kfull[s], lane * 64, wr0);
+        const int mode = s_mode;
+        if (mode != 0) {
+          if (t == 0) mbar_expect_tx(&kfull[s], kKBytes);
+          __syncwarp();
+          if (t < 8)
+            tma_load_2d(dstK + t * 8192, mode == 1 ? &km.c_box : &km.w_box, &kfull[s], t * 64,
+                        s_row0);
+          if (t != 0) mbar_arrive(&kfull[s]);
         } else {
-          // lane l: 4-key group g = l & 15, K-blocks 4*(l >> 4) .. +3
-          const int g = lane & 15;
-          int gr[4], gw = 0;
+#pragma unroll 1
+          for (int it0 = 0; it0 < 32; it0 += 16) {
+            uint4 v[16];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int k = 4 * g + u;
-            const int r0 = __shfl_sync(0xffffffffu, row[0], k & 31);
-            const int r1 = __shfl_sync(0xffffffffu, row[1], k & 31);
-            gr[u] = k < 32 ? r0 : r1;
+            for (int u = 0; u < 16; ++u) {
+              const int idx = (it0 + u) * 128 + t;
+              const int key = idx >> 6, ch = idx & 63;
+              const uint8_t* src = row_sm[key];
+              v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const int idx = (it0 + u) * 128 + t;
+              const int key = idx >> 6, ch = idx & 63;
+              const int kb = ch >> 3, c = ch & 7;
+              st_shared16(dstK + kb * 8192 + key * 128 + ((c ^ (key & 7)) << 4), v[u]);
+            }
           }
-          const unsigned wbits = (w0 >> (4 * (g & 7))) & 0xFu;  // keys 4g..4g+3 (g < 8)
-          const unsigned wbits_hi = (w1 >> (4 * (g & 7))) & 0xFu;
-          gw = g < 8 ? (int)wbits : (int)wbits_hi;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int kb = 4 * (lane >> 4) + q4;
-            uint8_t* dst = dstK + kb * 8192 + g * 4 * 128;
-            if (gw == 0)
-              tma_gather4(dst, &km.c_row, &kfull[s], kb * 64, gr[0], gr[1], gr[2], gr[3]);
-            else if (gw == 0xF)
-              tma_gather4(dst, &km.w_row, &kfull[s], kb * 64, gr[0], gr[1], gr[2], gr[3]);
-            else
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                tma_load_2d(dst + u * 128, ((gw >> u) & 1) ? &km.w_row : &km.c_row, &kfull[s],
-                            kb * 64, gr[u]);
-          }
+          fence_proxy_async_smem();
+          mbar_arrive(&kfull[s]);
         }
+        named_bar(1, 128);  // row_sm and the mode are rewritten by the next tile
       }
     } else if (FP8 && warp < 4) {
       // ------------------------------------------- key gather (FP8-mixed) --
@@ -380,7 +379,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (ok) ok = issue_qk(0);
         for (int i = 0; ok && i < ntiles; ++i) {
           const int s = i & 1, bb = i & 1;
-          if (i + 1 < ntiles && !issue_qk(i + 1)) break;  // overlaps softmax(i)
+          // QK(i+1) early only if its tile and S buffer are already there;
+          // P V(i) must not wait behind a late tile
+          bool qk_next = false;
+          if (i + 1 < ntiles && mbar_try_wait(&kfull[(i + 1) & 1], ((i + 1) >> 1) & 1) &&
+              mbar_try_wait(&sfree[(i + 1) & 1], (((i + 1) >> 1) & 1) ^ 1)) {
+            if (!issue_qk(i + 1)) break;
+            qk_next = true;
+          }
           if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort_sm)) break;
           tc_fence_after();
           const uint32_t kbase = smem_u32(sK + s * kKBytes);
@@ -406,6 +412,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           }
           mma_commit(&kempty[s]);
           mma_commit(&pvdone[bb]);
+          if (i + 1 < ntiles && !qk_next && !issue_qk(i + 1)) break;
         }
       }
     } else if (warp >= 5) {
