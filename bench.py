@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from long_context_sparse_09_b200 import binding as bd  # noqa: E402
+from long_context_sparse_09_b200 import dist as D  # noqa: E402
 from long_context_sparse_09_b200 import synth  # noqa: E402
 from long_context_sparse_09_b200.configs import DEFAULT_BENCH, WORKLOADS  # noqa: E402
 
@@ -41,7 +42,11 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 # ncu DRAM traffic per launch of the dominant kernel, with the hash of the
 # source file it was measured on (the value is dropped once the file changes).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --set full, pro_csa_decode_1m with 2 sequences (138.73 MB read+write),
+    # scaled by the units of a full launch (4 sequences)
+    "index_scores": (277.47e6, "eb1adcb86a1f"),
+}
 
 
 # ------------------------------------------------------------------ utils --
@@ -111,30 +116,18 @@ class ClockSampler:
 
 
 def _dist():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device(f"cuda:{local}"))
-    else:
-        torch.cuda.set_device(local)
+    world, rank, local = D.world()
+    torch.cuda.set_device(local)
+    D.init("nccl")
     return world, rank, local
 
 
 def _barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
+    D.barrier()
 
 
 def _max_over_ranks(x, world):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return D.max_over_ranks(x, device="cuda")
 
 
 # --------------------------------------------------------------- workloads --
@@ -144,7 +137,8 @@ class DecodeStep:
     def __init__(self, wl, device, seed_offset=0):
         self.wl = wl
         self.p = bd.params_for(wl)
-        inp = synth.decode_inputs(wl.with_(seed=wl.seed + seed_offset), device=device)
+        inp = synth.decode_inputs(wl.with_(seed=wl.seed + D.seed_offset(seed_offset)),
+                                  device=device)
         self.inp = inp
         B, N = wl.B, inp["N"]
         self.N = N
@@ -185,10 +179,10 @@ class DecodeStep:
         wl, B, N = self.wl, self.wl.B, self.N
         if wl.variant == "csa":
             nbytes = B * N * wl.c_I * 2 + B * wl.n_hI * (wl.c_I * 2 + 4) + B * 4
-            return "index_scores", nbytes, "index_topk.cu", "hbm"
+            return "index_scores", nbytes, "index_tc.cu", "hbm"
         rb = synth.kv_record_bytes(wl)
         nbytes = B * (N + wl.n_win) * rb + 2 * B * wl.n_h * wl.c * 2
-        return "attend", nbytes, "attend.cu", "hbm"
+        return "attend", nbytes, "attend_tc.cu", "hbm"
 
     def cpu_baseline(self, max_queries=None):
         """Oracle (as it stands) on the queries of one step; returns
@@ -495,8 +489,7 @@ def main():
         else:
             run_ours(args, world, rank, local)
     finally:
-        if world > 1:
-            torch.distributed.destroy_process_group()
+        D.finalize()
 
 
 if __name__ == "__main__":
