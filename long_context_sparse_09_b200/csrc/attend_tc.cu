@@ -50,6 +50,7 @@ struct AttnTcArgs {
   unsigned* err;
   int Q, N, W, n_h, m, topk, n_win, nsplit, keys_per_split, dense, R, hblocks;
   int R_rows_c, R_rows_w;  // total rows of the cache / window tensors (out of range)
+  int box_rows;            // rows of one output box: min(64, n_h)
   float scale2;  // softmax scale times log2(e): the softmax runs in base 2
   double base;
 };
@@ -108,9 +109,11 @@ __device__ __forceinline__ void widen_e4m3(uint4 raw, uint4& lo, uint4& hi) {
 }
 
 // Key-row tensor maps (bf16 caches): boxes of 64 columns x 64 rows for
-// contiguous key runs, and of 64 x 1 rows for gathers of selected rows.
+// contiguous key runs, and of 64 x 1 rows for gathers of selected rows; and
+// the output maps: bf16 O [R*n_h][512] and fp32 split partials
+// [S*R*n_h][512], both in 128-byte boxes of box_rows rows.
 struct KeyMaps {
-  CUtensorMap c_box, c_row, w_box, w_row;
+  CUtensorMap c_box, c_row, w_box, w_row, o_out, o_ws;
 };
 
 template <bool FP8>
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint32_t* tbase_sm = (uint32_t*)(bars + 13);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
   __shared__ const uint8_t* row_sm[kAtKeys];
+  __shared__ float rope_tab[64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int item = blockIdx.x;
@@ -278,6 +282,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       for (int i = 0; i < ntiles; ++i) {
         const int s = i & 1;
         if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
+        float sc_reg = 1.f;
         if (t < kAtKeys) {
           const int j = j_begin + i * kAtKeys + t;
           int valid = 0;
@@ -307,7 +312,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
           }
           row_sm[t] = valid ? row : nullptr;
-          meta_scale[s * 64 + t] = sc;
+          sc_reg = sc;  // in flight with the row loads below
           const unsigned bits = __ballot_sync(0xffffffffu, valid);
           if ((t & 31) == 0) reinterpret_cast<unsigned*>(&meta_mask[s])[t >> 5] = bits;
         }
@@ -340,6 +345,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             st_shared16(rowp + 7 * 8192 + ((c ^ sw) << 4), v[u]);
           }
         }
+        if (t < kAtKeys) meta_scale[s * 64 + t] = sc_reg;
         fence_proxy_async_smem();
         mbar_arrive(&kfull[s]);
         named_bar(1, 128);  // row_sm is rewritten by the next tile
@@ -531,56 +537,86 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (lane == 0) mbar_arrive(&pfull[bb]);
       }
       // ---------------------------------------------------------- output --
+      // O rows are staged in the idle key buffers (128-byte swizzle) and
+      // written by TMA stores: bf16 O when the slice is the whole key list,
+      // else fp32 partials plus (max, sum) for the combine.
       if (ok && mbar_wait(&pvdone[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_sm)) {
         tc_fence_after();
         const uint32_t orow = trow + ((uint32_t)(16 * half) << 16);
-        const bool store = head < a.n_h;
+        const int brows = a.box_rows;
+        const bool store = hl < brows;  // head < n_h
         const int dim0 = half * 256;
         const bool any = m_used > 0.5f * kMasked;
         float f = 1.f;
         if (a.nsplit == 1) {
+          if (warp == 5) {  // R_{-t0} of the 32 RoPE pairs
+            float cs, sn;
+            rope_cs(-(double)t0, lane, 64, a.base, &cs, &sn);
+            rope_tab[2 * lane] = cs;
+            rope_tab[2 * lane + 1] = sn;
+          }
           const float zs = store ? a.sink[head] * kLog2e : 0.f;
           const float M = fmaxf(any ? m_used : zs, zs);
           const float em = any ? fast_exp2(m_used - M) : 0.f;
           f = em / (l * em + fast_exp2(zs - M));
+          named_bar(2, 128);
         }
+        uint8_t* stage = sK;  // 2 x 64 KB, free once the last P V is done
+        const int box_bytes = brows * 128;
+        const int sw = hl & 7;
         for (int c0 = 0; c0 < 256; c0 += 64) {
           float v[64];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            float w16[16];
-            tmem_ld16(orow + c0 + q4 * 16, w16);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) v[q4 * 16 + u] = w16[u];
-          }
+          for (int q4 = 0; q4 < 4; ++q4)
+            tmem_ld16(orow + c0 + q4 * 16, *reinterpret_cast<float(*)[16]>(v + q4 * 16));
           tmem_wait_ld();
           if (!store) continue;
+          const int d0 = dim0 + c0;
           if (a.nsplit == 1) {
 #pragma unroll
             for (int u = 0; u < 64; ++u) v[u] *= f;
-            if (dim0 + c0 >= 448) {  // RoPE dims: apply R_{-t0}
+            if (d0 >= 448) {  // RoPE dims
 #pragma unroll
               for (int u = 0; u < 64; u += 2) {
-                float cs, sn;
-                rope_cs(-(double)t0, (dim0 + c0 + u - 448) >> 1, 64, a.base, &cs, &sn);
+                const float cs = rope_tab[u], sn = rope_tab[u + 1];
                 const float x0 = v[u], x1 = v[u + 1];
                 v[u] = x0 * cs - x1 * sn;
                 v[u + 1] = x0 * sn + x1 * cs;
               }
             }
-            __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + head) * 512 + dim0 + c0;
+            uint8_t* rowp = stage + (d0 >> 6) * box_bytes + hl * 128;
 #pragma unroll
-            for (int u = 0; u < 64; u += 8)
-              *reinterpret_cast<uint4*>(dst + u) =
-                  make_uint4(pack_bf16(v[u], v[u + 1]), pack_bf16(v[u + 2], v[u + 3]),
-                             pack_bf16(v[u + 4], v[u + 5]), pack_bf16(v[u + 6], v[u + 7]));
+            for (int cc = 0; cc < 8; ++cc) {
+              const float* x = v + 8 * cc;
+              st_shared16(rowp + ((cc ^ sw) << 4),
+                          make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7])));
+            }
           } else {
-            const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
-            float* dst = a.ws_o + slot * 512 + dim0 + c0;
 #pragma unroll
-            for (int u = 0; u < 64; u += 4)
-              *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              uint8_t* rowp = stage + ((d0 >> 5) + h2) * box_bytes + hl * 128;
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                const float* x = v + 32 * h2 + 4 * cc;
+                *reinterpret_cast<float4*>(rowp + ((cc ^ sw) << 4)) =
+                    make_float4(x[0], x[1], x[2], x[3]);
+              }
+            }
           }
+        }
+        fence_proxy_async_smem();
+        named_bar(2, 128);
+        if (threadIdx.x == 160) {
+          if (a.nsplit == 1) {
+            const int row0 = r * a.n_h + hb * 64;
+            for (int bx = 0; bx < 8; ++bx) tma_store_2d(&km.o_out, stage + bx * box_bytes, bx * 64, row0);
+          } else {
+            const int row0 = (sp * a.R + r) * a.n_h + hb * 64;
+            for (int bx = 0; bx < 16; ++bx) tma_store_2d(&km.o_ws, stage + bx * box_bytes, bx * 32, row0);
+          }
+          bulk_commit();
+          bulk_wait_all();
         }
         if (store && a.nsplit > 1 && half == 0) {  // natural-log max for the combine
           const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
@@ -625,6 +661,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 // ------------------------------------------------------------------ host --
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows);
 bool tma_available();
 
 bool attend_tc_supported(const csa_params& p) {
@@ -689,6 +727,12 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
     a.R_rows_c = (int)crows;
     a.R_rows_w = (int)wrows;
   }
+  a.box_rows = p.n_h < 64 ? p.n_h : 64;
+  if (!make_tmap_bf16(&km.o_out, out, (uint64_t)R * p.n_h, 512, (uint32_t)a.box_rows))
+    return CSA_ERR_CUDA;
+  if (nsplit > 1 &&
+      !make_tmap_f32(&km.o_ws, ws_o, (uint64_t)nsplit * R * p.n_h, 512, (uint32_t)a.box_rows))
+    return CSA_ERR_CUDA;
   if (p.kv == CSA_KV_FP8MIX) {
     const int smem = AtLayout<true>::total + 1024;
     if (cudaFuncSetAttribute(attend_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=

@@ -34,16 +34,19 @@ using namespace sm100;
 struct IdxTcArgs {
   const int32_t* q_pos;
   const float* w;
-  const int* prefix;  // [ngroups + 1] exclusive prefix of tiles per group
+  const int* prefix;  // [ngroups + 1] exclusive prefix of tiles per group, or null:
+                      // each CTA computes it (ngroups <= kInlineGroups)
   float* scores;      // [R][N]
   unsigned* err;
   unsigned* ghist;    // [R][4096] key histograms for the top-k (G == 1), or null
   int Q, N, m, nhI, ngroups;
+  int stream_keys;    // every key tile is read by one group only: read it evict-first
 };
 
 constexpr int kHistBins = 4096;  // top 12 bits of the order-preserving score key
 
 constexpr int kTileM = 128;
+constexpr int kInlineGroups = 64;  // groups whose tile prefix a CTA computes itself
 constexpr int kMaxAcc = 8;  // TMEM accumulator ring depth (bounded by 512 columns)
 constexpr int kKBlockBytes = kTileM * 128;  // 128 rows x 64 bf16
 
@@ -89,20 +92,20 @@ struct TileCursor {
     int lo = 0, hi = ngroups;
     while (lo < hi) {  // last g with prefix[g] <= start
       int mid = (lo + hi + 1) >> 1;
-      if (__ldg(prefix + mid) <= start) lo = mid; else hi = mid - 1;
+      if (prefix[mid] <= start) lo = mid; else hi = mid - 1;
     }
     g = lo;
-    t = start - __ldg(prefix + g);
+    t = start - prefix[g];
     left = count;
   }
-  __device__ int tiles(const int* prefix) const { return __ldg(prefix + g + 1) - __ldg(prefix + g); }
+  __device__ int tiles(const int* prefix) const { return prefix[g + 1] - prefix[g]; }
   __device__ bool first(int pos_in_cta) const { return t == 0 || pos_in_cta == 0; }
   __device__ bool last(const int* prefix) const { return left == 1 || t + 1 == tiles(prefix); }
   __device__ void next(const int* prefix, int ngroups) {
     --left;
     if (++t >= tiles(prefix)) {
       t = 0;
-      do { ++g; } while (g < ngroups && __ldg(prefix + g + 1) == __ldg(prefix + g));
+      do { ++g; } while (g < ngroups && prefix[g + 1] == prefix[g]);
     }
   }
 };
@@ -112,6 +115,9 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
     index_scores_tc(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmQ, IdxTcArgs a) {
   using Cfg = IdxTcCfg<G, KB, S, NE, NQ>;
+  // one query per group and two warps per TMEM lane quadrant: the two
+  // epilogue warp groups take alternate tiles
+  constexpr bool kAlt = G == 1 && NE == 8;
   const int NROWS = G * a.nhI;  // MMA N: the group's query heads
   const int NCOL = NROWS;       // TMEM columns per accumulator
   const int qslot_bytes = KB * NROWS * 128;
@@ -130,6 +136,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
   uint32_t* tbase_sm = (uint32_t*)(tempty + kMaxAcc);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
   unsigned* shist = (unsigned*)((uint8_t*)bars + 512);  // [kHistBins] when G == 1
+  int* s_prefix = (int*)((uint8_t*)bars + 512 + (G == 1 ? kHistBins * 4 : 0));  // [65]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // as many TMEM accumulators as fit (up to 8): more products in flight
@@ -149,7 +156,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
     }
     for (int i = 0; i < kMaxAcc; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], NE);
+      mbar_init(&tempty[i], kAlt ? 4 : NE);
     }
     *abort_sm = 0;
     fence_mbar_init();
@@ -167,7 +174,30 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tbase_sm;
 
-  const int total = __ldg(a.prefix + a.ngroups);
+  if (a.prefix == nullptr) {
+    // tiles of each group (threads 0..63) and their prefix: two warp scans
+    if (threadIdx.x < kInlineGroups) {
+      const int g = threadIdx.x;
+      int tiles = 0;
+      if (g < a.ngroups) {
+        int nv = 0;
+        for (int i = 0; i < G; ++i) nv = max(nv, n_visible(__ldg(a.q_pos + g * G + i), a.m, a.N));
+        tiles = (nv + kTileM - 1) / kTileM;
+      }
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, tiles, o);
+        if (lane >= o) tiles += y;
+      }
+      s_prefix[g + 1] = tiles;
+      if (g == 0) s_prefix[0] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32 && threadIdx.x < kInlineGroups) s_prefix[threadIdx.x + 1] += s_prefix[32];
+    __syncthreads();
+  }
+  const int* prefix = a.prefix ? a.prefix : s_prefix;
+  const int total = prefix[a.ngroups];
   const int start = (int)((long long)total * blockIdx.x / gridDim.x);
   const int count = (int)((long long)total * (blockIdx.x + 1) / gridDim.x) - start;
 
@@ -175,7 +205,8 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------- producer --
       TileCursor cur;
-      cur.init(a.prefix, a.ngroups, start, count);
+      cur.init(prefix, a.ngroups, start, count);
+      const uint64_t pol = l2_evict_first_policy();
       int kn = 0, qn = 0;
       for (int i = 0; i < count; ++i) {
         if (cur.first(i)) {
@@ -193,20 +224,24 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
         mbar_expect_tx(&kfull[s], (uint32_t)Cfg::kStageBytes);
         const int b = (cur.g * G) / a.Q;
         const int row = b * a.N + cur.t * kTileM;
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_2d(kst + s * Cfg::kStageBytes + kb * kKBlockBytes, &tmK, &kfull[s], kb * 64,
-                      row);
+        for (int kb = 0; kb < KB; ++kb) {
+          uint8_t* dst = kst + s * Cfg::kStageBytes + kb * kKBlockBytes;
+          if (a.stream_keys)
+            tma_load_2d_hint(dst, &tmK, &kfull[s], kb * 64, row, pol);
+          else
+            tma_load_2d(dst, &tmK, &kfull[s], kb * 64, row);
+        }
         ++kn;
-        cur.next(a.prefix, a.ngroups);
+        cur.next(prefix, a.ngroups);
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA --
       TileCursor cur;
-      cur.init(a.prefix, a.ngroups, start, count);
+      cur.init(prefix, a.ngroups, start, count);
       const uint32_t idesc = idesc_bf16(kTileM, NROWS);
       int kn = 0, qn = 0, an = 0;
       for (int i = 0; i < count; ++i) {
-        const bool first = cur.first(i), last = cur.last(a.prefix);
+        const bool first = cur.first(i), last = cur.last(prefix);
         const int slot = qn % NQ;
         if (first && !mbar_wait(&qfull[slot], (qn / NQ) & 1, abort_sm)) break;
         const int s = kn % S;
@@ -232,14 +267,15 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
         }
         ++kn;
         ++an;
-        cur.next(a.prefix, a.ngroups);
+        cur.next(prefix, a.ngroups);
       }
     } else if (warp >= 2) {
       // ------------------------------------------------------- epilogue --
       const int e = warp - 2;
       const int quad = warp & 3;         // TMEM lane quadrant of this warp
-      const int nq_mine = NE == 4 ? G : G / 2;
-      const int q0 = NE == 4 ? 0 : (e >> 2) * (G / 2);
+      const int nq_mine = (NE == 4 || kAlt) ? G : G / 2;
+      const int q0 = (NE == 4 || kAlt) ? 0 : (e >> 2) * (G / 2);
+      const int alt = e >> 2;  // kAlt: this warp group's tile parity
       const bool hist = G == 1 && a.ghist != nullptr;
       const int et = threadIdx.x - 64;  // 0 .. 32*NE-1
       if (hist) {
@@ -247,7 +283,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
         named_bar(2, 32 * NE);
       }
       TileCursor cur;
-      cur.init(a.prefix, a.ngroups, start, count);
+      cur.init(prefix, a.ngroups, start, count);
       int an = 0, hist_r = cur.g;
       float wreg[G == 1 ? 64 : 1];
       int w_r = -1;
@@ -263,6 +299,11 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
           }
           named_bar(2, 32 * NE);
           hist_r = cur.g;
+        }
+        if (kAlt && (an & 1) != alt) {  // the other warp group's tile
+          ++an;
+          cur.next(prefix, a.ngroups);
+          continue;
         }
         const int acc = an % nacc;
         if (!mbar_wait(&tfull[acc], (an / nacc) & 1, abort_sm)) break;
@@ -337,7 +378,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
           }
         }
         ++an;
-        cur.next(a.prefix, a.ngroups);
+        cur.next(prefix, a.ngroups);
       }
       if (hist) {  // flush the last query's histogram
         named_bar(2, 32 * NE);
@@ -396,6 +437,21 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 rows of `cols` floats; boxes of 32 columns (128 bytes) x box_rows rows
+bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tma_available() { return encode_fn() != nullptr; }
 
 bool index_tc_supported(const csa_params& p) {
@@ -418,7 +474,7 @@ static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
   using Cfg = IdxTcCfg<G, KB, S, NE, NQ>;
   const int NROWS = G * a.nhI;
   size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + NQ * (size_t)KB * NROWS * 128 + 512 +
-                (G == 1 ? kHistBins * 4 : 0);
+                (G == 1 ? kHistBins * 4 : 0) + (kInlineGroups + 1) * 4;
   auto kern = index_scores_tc<G, KB, S, NE, NQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -440,20 +496,22 @@ csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32
   const int R = B * Q;
   const int G = index_tc_group(p, Q);
   const int ngroups = R / G;
-  const unsigned zblocks = (unsigned)std::min<size_t>(64, (nzero + 16383) / 16384 + 1);
-  CSA_LAUNCH(KK_PLAN, st, index_plan<<<zblocks, 1024, 0, st>>>(q_pos, G, ngroups, p.m, N, plan,
-                                                               zero_words, nzero));
+  const bool inline_plan = ngroups <= kInlineGroups;
+  if (nzero && cudaMemsetAsync(zero_words, 0, nzero * 4, st) != cudaSuccess) return CSA_ERR_CUDA;
+  if (!inline_plan)
+    CSA_LAUNCH(KK_PLAN, st, index_plan<<<1, 1024, 0, st>>>(q_pos, G, ngroups, p.m, N, plan,
+                                                           nullptr, 0));
   *hist_done = false;
   if (N == 0) return last_launch_status();
   CUtensorMap tmK, tmQ;
   if (!make_tmap_bf16(&tmK, kI, (uint64_t)B * N, p.c_I, kTileM)) return CSA_ERR_CUDA;
   if (!make_tmap_bf16(&tmQ, qI, (uint64_t)R * p.n_hI, p.c_I, G * p.n_hI)) return CSA_ERR_CUDA;
-  IdxTcArgs a{q_pos, w, plan, scores, device_error_word(), G == 1 ? ghist : nullptr,
-              Q, N, p.m, p.n_hI, ngroups};
+  IdxTcArgs a{q_pos, w, inline_plan ? nullptr : plan, scores, device_error_word(), G == 1 ? ghist : nullptr,
+              Q, N, p.m, p.n_hI, ngroups, Q == G ? 1 : 0};
   if (a.err == nullptr) return CSA_ERR_CUDA;
   *hist_done = a.ghist != nullptr;
   const bool k2 = p.c_I == 128;
-  if (G == 1) return k2 ? launch_tc_t<1, 2, 6, 4, 1>(tmK, tmQ, a, st) : launch_tc_t<1, 1, 8, 4>(tmK, tmQ, a, st);
+  if (G == 1) return k2 ? launch_tc_t<1, 2, 6, 8, 1>(tmK, tmQ, a, st) : launch_tc_t<1, 1, 8, 4>(tmK, tmQ, a, st);
   if (G == 2) return k2 ? launch_tc_t<2, 2, 4, 4>(tmK, tmQ, a, st) : launch_tc_t<2, 1, 6, 4>(tmK, tmQ, a, st);
   return k2 ? launch_tc_t<4, 2, 2, 8>(tmK, tmQ, a, st) : launch_tc_t<4, 1, 4, 8>(tmK, tmQ, a, st);
 }

@@ -163,23 +163,39 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
 }
 
 // ------------------------------------------------- multi-CTA top-k (few q) --
-// For a handful of queries with long visible ranges (decode): (1) every CTA
-// histograms the top 12 key bits of a chunk, (2) every CTA finds the bin T
-// that holds the k-th largest key, marks the entries of higher bins in a
-// bitmap and lists the entries of bin T as candidates, (3) one CTA per query
-// orders the candidates (key desc, index asc), marks the ones still needed
-// and compacts the bitmap into ascending indices.  If bin T overflows the
-// candidate list, (3) falls back to the exact block-wide radix select.
+// For a handful of queries with long visible ranges (decode).  (1) The top 12
+// key bits of every visible score are histogrammed (by the tensor-core
+// scorer's epilogue, or by topk_hist).  (2) Every CTA of the select pass
+// takes a chunk of one query's scores, finds the bin T that holds the k-th
+// largest key, and appends the indices of higher bins to the query's "above"
+// list and the (key, index) pairs of bin T to its candidate list.  (3) The
+// last CTA of the query to finish selects the still needed candidates (radix
+// select over the low 20 key bits, equal keys towards the lower index),
+// marks the above list and the chosen candidates in a shared-memory bitmap
+// of the index range and compacts it into ascending indices.  If bin T
+// overflows the candidate list, (3) falls back to the exact block-wide radix
+// select over all scores.
 constexpr int kBins = 4096;
 constexpr int kChunk = 8192;    // entries per CTA in (1) and (2)
+constexpr int kPer = kChunk / 1024;
 constexpr int kCandCap = 4096;  // candidates per query
+constexpr int kAboveCap = 4096; // entries of bins above T (< k) per query
+constexpr int kLocalCap = 2048; // candidates one select CTA may hold locally
+constexpr int kWinWords = 8192;  // bitmap window of the compaction (262144 entries)
 
 struct MultiTopkWs {
   unsigned* ghist;     // [R][kBins]
-  unsigned* cand_cnt;  // [R]
+  unsigned* cnt;       // [R][2]: candidates, above
   unsigned* done;      // [R] CTAs of the select pass that have finished
-  unsigned* bitmap;    // [R][N32]
-  uint2* cand;         // [R][kCandCap] (key, index)
+  int* above;          // [R][kAboveCap] indices in bins above T
+  uint2* cand;         // [R][kCandCap] (key, index) in bin T
+};
+
+// dynamic shared memory of topk_select_final
+struct SelectSmem {
+  uint2 cand[kCandCap];
+  unsigned bm[kWinWords];  // select pass: local above list; final: bitmap window
+  unsigned char flag[kCandCap];
 };
 
 __global__ void __launch_bounds__(1024) topk_hist(const float* __restrict__ scores, int N,
@@ -228,45 +244,41 @@ __device__ void find_threshold_bin(const unsigned* __restrict__ gh, unsigned k, 
   *above_out = *sAbove;
 }
 
-constexpr int kLocalCap = 2048;  // candidates one select CTA may hold locally
-
-// Exact completion of one query's selection (one CTA): a two-pass radix
-// select over the low 20 key bits of the bin-T candidates (all share the top
-// 12), equal keys resolved towards the lower index, the chosen ones marked
-// in the bitmap, then the bitmap compacted in index order.
-__device__ void finalize_query(const float* __restrict__ sc, int nv, int N, int k, int r,
-                               const MultiTopkWs& ws, int32_t* __restrict__ out,
-                               float* __restrict__ sout, uint2* cand, RadixShared& sh,
-                               int* sT, unsigned* sAbove) {
+// Exact completion of one query's selection (one CTA, 1024 threads), given
+// the bin T of the k-th key and the count of keys above it.
+__device__ void finalize_query(const float* __restrict__ sc, int nv, int k, int r, int T,
+                               unsigned above, const MultiTopkWs& ws, int32_t* __restrict__ out,
+                               float* __restrict__ sout, SelectSmem& S, RadixShared& sh) {
   __shared__ unsigned s_eq_n;
-  __shared__ int s_fallback;
-  if (nv <= k) {
-    write_all_visible(sc, nv, k, out, sout);
-    return;
-  }
-  int T;
-  unsigned above;
-  find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, sT, sAbove);
-  const unsigned nc = __ldcg(ws.cand_cnt + r);
-  if (nc > (unsigned)kCandCap) {  // bin T too crowded: exact block-wide select
+  const unsigned nc = __ldcg(ws.cnt + 2 * r);
+  const unsigned na = __ldcg(ws.cnt + 2 * r + 1);
+  if (nc > (unsigned)kCandCap || na != above) {  // bin T too crowded: exact block-wide select
     radix_select_block(sc, nv, k, out, sout, sh);
     return;
   }
+  // the above list stays in registers (na < k <= kAboveCap)
+  constexpr int kAPer = kAboveCap / 1024;
+  int ab[kAPer];
+#pragma unroll
+  for (int u = 0; u < kAPer; ++u) {
+    const unsigned j = u * 1024u + threadIdx.x;
+    ab[u] = j < na ? __ldcg(ws.above + (size_t)r * kAboveCap + j) : -1;
+  }
   for (int i = threadIdx.x; i < (int)nc; i += blockDim.x)
-    cand[i] = __ldcg(ws.cand + (size_t)r * kCandCap + i);
-  // radix select of the need-th largest key among the candidates
+    S.cand[i] = __ldcg(ws.cand + (size_t)r * kCandCap + i);
+  // radix select of the remaining-th largest key among the candidates
   unsigned remaining = (unsigned)k - above;  // 1 <= remaining <= nc
   unsigned prefix = (unsigned)T << 20, mask = 0xFFF00000u;
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = pass == 0 ? 10 : 0;
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) sh.hist[i] = 0;
+    for (int i = threadIdx.x; i < 1024; i += blockDim.x) sh.hist[i] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
-      const unsigned key = cand[i].x;
+      const unsigned key = S.cand[i].x;
       if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 1023u], 1u);
     }
     __syncthreads();
-    // thread t owns bin 1023 - t (1024 threads): exclusive scan counts higher bins
+    // thread t owns bin 1023 - t: the exclusive scan counts higher bins
     const int bin = 1023 - (int)threadIdx.x;
     const unsigned hcount = sh.hist[bin];
     unsigned tot;
@@ -282,64 +294,71 @@ __device__ void finalize_query(const float* __restrict__ sc, int nv, int N, int 
     __syncthreads();
   }
   const unsigned K = prefix;  // exact key of the k-th largest score
-  // equal keys: the `remaining` lowest indices win
-  if (threadIdx.x == 0) { s_eq_n = 0; s_fallback = 0; }
+  // keys above K are in; of the keys equal to K the `remaining` lowest
+  // indices are in (their candidate slots are listed in sh.hist)
+  if (threadIdx.x == 0) s_eq_n = 0;
   __syncthreads();
-  const int N32 = (N + 31) >> 5;
-  unsigned* bm = ws.bitmap + (size_t)r * N32;
   for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
-    const uint2 c = cand[i];
-    if (c.x > K) {
-      atomicOr(bm + (c.y >> 5), 1u << (c.y & 31));
-    } else if (c.x == K) {
+    const unsigned key = S.cand[i].x;
+    S.flag[i] = key > K;
+    if (key == K) {
       const unsigned p = atomicAdd(&s_eq_n, 1u);
-      if (p < 2048) sh.hist[p] = c.y;  // reuse the histogram as an index list
+      if (p < 2048) sh.hist[p] = (unsigned)i;
     }
   }
   __syncthreads();
   const unsigned neq = s_eq_n;
-  if (neq > 2048) {
-    s_fallback = 1;
-  } else if (neq == remaining) {
-    for (unsigned i = threadIdx.x; i < neq; i += blockDim.x) {
-      const unsigned s = sh.hist[i];
-      atomicOr(bm + (s >> 5), 1u << (s & 31));
-    }
-  } else {
-    // rank each equal-key index among the others (neq is small)
-    for (unsigned i = threadIdx.x; i < neq; i += blockDim.x) {
-      const unsigned s = sh.hist[i];
-      unsigned rank = 0;
-      for (unsigned j = 0; j < neq; ++j) rank += sh.hist[j] < s;
-      if (rank < remaining) atomicOr(bm + (s >> 5), 1u << (s & 31));
-    }
-  }
-  __syncthreads();
-  if (s_fallback) {  // a huge tie: exact block-wide select over all scores
+  if (neq > 2048) {  // a huge tie: exact block-wide select over all scores
     radix_select_block(sc, nv, k, out, sout, sh);
     return;
   }
-  __threadfence();
+  for (unsigned e = threadIdx.x; e < neq; e += blockDim.x) {
+    const unsigned i = sh.hist[e];
+    const unsigned s = S.cand[i].y;
+    unsigned rank = 0;
+    if (neq != remaining)
+      for (unsigned j = 0; j < neq; ++j) rank += S.cand[sh.hist[j]].y < s;
+    S.flag[i] = rank < remaining;
+  }
   __syncthreads();
-  // ordered compaction of the bitmap
-  const int per = (N32 + blockDim.x - 1) / blockDim.x;
-  const int w0 = threadIdx.x * per, w1 = min(N32, w0 + per);
-  unsigned cnt = 0;
-  for (int wi = w0; wi < w1; ++wi) cnt += __popc(__ldcg(bm + wi));
-  unsigned tot;
-  unsigned pos = block_exclusive_scan(cnt, sh.scan, &tot);
-  for (int wi = w0; wi < w1; ++wi) {
-    unsigned word = __ldcg(bm + wi);
-    while (word) {
-      const int bit = __ffs(word) - 1;
-      word &= word - 1;
-      const int s = wi * 32 + bit;
-      if (pos < (unsigned)k) {
-        out[pos] = s;
-        if (sout) sout[pos] = sc[s];
-      }
-      ++pos;
+  // compaction, one bitmap window of the index range at a time
+  unsigned written = 0;
+  for (int w0 = 0; w0 < nv; w0 += kWinWords * 32) {
+    const int nbits = min(nv - w0, kWinWords * 32);
+    const int nwords = (nbits + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) S.bm[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kAPer; ++u) {
+      const int s = ab[u] - w0;
+      if (ab[u] >= 0 && s >= 0 && s < nbits) atomicOr(&S.bm[s >> 5], 1u << (s & 31));
     }
+    for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
+      const int s = (int)S.cand[i].y - w0;
+      if (S.flag[i] && s >= 0 && s < nbits) atomicOr(&S.bm[s >> 5], 1u << (s & 31));
+    }
+    __syncthreads();
+    const int per = (nwords + blockDim.x - 1) / blockDim.x;
+    const int a0 = threadIdx.x * per, a1 = min(nwords, a0 + per);
+    unsigned cnt = 0;
+    for (int wi = a0; wi < a1; ++wi) cnt += __popc(S.bm[wi]);
+    unsigned tot;
+    unsigned pos = written + block_exclusive_scan(cnt, sh.scan, &tot);
+    for (int wi = a0; wi < a1; ++wi) {
+      unsigned word = S.bm[wi];
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1;
+        const int s = w0 + wi * 32 + bit;
+        if (pos < (unsigned)k) {
+          out[pos] = s;
+          if (sout) sout[pos] = sc[s];
+        }
+        ++pos;
+      }
+    }
+    written += tot;
+    __syncthreads();  // the window is rewritten next
   }
 }
 
@@ -348,48 +367,62 @@ __device__ void finalize_query(const float* __restrict__ sc, int nv, int N, int 
 __global__ void __launch_bounds__(1024) topk_select_final(
     const float* __restrict__ scores, int N, const int32_t* __restrict__ q_pos, int m, int k,
     MultiTopkWs ws, int32_t* __restrict__ idx_out, float* __restrict__ score_out) {
-  __shared__ uint2 cand[kCandCap];
+  extern __shared__ __align__(16) uint8_t topk_smem[];
+  SelectSmem& S = *reinterpret_cast<SelectSmem*>(topk_smem);
   __shared__ RadixShared sh;
   __shared__ int sT;
   __shared__ unsigned sAbove;
   __shared__ int s_last;
-  __shared__ unsigned s_lcount, s_base;
+  __shared__ unsigned s_nc, s_na, s_bc, s_ba;
   const int r = blockIdx.x;
   const int nv = n_visible(q_pos[r], m, N);
   const float* sc = scores + (size_t)r * N;
+  int32_t* out = idx_out + (size_t)r * k;
+  float* sout = score_out ? score_out + (size_t)r * k : nullptr;
   const int s0 = blockIdx.y * kChunk;
-  if (threadIdx.x == 0) s_lcount = 0;
-  __syncthreads();
-  if (nv > k && s0 < N) {
-    int T;
-    unsigned above;
+  int T = 0;
+  unsigned above = 0;
+  if (threadIdx.x == 0) { s_nc = 0; s_na = 0; }
+  if (nv > k) {
+    // this CTA's scores first (in flight while the threshold is found)
+    float v[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int s = s0 + u * 1024 + (int)threadIdx.x;
+      v[u] = s < nv ? __ldcg(sc + s) : 0.f;
+    }
     find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, &sT,
-                       &sAbove);
-    const int N32 = (N + 31) >> 5;
-    const int s1 = min(N, s0 + kChunk);
-    for (int base = s0; base < s1; base += blockDim.x) {
-      const int s = base + threadIdx.x;
-      const bool vis = s < nv && s < s1;
-      const unsigned key = vis ? score_key(sc[s]) : 0u;
-      const int bin = (int)(key >> 20);
-      const bool gt = vis && bin > T;
-      const bool eq = vis && bin == T;
-      const unsigned word = __ballot_sync(0xffffffffu, gt);
-      if ((threadIdx.x & 31) == 0 && (s >> 5) < N32 && s < s1)
-        ws.bitmap[(size_t)r * N32 + (s >> 5)] = word;
-      if (eq) {  // collect locally, publish with one global atomic per CTA
-        const unsigned pos = atomicAdd(&s_lcount, 1u);
-        if (pos < kLocalCap) cand[pos] = make_uint2(key, (unsigned)s);
+                       &sAbove);  // ends with a barrier: s_nc / s_na are zero
+    int* above_l = reinterpret_cast<int*>(S.bm);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int s = s0 + u * 1024 + (int)threadIdx.x;
+      if (s < nv) {
+        const unsigned key = score_key(v[u]);
+        const int bin = (int)(key >> 20);
+        if (bin > T) {
+          const unsigned p = atomicAdd(&s_na, 1u);  // < above < k <= kAboveCap
+          if (p < (unsigned)kAboveCap) above_l[p] = s;
+        } else if (bin == T) {
+          const unsigned p = atomicAdd(&s_nc, 1u);
+          if (p < (unsigned)kLocalCap) S.cand[p] = make_uint2(key, (unsigned)s);
+        }
       }
     }
     __syncthreads();
-    const unsigned ln = s_lcount;
-    if (threadIdx.x == 0 && ln > 0)
-      s_base = atomicAdd(&ws.cand_cnt[r], ln > kLocalCap ? (unsigned)kCandCap + 1u : ln);
+    const unsigned na = min(s_na, (unsigned)kAboveCap), nc = s_nc;
+    if (threadIdx.x == 0) {
+      s_ba = na ? atomicAdd(&ws.cnt[2 * r + 1], na) : 0u;
+      // an overflowing chunk pushes the query's count past the capacity
+      s_bc = nc ? atomicAdd(&ws.cnt[2 * r], nc > (unsigned)kLocalCap ? (unsigned)kCandCap + 1u : nc)
+                : 0u;
+    }
     __syncthreads();
-    if (ln > 0 && ln <= kLocalCap)
-      for (unsigned i = threadIdx.x; i < ln; i += blockDim.x)
-        if (s_base + i < (unsigned)kCandCap) ws.cand[(size_t)r * kCandCap + s_base + i] = cand[i];
+    for (unsigned i = threadIdx.x; i < na; i += blockDim.x)
+      if (s_ba + i < (unsigned)kAboveCap) ws.above[(size_t)r * kAboveCap + s_ba + i] = above_l[i];
+    if (nc <= (unsigned)kLocalCap)
+      for (unsigned i = threadIdx.x; i < nc; i += blockDim.x)
+        if (s_bc + i < (unsigned)kCandCap) ws.cand[(size_t)r * kCandCap + s_bc + i] = S.cand[i];
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -400,8 +433,11 @@ __global__ void __launch_bounds__(1024) topk_select_final(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  finalize_query(sc, nv, N, k, r, ws, idx_out + (size_t)r * k,
-                 score_out ? score_out + (size_t)r * k : nullptr, cand, sh, &sT, &sAbove);
+  if (nv <= k) {
+    write_all_visible(sc, nv, k, out, sout);
+    return;
+  }
+  finalize_query(sc, nv, k, r, T, above, ws, out, sout, S, sh);
 }
 
 // ------------------------------------------------------------------ host --
@@ -414,11 +450,12 @@ csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32
 __global__ void index_plan(const int32_t* q_pos, int G, int ngroups, int m, int N, int* prefix,
                            unsigned* zero_words, size_t nzero);
 
-static bool use_multi_topk(int R, int N) { return R <= 64 && N >= 4096; }
+static bool use_multi_topk(int R, int N, int k) {
+  return R <= 64 && N >= 4096 && k <= kAboveCap;
+}
 
 struct IdxWsLayout {
-  size_t scores = 0, plan = 0, ghist = 0, cand_cnt = 0, done = 0, bitmap = 0, cand = 0,
-         total = 0;
+  size_t scores = 0, plan = 0, ghist = 0, cnt = 0, done = 0, above = 0, cand = 0, total = 0;
 };
 
 static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
@@ -427,15 +464,15 @@ static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
   size_t off = align_up(R * N * sizeof(float), 256);
   L.plan = off;
   off += align_up((R + 1) * sizeof(int), 256);
-  if (use_multi_topk((int)R, N)) {
-    L.ghist = off;
+  if (use_multi_topk((int)R, N, p.topk)) {
+    L.ghist = off;  // ghist, cnt and done are contiguous (zeroed together)
     off += R * kBins * 4;
-    L.cand_cnt = off;
-    off += R * 4;
+    L.cnt = off;
+    off += R * 2 * 4;
     L.done = off;
     off = align_up(off + R * 4, 256);
-    L.bitmap = off;
-    off += align_up(R * ((N + 31) / 32) * 4, 256);
+    L.above = off;
+    off += align_up(R * kAboveCap * sizeof(int), 256);
     L.cand = off;
     off += align_up(R * kCandCap * sizeof(uint2), 256);
   }
@@ -483,14 +520,13 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
   char* base = (char*)ws;
   float* scores = (float*)base;
   int* plan = (int*)(base + L.plan);
-  const bool multi = use_multi_topk(R, N);
+  const bool multi = use_multi_topk(R, N, p.topk);
   MultiTopkWs mw{};
   size_t nzero = 0;
   if (multi) {
-    mw = MultiTopkWs{(unsigned*)(base + L.ghist), (unsigned*)(base + L.cand_cnt),
-                     (unsigned*)(base + L.done), (unsigned*)(base + L.bitmap),
-                     (uint2*)(base + L.cand)};
-    nzero = (L.bitmap - L.ghist) / 4;  // ghist, cand_cnt and done are contiguous
+    mw = MultiTopkWs{(unsigned*)(base + L.ghist), (unsigned*)(base + L.cnt),
+                     (unsigned*)(base + L.done), (int*)(base + L.above), (uint2*)(base + L.cand)};
+    nzero = (L.above - L.ghist) / 4;  // ghist, cnt and done
   }
   bool hist_done = false;
   if (index_tc_supported(p)) {
@@ -498,9 +534,7 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
                                           nzero, multi ? mw.ghist : nullptr, &hist_done, st);
     if (s != CSA_OK) return s;
   } else {
-    if (multi)
-      CSA_LAUNCH(KK_PLAN, st, index_plan<<<1, 1024, 0, st>>>(q_pos, 1, 0, p.m, N, plan, mw.ghist,
-                                                             nzero));
+    if (multi && cudaMemsetAsync(mw.ghist, 0, nzero * 4, st) != cudaSuccess) return CSA_ERR_CUDA;
     if (p.act == CSA_F32)
       launch_scores<float>(p, B, Q, q_pos, qI, w, kI, N, scores, st);
     else
@@ -511,7 +545,11 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
     if (!hist_done)
       CSA_LAUNCH(KK_TOPK_HIST, st, topk_hist<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m, p.topk,
                                                                     mw.ghist));
-    CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select_final<<<grid, 1024, 0, st>>>(
+    const int smem = (int)sizeof(SelectSmem);
+    if (cudaFuncSetAttribute(topk_select_final, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return CSA_ERR_CUDA;
+    CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select_final<<<grid, 1024, smem, st>>>(
                                        scores, N, q_pos, p.m, p.topk, mw, idx_out, score_out));
   } else {
     CSA_LAUNCH(KK_TOPK, st, topk_radix<<<R, kTopkThreads, 0, st>>>(scores, N, q_pos, p.m,
