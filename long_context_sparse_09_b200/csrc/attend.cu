@@ -320,18 +320,20 @@ __global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
 static int head_block(int n_h) { return n_h >= 16 ? 16 : n_h; }
 
 bool attend_tc_supported(const csa_params& p);
-void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps);
+void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps,
+                    int* cluster);
 csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
                             const int32_t* q_pos, const void* q, const int32_t* idx,
                             const void* ckv, const float* ckv_scale, int N, const void* win,
                             const float* win_scale, int W, const int32_t* win_pos0,
                             const float* sink, void* out, float* ws_o, float* ws_ml,
-                            int nsplit, int kps, cudaStream_t st);
+                            int nsplit, int kps, int cluster, cudaStream_t st);
 
 static void split_plan(const csa_params& p, int R, int N, bool dense, int* nsplit,
                        int* kps) {
   if (attend_tc_supported(p)) {
-    attend_tc_plan(p, R, N, dense, nsplit, kps);
+    int cluster = 0;
+    attend_tc_plan(p, R, N, dense, nsplit, kps, &cluster);
     return;
   }
   const int HB = head_block(p.n_h);
@@ -408,10 +410,14 @@ csa_status launch_attend(const csa_params& p, bool dense, int B, int Q,
     a.ws_ml = (float*)((char*)ws + align_up((size_t)a.nsplit * R * p.n_h * p.c * 4, 256));
   }
   if (attend_tc_supported(p)) {
+    // up to 8 key slices of a (query, head block) are combined inside the
+    // kernel (one cluster each); more slices are combined by attend_combine
+    int cluster = 0, ns = 0, kps = 0;
+    attend_tc_plan(p, R, N, dense, &ns, &kps, &cluster);  // the split of a.nsplit
     csa_status s = launch_attend_tc(p, dense, B, Q, q_pos, q, idx, ckv, ckv_scale, N, win,
                                     win_scale, W, win_pos0, sink, out, a.ws_o, a.ws_ml,
-                                    a.nsplit, a.keys_per_split, st);
-    if (s != CSA_OK || a.nsplit <= 1) return s;
+                                    a.nsplit, a.keys_per_split, cluster, st);
+    if (s != CSA_OK || a.nsplit <= 1 || cluster) return s;
     CSA_LAUNCH(KK_COMBINE, st, attend_combine<__nv_bfloat16><<<dim3(R, a.n_h), 128, 0, st>>>(a));
     return last_launch_status();
   }

@@ -45,12 +45,13 @@ struct AttnTcArgs {
   const int32_t* win_pos0;
   const float* sink;
   __nv_bfloat16* out;
-  float* ws_o;
-  float* ws_ml;
+  float* ws_o;   // split partials [nsplit][R][n_h][512] (global combine)
+  float* ws_ml;  // their (max, sum) [nsplit][R][n_h][2]
   unsigned* err;
   int Q, N, W, n_h, m, topk, n_win, nsplit, keys_per_split, dense, R, hblocks;
   int R_rows_c, R_rows_w;  // total rows of the cache / window tensors (out of range)
   int box_rows;            // rows of one output box: min(64, n_h)
+  int cluster;             // the key slices of a (query, head block) form a cluster
   float scale2;  // softmax scale times log2(e): the softmax runs in base 2
   double base;
 };
@@ -71,6 +72,7 @@ constexpr int kQBytes = 64 * 1024;
 constexpr int kKBytes = 64 * 1024;
 constexpr int kPBytes = 8 * 1024;
 constexpr float kLazyRescale = 8.0f;  // log2 units: rescale when the max grows 256x
+constexpr int kMaxSlices = 8;         // key slices of one (query, head block): one cluster
 
 template <bool FP8>
 struct AtLayout {
@@ -138,6 +140,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint64_t* pvdone = bars + 11;
   uint32_t* tbase_sm = (uint32_t*)(bars + 13);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
+  int& valid_sm = *(int*)(tbase_sm + 2);  // the slice had keys (cluster combine)
+  // slice max (base 2) and sum per head for the cluster combine; written
+  // after the last tile, when the per-tile key scales are no longer read
+  float2* ml_sm = (float2*)meta_scale;  // [64]
   __shared__ const uint8_t* row_sm[kAtKeys];
   __shared__ float rope_tab[64];
 
@@ -537,30 +543,42 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (lane == 0) mbar_arrive(&pfull[bb]);
       }
       // ---------------------------------------------------------- output --
-      // O rows are staged in the idle key buffers (128-byte swizzle) and
-      // written by TMA stores: bf16 O when the slice is the whole key list,
-      // else fp32 partials plus (max, sum) for the combine.
-      if (ok && mbar_wait(&pvdone[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_sm)) {
-        tc_fence_after();
+      // One slice (nsplit == 1): O rows are normalised with the sink,
+      // de-rotated, staged in the idle key buffers (128-byte swizzle) and
+      // written by TMA stores.  Several slices in a cluster: the running max
+      // and sum go to shared memory and the cluster combines the slices
+      // below.  Several slices without a cluster: fp32 partials and (max,
+      // sum) go to the workspace for attend_combine.
+      // (every softmax thread reaches the named barriers below, also after a
+      // timed-out wait, so that none of them waits for ever)
+      const bool fin =
+          ok && mbar_wait(&pvdone[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_sm);
+      tc_fence_after();
+      const bool any = m_used > 0.5f * kMasked;
+      if (a.nsplit > 1 && a.cluster) {
+        named_bar(2, 128);  // every softmax thread is done with the key scales
+        if (half == 0) ml_sm[hl] = fin ? make_float2(any ? m_used : -INFINITY, l)
+                                       : make_float2(-INFINITY, 0.f);
+      } else {
+        const bool split = a.nsplit > 1;
         const uint32_t orow = trow + ((uint32_t)(16 * half) << 16);
         const int brows = a.box_rows;
-        const bool store = hl < brows;  // head < n_h
+        const bool store = fin && hl < brows;  // head < n_h
         const int dim0 = half * 256;
-        const bool any = m_used > 0.5f * kMasked;
         float f = 1.f;
-        if (a.nsplit == 1) {
+        if (!split) {
           if (warp == 5) {  // R_{-t0} of the 32 RoPE pairs
             float cs, sn;
             rope_cs(-(double)t0, lane, 64, a.base, &cs, &sn);
             rope_tab[2 * lane] = cs;
             rope_tab[2 * lane + 1] = sn;
           }
-          const float zs = store ? a.sink[head] * kLog2e : 0.f;
+          const float zs = hl < brows ? a.sink[head] * kLog2e : 0.f;
           const float M = fmaxf(any ? m_used : zs, zs);
           const float em = any ? fast_exp2(m_used - M) : 0.f;
           f = em / (l * em + fast_exp2(zs - M));
-          named_bar(2, 128);
         }
+        named_bar(2, 128);
         uint8_t* stage = sK;  // 2 x 64 KB, free once the last P V is done
         const int box_bytes = brows * 128;
         const int sw = hl & 7;
@@ -572,7 +590,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           tmem_wait_ld();
           if (!store) continue;
           const int d0 = dim0 + c0;
-          if (a.nsplit == 1) {
+          if (!split) {
 #pragma unroll
             for (int u = 0; u < 64; ++u) v[u] *= f;
             if (d0 >= 448) {  // RoPE dims
@@ -607,30 +625,35 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
         fence_proxy_async_smem();
         named_bar(2, 128);
-        if (threadIdx.x == 160) {
-          if (a.nsplit == 1) {
+        if (threadIdx.x == 160 && fin) {
+          if (!split) {
             const int row0 = r * a.n_h + hb * 64;
-            for (int bx = 0; bx < 8; ++bx) tma_store_2d(&km.o_out, stage + bx * box_bytes, bx * 64, row0);
+            for (int bx = 0; bx < 8; ++bx)
+              tma_store_2d(&km.o_out, stage + bx * box_bytes, bx * 64, row0);
           } else {
             const int row0 = (sp * a.R + r) * a.n_h + hb * 64;
-            for (int bx = 0; bx < 16; ++bx) tma_store_2d(&km.o_ws, stage + bx * box_bytes, bx * 32, row0);
+            for (int bx = 0; bx < 16; ++bx)
+              tma_store_2d(&km.o_ws, stage + bx * box_bytes, bx * 32, row0);
           }
           bulk_commit();
           bulk_wait_all();
         }
-        if (store && a.nsplit > 1 && half == 0) {  // natural-log max for the combine
+        if (split && hl < brows && half == 0) {  // natural-log max for the combine
           const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
-          a.ws_ml[slot * 2] = any ? m_used * kLn2 : -INFINITY;
-          a.ws_ml[slot * 2 + 1] = l;
+          a.ws_ml[slot * 2] = (fin && any) ? m_used * kLn2 : -INFINITY;
+          a.ws_ml[slot * 2 + 1] = fin ? l : 0.f;
         }
       }
     }
   }
   if (ntiles == 0 && warp >= 5) {
-    // no keys in this slice: all weight on the sink (or an empty partial)
+    // no keys in this slice: all weight on the sink (or an empty slice)
     const int quad = warp & 3, half = lane >> 4;
-    const int head = hb * 64 + quad * 16 + (lane & 15);
-    if (head < a.n_h) {
+    const int hl = quad * 16 + (lane & 15);
+    const int head = hb * 64 + hl;
+    if (a.nsplit > 1 && a.cluster) {
+      if (half == 0) ml_sm[hl] = make_float2(-INFINITY, 0.f);
+    } else if (head < a.n_h) {
       if (a.nsplit == 1) {
         __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + head) * 512 + half * 256;
         for (int c0 = 0; c0 < 256; c0 += 8) *reinterpret_cast<uint4*>(dst + c0) = zero4();
@@ -650,6 +673,111 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (a.nsplit > 1 && a.cluster) {
+    // --------------------------------------------- slice combine (cluster) --
+    // The CTAs of the cluster hold the key slices of one (query, head
+    // block), CTA rank = slice.  Each CTA weighs its O by its share of the
+    // softmax (running maxima and sums read from every CTA through
+    // distributed shared memory, sink included), stages it in its idle key
+    // buffers, and CTA c sums heads [h0, h1) over the cluster, applies
+    // R_{-t0} and stores bf16 O.
+    const int S = a.nsplit;
+    const int brows = a.box_rows;
+    if (threadIdx.x == 0) valid_sm = (ntiles > 0 && !*abort_sm) ? 1 : 0;
+    if (warp == 4) {  // R_{-t0} of the 32 RoPE pairs
+      float cs, sn;
+      rope_cs(-(double)t0, lane, 64, a.base, &cs, &sn);
+      rope_tab[2 * lane] = cs;
+      rope_tab[2 * lane + 1] = sn;
+    }
+    __syncwarp();
+    cluster_sync_all();  // maxima, sums and flags of every slice are visible
+    unsigned live = 0;   // slices that hold keys (and did not time out)
+    for (int p = 0; p < S; ++p) {
+      int vp;
+      asm volatile("ld.shared::cluster.u32 %0, [%1];"
+                   : "=r"(vp)
+                   : "r"(mapa_shared(smem_u32(&valid_sm), p))
+                   : "memory");
+      live |= (vp ? 1u : 0u) << p;
+    }
+    uint8_t* stage = sK;  // [64 heads][512] fp32, 16-byte chunks swizzled by head
+    if (warp >= 5 && ((live >> sp) & 1u)) {
+      const int quad = warp & 3, half = lane >> 4;
+      const int hl = quad * 16 + (lane & 15);
+      const bool hv = hl < brows;  // head < n_h
+      const float zs = hv ? a.sink[hb * 64 + hl] * kLog2e : 0.f;
+      const uint32_t mla = smem_u32(&ml_sm[hl]);
+      float2 mlp[kMaxSlices];
+      float M = zs;
+#pragma unroll
+      for (int p = 0; p < kMaxSlices; ++p) {
+        mlp[p] = (p < S && ((live >> p) & 1u)) ? ld_dsmem_f2(mapa_shared(mla, p))
+                                               : make_float2(-INFINITY, 0.f);
+        M = fmaxf(M, mlp[p].x);
+      }
+      float den = fast_exp2(zs - M);
+#pragma unroll
+      for (int p = 0; p < kMaxSlices; ++p)
+        den += mlp[p].x > -INFINITY ? mlp[p].y * fast_exp2(mlp[p].x - M) : 0.f;
+      const float2 mine = ml_sm[hl];
+      const float f = mine.x > -INFINITY ? fast_exp2(mine.x - M) / den : 0.f;
+      const uint32_t orow = tbase + ((uint32_t)(quad * 32 + 16 * half) << 16);
+      uint8_t* rowp = stage + hl * 2048;
+      for (int c0 = 0; c0 < 256; c0 += 64) {
+        float v[64];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          tmem_ld16(orow + c0 + q4 * 16, *reinterpret_cast<float(*)[16]>(v + q4 * 16));
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {  // 16-byte chunk of dims half*256 + c0 + 4cc
+          const int ch = (half * 256 + c0) / 4 + cc;
+          const int off = (ch >> 3) * 128 + (((ch & 7) ^ (hl & 7)) << 4);
+          *reinterpret_cast<float4*>(rowp + off) =
+              make_float4(v[4 * cc] * f, v[4 * cc + 1] * f, v[4 * cc + 2] * f, v[4 * cc + 3] * f);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();  // weighted slices are staged
+    {
+      const int hper = (brows + S - 1) / S;
+      const int h0 = sp * hper, h1 = min(brows, h0 + hper);
+      const uint32_t sbase = smem_u32(stage);
+      for (int it = threadIdx.x; it < (h1 - h0) * 128; it += kAtThreads) {
+        const int h = h0 + (it >> 7), ch = it & 127;  // 16-byte chunk: dims 4ch .. 4ch+3
+        const uint32_t off = sbase + h * 2048 + (ch >> 3) * 128 + (((ch & 7) ^ (h & 7)) << 4);
+        float4 x[kMaxSlices];  // all peers' chunks in flight, then the sum
+#pragma unroll
+        for (int p = 0; p < kMaxSlices; ++p)
+          x[p] = (p < S && ((live >> p) & 1u)) ? ld_dsmem_f4(mapa_shared(off, p))
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = x[0];
+#pragma unroll
+        for (int p = 1; p < kMaxSlices; ++p) {
+          acc.x += x[p].x; acc.y += x[p].y; acc.z += x[p].z; acc.w += x[p].w;
+        }
+        const int d = ch * 4;
+        if (d >= 448) {  // RoPE dims: pairs (d, d+1), (d+2, d+3)
+          const int pr = (d - 448) >> 1;
+          const float c0 = rope_tab[2 * pr], s0 = rope_tab[2 * pr + 1];
+          const float c1 = rope_tab[2 * pr + 2], s1 = rope_tab[2 * pr + 3];
+          const float x0 = acc.x, x1 = acc.y, x2 = acc.z, x3 = acc.w;
+          acc.x = x0 * c0 - x1 * s0;
+          acc.y = x0 * s0 + x1 * c0;
+          acc.z = x2 * c1 - x3 * s1;
+          acc.w = x2 * s1 + x3 * c1;
+        }
+        __nv_bfloat16* dst = a.out + ((size_t)r * a.n_h + hb * 64 + h) * 512 + d;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while its staged slice is read
+    tc_fence_after();
+  }
   if (*abort_sm) {
     if (threadIdx.x == 0) atomicOr(a.err, CSA_DEV_TIMEOUT);
     const uint64_t t0w = globaltimer();
@@ -671,11 +799,14 @@ bool attend_tc_supported(const csa_params& p) {
          tma_available();
 }
 
-void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps) {
+// Key slices per (query, head block): at most one wave of CTAs (148 SMs, one
+// CTA each).  Up to kMaxSlices slices are launched as a cluster and combined
+// in the kernel; more slices write partials for attend_combine.
+void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps,
+                    int* cluster) {
   const int hbn = (p.n_h + 63) / 64;
   const int base = R * hbn;
   const int nk_max = (dense ? N : p.topk) + p.n_win;
-  // at most one wave of CTAs (148 SMs, one CTA each)
   const int ntiles = (nk_max + kAtKeys - 1) / kAtKeys;
   int s = base >= 148 ? 1 : 148 / base;
   if (s > ntiles) s = ntiles;
@@ -686,6 +817,35 @@ void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, 
   if (k < kAtKeys) k = kAtKeys;
   *kps = k;
   *nsplit = nk_max > 0 ? (nk_max + k - 1) / k : 1;
+  *cluster = *nsplit > 1 && *nsplit <= kMaxSlices;
+}
+
+// one CTA per (query, head block, key slice); the slices of one (query, head
+// block) are launched as a cluster
+template <bool FP8>
+static cudaError_t launch_attend_kernel(unsigned items, int smem, int cluster, cudaStream_t st,
+                                        const CUtensorMap& tmQ, const KeyMaps& km,
+                                        const AttnTcArgs& a) {
+  if (cudaFuncSetAttribute(attend_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return cudaErrorInvalidValue;
+  if (cluster <= 1) {
+    attend_tc<FP8><<<items, kAtThreads, smem, st>>>(tmQ, km, a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(items);
+  cfg.blockDim = dim3(kAtThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attend_tc<FP8>, tmQ, km, a);
 }
 
 csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
@@ -693,7 +853,7 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
                             const void* ckv, const float* ckv_scale, int N, const void* win,
                             const float* win_scale, int W, const int32_t* win_pos0,
                             const float* sink, void* out, float* ws_o, float* ws_ml,
-                            int nsplit, int kps, cudaStream_t st) {
+                            int nsplit, int kps, int cluster, cudaStream_t st) {
   const int R = B * Q;
   const int hbn = (p.n_h + 63) / 64;
   CUtensorMap tmQ;
@@ -702,6 +862,7 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
   a.q_pos = q_pos; a.idx = idx; a.ckv = (const uint8_t*)ckv; a.ckv_scale = ckv_scale;
   a.win = (const uint8_t*)win; a.win_scale = win_scale; a.win_pos0 = win_pos0; a.sink = sink;
   a.out = (__nv_bfloat16*)out; a.ws_o = ws_o; a.ws_ml = ws_ml; a.err = device_error_word();
+  a.cluster = cluster;
   a.Q = Q; a.N = N; a.W = W; a.n_h = p.n_h; a.m = p.m; a.topk = p.topk; a.n_win = p.n_win;
   a.nsplit = nsplit; a.keys_per_split = kps; a.dense = dense ? 1 : 0; a.R = R; a.hblocks = hbn;
   a.scale2 = p.softmax_scale * kLog2e; a.base = (double)p.rope_base;
@@ -730,23 +891,21 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
   a.box_rows = p.n_h < 64 ? p.n_h : 64;
   if (!make_tmap_bf16(&km.o_out, out, (uint64_t)R * p.n_h, 512, (uint32_t)a.box_rows))
     return CSA_ERR_CUDA;
-  if (nsplit > 1 &&
+  if (nsplit > 1 && !cluster &&
       !make_tmap_f32(&km.o_ws, ws_o, (uint64_t)nsplit * R * p.n_h, 512, (uint32_t)a.box_rows))
     return CSA_ERR_CUDA;
-  if (p.kv == CSA_KV_FP8MIX) {
-    const int smem = AtLayout<true>::total + 1024;
-    if (cudaFuncSetAttribute(attend_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return CSA_ERR_CUDA;
-    CSA_LAUNCH(KK_ATTN, st, attend_tc<true><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, km, a));
-  } else {
-    const int smem = AtLayout<false>::total + 1024;
-    if (cudaFuncSetAttribute(attend_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return CSA_ERR_CUDA;
-    CSA_LAUNCH(KK_ATTN, st, attend_tc<false><<<(unsigned)items, kAtThreads, smem, st>>>(tmQ, km, a));
-  }
-  return last_launch_status();
+  if (nsplit < 1 || (cluster && nsplit > kMaxSlices)) return CSA_ERR_UNSUPPORTED;
+  const int cl = cluster ? nsplit : 1;
+  cudaError_t e;
+  if (p.kv == CSA_KV_FP8MIX)
+    CSA_LAUNCH(KK_ATTN, st,
+               e = launch_attend_kernel<true>((unsigned)items, AtLayout<true>::total + 1024,
+                                              cl, st, tmQ, km, a));
+  else
+    CSA_LAUNCH(KK_ATTN, st,
+               e = launch_attend_kernel<false>((unsigned)items, AtLayout<false>::total + 1024,
+                                               cl, st, tmQ, km, a));
+  return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
 }  // namespace csa

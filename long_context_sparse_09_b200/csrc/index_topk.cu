@@ -166,36 +166,37 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
 // For a handful of queries with long visible ranges (decode).  (1) The top 12
 // key bits of every visible score are histogrammed (by the tensor-core
 // scorer's epilogue, or by topk_hist).  (2) Every CTA of the select pass
-// takes a chunk of one query's scores, finds the bin T that holds the k-th
-// largest key, and appends the indices of higher bins to the query's "above"
-// list and the (key, index) pairs of bin T to its candidate list.  (3) The
-// last CTA of the query to finish selects the still needed candidates (radix
-// select over the low 20 key bits, equal keys towards the lower index),
-// marks the above list and the chosen candidates in a shared-memory bitmap
-// of the index range and compacts it into ascending indices.  If bin T
-// overflows the candidate list, (3) falls back to the exact block-wide radix
-// select over all scores.
+// takes a chunk of one query's scores (8 consecutive entries per thread),
+// finds the bin T that holds the k-th largest key, and writes, in index
+// order, the entries of higher bins ("above") and the (key, index) pairs of
+// bin T ("candidates") to its chunk's slots, with their counts.  (3) The last
+// CTA of the query gathers both lists in index order, finds the exact k-th
+// key among the candidates (radix select over the low 20 key bits), keeps the
+// candidates above it and, of those equal to it, the lowest indices, and
+// merges the two ascending lists into the output.  A chunk or query whose
+// candidates overflow the slots falls back to the exact block-wide select.
 constexpr int kBins = 4096;
-constexpr int kChunk = 8192;    // entries per CTA in (1) and (2)
+constexpr int kChunk = 8192;     // entries per CTA in (1) and (2)
 constexpr int kPer = kChunk / 1024;
-constexpr int kCandCap = 4096;  // candidates per query
-constexpr int kAboveCap = 4096; // entries of bins above T (< k) per query
-constexpr int kLocalCap = 2048; // candidates one select CTA may hold locally
-constexpr int kWinWords = 8192;  // bitmap window of the compaction (262144 entries)
+constexpr int kMaxChunks = 1024; // one chunk per finalize thread
+constexpr int kCandCap = 4096;   // candidates per query in (3)
+constexpr int kAboveCap = 4096;  // largest k of this path
+constexpr int kLocalCap = 2048;  // candidate slots per chunk
 
 struct MultiTopkWs {
-  unsigned* ghist;     // [R][kBins]
-  unsigned* cnt;       // [R][2]: candidates, above
-  unsigned* done;      // [R] CTAs of the select pass that have finished
-  int* above;          // [R][kAboveCap] indices in bins above T
-  uint2* cand;         // [R][kCandCap] (key, index) in bin T
+  unsigned* ghist;  // [R][kBins]
+  unsigned* done;   // [R] CTAs of the select pass that have finished
+  uint2* ccnt;      // [R][nch] (above, candidates) per chunk
+  int* above;       // [R][nch][k] above entries of each chunk, ascending
+  uint2* cand;      // [R][nch][kLocalCap] (key, index) of each chunk, ascending
 };
 
-// dynamic shared memory of topk_select_final
+// dynamic shared memory of topk_select_final (finalize)
 struct SelectSmem {
-  uint2 cand[kCandCap];
-  unsigned bm[kWinWords];  // select pass: local above list; final: bitmap window
-  unsigned char flag[kCandCap];
+  int a[kAboveCap];       // above entries of the query, ascending
+  uint2 c[kCandCap];      // candidates of the query, ascending by index
+  int cs[kAboveCap];      // chosen candidates, ascending
+  unsigned oa[kMaxChunks + 1], oc[kMaxChunks + 1];  // chunk offsets
 };
 
 __global__ void __launch_bounds__(1024) topk_hist(const float* __restrict__ scores, int N,
@@ -244,46 +245,77 @@ __device__ void find_threshold_bin(const unsigned* __restrict__ gh, unsigned k, 
   *above_out = *sAbove;
 }
 
-// Exact completion of one query's selection (one CTA, 1024 threads), given
-// the bin T of the k-th key and the count of keys above it.
-__device__ void finalize_query(const float* __restrict__ sc, int nv, int k, int r, int T,
+// first position in the ascending list v[0..n) whose value is >= x
+template <typename F>
+__device__ __forceinline__ unsigned lower_bound(unsigned n, int x, F at) {
+  unsigned lo = 0, hi = n;
+  while (lo < hi) {
+    const unsigned mid = (lo + hi) >> 1;
+    if (at(mid) < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// Exact completion of one query's selection (1024 threads).  Returns false,
+// before writing any output, when the candidates do not fit (the caller then
+// runs the exact block-wide select).
+__device__ bool finalize_query(const float* __restrict__ sc, int k, int r, int nch, int T,
                                unsigned above, const MultiTopkWs& ws, int32_t* __restrict__ out,
                                float* __restrict__ sout, SelectSmem& S, RadixShared& sh) {
-  __shared__ unsigned s_eq_n;
-  const unsigned nc = __ldcg(ws.cnt + 2 * r);
-  const unsigned na = __ldcg(ws.cnt + 2 * r + 1);
-  if (nc > (unsigned)kCandCap || na != above) {  // bin T too crowded: exact block-wide select
-    radix_select_block(sc, nv, k, out, sout, sh);
-    return;
+  const int t = threadIdx.x;
+  // chunk counts -> offsets of each chunk's lists in the query's lists
+  uint2 cc = make_uint2(0u, 0u);
+  if (t < nch) cc = __ldcg(ws.ccnt + (size_t)r * nch + t);
+  const int bad = __syncthreads_or(t < nch && cc.y > (unsigned)kLocalCap);
+  unsigned na, ncand;
+  const unsigned xa = block_exclusive_scan(cc.x, sh.scan, &na);
+  const unsigned xc = block_exclusive_scan(min(cc.y, (unsigned)kLocalCap), sh.scan, &ncand);
+  if (t < nch) {
+    S.oa[t] = xa;
+    S.oc[t] = xc;
   }
-  // the above list stays in registers (na < k <= kAboveCap)
-  constexpr int kAPer = kAboveCap / 1024;
-  int ab[kAPer];
-#pragma unroll
-  for (int u = 0; u < kAPer; ++u) {
-    const unsigned j = u * 1024u + threadIdx.x;
-    ab[u] = j < na ? __ldcg(ws.above + (size_t)r * kAboveCap + j) : -1;
+  if (t == 0) {
+    S.oa[nch] = na;
+    S.oc[nch] = ncand;
   }
-  for (int i = threadIdx.x; i < (int)nc; i += blockDim.x)
-    S.cand[i] = __ldcg(ws.cand + (size_t)r * kCandCap + i);
-  // radix select of the remaining-th largest key among the candidates
-  unsigned remaining = (unsigned)k - above;  // 1 <= remaining <= nc
+  __syncthreads();
+  if (bad || na != above || ncand > (unsigned)kCandCap) return false;
+  // gather both lists in index order (chunk c's slice follows chunk c-1's)
+  auto chunk_of = [&](const unsigned* off, unsigned j) {
+    unsigned lo = 0, hi = (unsigned)nch - 1;  // last c with off[c] <= j
+    while (lo < hi) {
+      const unsigned mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= j) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  for (unsigned j = t; j < na; j += 1024) {
+    const unsigned c = chunk_of(S.oa, j);
+    S.a[j] = __ldcg(ws.above + ((size_t)r * nch + c) * k + (j - S.oa[c]));
+  }
+  for (unsigned j = t; j < ncand; j += 1024) {
+    const unsigned c = chunk_of(S.oc, j);
+    S.c[j] = __ldcg(ws.cand + ((size_t)r * nch + c) * kLocalCap + (j - S.oc[c]));
+  }
+  __syncthreads();
+  // radix select of the remaining-th largest key among the candidates: two
+  // 10-bit digits below the 12 bits of bin T
+  unsigned remaining = (unsigned)k - above;  // 1 <= remaining <= ncand
   unsigned prefix = (unsigned)T << 20, mask = 0xFFF00000u;
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = pass == 0 ? 10 : 0;
-    for (int i = threadIdx.x; i < 1024; i += blockDim.x) sh.hist[i] = 0;
+    sh.hist[t] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
-      const unsigned key = S.cand[i].x;
+    for (unsigned j = t; j < ncand; j += 1024) {
+      const unsigned key = S.c[j].x;
       if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 1023u], 1u);
     }
     __syncthreads();
-    // thread t owns bin 1023 - t: the exclusive scan counts higher bins
-    const int bin = 1023 - (int)threadIdx.x;
-    const unsigned hcount = sh.hist[bin];
+    const int bin = 1023 - t;  // the scan over t counts the higher bins
+    const unsigned hc = sh.hist[bin];
     unsigned tot;
-    const unsigned higher = block_exclusive_scan(hcount, sh.scan, &tot);
-    if (higher < remaining && higher + hcount >= remaining) {
+    const unsigned higher = block_exclusive_scan(hc, sh.scan, &tot);
+    if (higher < remaining && higher + hc >= remaining) {
       sh.digit = (unsigned)bin;
       sh.remaining = remaining - higher;
     }
@@ -291,75 +323,60 @@ __device__ void finalize_query(const float* __restrict__ sc, int nv, int k, int 
     prefix |= sh.digit << shift;
     mask |= 1023u << shift;
     remaining = sh.remaining;
-    __syncthreads();
   }
   const unsigned K = prefix;  // exact key of the k-th largest score
-  // keys above K are in; of the keys equal to K the `remaining` lowest
-  // indices are in (their candidate slots are listed in sh.hist)
-  if (threadIdx.x == 0) s_eq_n = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
-    const unsigned key = S.cand[i].x;
-    S.flag[i] = key > K;
-    if (key == K) {
-      const unsigned p = atomicAdd(&s_eq_n, 1u);
-      if (p < 2048) sh.hist[p] = (unsigned)i;
-    }
-  }
-  __syncthreads();
-  const unsigned neq = s_eq_n;
-  if (neq > 2048) {  // a huge tie: exact block-wide select over all scores
-    radix_select_block(sc, nv, k, out, sout, sh);
-    return;
-  }
-  for (unsigned e = threadIdx.x; e < neq; e += blockDim.x) {
-    const unsigned i = sh.hist[e];
-    const unsigned s = S.cand[i].y;
-    unsigned rank = 0;
-    if (neq != remaining)
-      for (unsigned j = 0; j < neq; ++j) rank += S.cand[sh.hist[j]].y < s;
-    S.flag[i] = rank < remaining;
-  }
-  __syncthreads();
-  // compaction, one bitmap window of the index range at a time
-  unsigned written = 0;
-  for (int w0 = 0; w0 < nv; w0 += kWinWords * 32) {
-    const int nbits = min(nv - w0, kWinWords * 32);
-    const int nwords = (nbits + 31) >> 5;
-    for (int i = threadIdx.x; i < nwords; i += blockDim.x) S.bm[i] = 0u;
-    __syncthreads();
+  // candidates kept: keys above K, and the `remaining` lowest indices with
+  // key K.  Thread t owns the four consecutive candidates 4t .. 4t+3.
+  unsigned keq = 0;
+  uint2 cv[4];
 #pragma unroll
-    for (int u = 0; u < kAPer; ++u) {
-      const int s = ab[u] - w0;
-      if (ab[u] >= 0 && s >= 0 && s < nbits) atomicOr(&S.bm[s >> 5], 1u << (s & 31));
-    }
-    for (int i = threadIdx.x; i < (int)nc; i += blockDim.x) {
-      const int s = (int)S.cand[i].y - w0;
-      if (S.flag[i] && s >= 0 && s < nbits) atomicOr(&S.bm[s >> 5], 1u << (s & 31));
-    }
-    __syncthreads();
-    const int per = (nwords + blockDim.x - 1) / blockDim.x;
-    const int a0 = threadIdx.x * per, a1 = min(nwords, a0 + per);
-    unsigned cnt = 0;
-    for (int wi = a0; wi < a1; ++wi) cnt += __popc(S.bm[wi]);
-    unsigned tot;
-    unsigned pos = written + block_exclusive_scan(cnt, sh.scan, &tot);
-    for (int wi = a0; wi < a1; ++wi) {
-      unsigned word = S.bm[wi];
-      while (word) {
-        const int bit = __ffs(word) - 1;
-        word &= word - 1;
-        const int s = w0 + wi * 32 + bit;
-        if (pos < (unsigned)k) {
-          out[pos] = s;
-          if (sout) sout[pos] = sc[s];
-        }
-        ++pos;
+  for (int u = 0; u < 4; ++u) {
+    const unsigned j = 4u * t + u;
+    cv[u] = j < ncand ? S.c[j] : make_uint2(0u, 0u);
+    keq += (j < ncand && cv[u].x == K) ? 1u : 0u;
+  }
+  unsigned teq;
+  unsigned req = block_exclusive_scan(keq, sh.scan, &teq);
+  unsigned keep = 0, kmask = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const unsigned j = 4u * t + u;
+    bool kp = false;
+    if (j < ncand) {
+      if (cv[u].x > K) {
+        kp = true;
+      } else if (cv[u].x == K) {
+        kp = req < remaining;
+        ++req;
       }
     }
-    written += tot;
-    __syncthreads();  // the window is rewritten next
+    kmask |= (kp ? 1u : 0u) << u;
+    keep += kp ? 1u : 0u;
   }
+  unsigned nkeep;
+  unsigned pk = block_exclusive_scan(keep, sh.scan, &nkeep);
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    if ((kmask >> u) & 1u) S.cs[pk++] = (int)cv[u].y;
+  __syncthreads();
+  // merge the two ascending lists: position = own rank + rank in the other
+  for (unsigned j = t; j < na; j += 1024) {
+    const int s = S.a[j];
+    const unsigned pos = j + lower_bound(nkeep, s, [&](unsigned i) { return S.cs[i]; });
+    if (pos < (unsigned)k) {
+      out[pos] = s;
+      if (sout) sout[pos] = sc[s];
+    }
+  }
+  for (unsigned j = t; j < nkeep; j += 1024) {
+    const int s = S.cs[j];
+    const unsigned pos = j + lower_bound(na, s, [&](unsigned i) { return S.a[i]; });
+    if (pos < (unsigned)k) {
+      out[pos] = s;
+      if (sout) sout[pos] = sc[s];
+    }
+  }
+  return true;
 }
 
 // Selection pass over a chunk of one query's scores; the last CTA of the
@@ -372,63 +389,58 @@ __global__ void __launch_bounds__(1024) topk_select_final(
   __shared__ RadixShared sh;
   __shared__ int sT;
   __shared__ unsigned sAbove;
-  __shared__ int s_last;
-  __shared__ unsigned s_nc, s_na, s_bc, s_ba;
-  const int r = blockIdx.x;
+  __shared__ int s_last, s_exact;
+  const int r = blockIdx.x, c = blockIdx.y, nch = gridDim.y;
   const int nv = n_visible(q_pos[r], m, N);
   const float* sc = scores + (size_t)r * N;
   int32_t* out = idx_out + (size_t)r * k;
   float* sout = score_out ? score_out + (size_t)r * k : nullptr;
-  const int s0 = blockIdx.y * kChunk;
   int T = 0;
   unsigned above = 0;
-  if (threadIdx.x == 0) { s_nc = 0; s_na = 0; }
   if (nv > k) {
-    // this CTA's scores first (in flight while the threshold is found)
+    // this thread's 8 consecutive scores first (in flight while the
+    // threshold is found)
+    const int sb = c * kChunk + (int)threadIdx.x * kPer;
     float v[kPer];
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int s = s0 + u * 1024 + (int)threadIdx.x;
-      v[u] = s < nv ? __ldcg(sc + s) : 0.f;
-    }
+    for (int u = 0; u < kPer; ++u) v[u] = sb + u < nv ? __ldcg(sc + sb + u) : 0.f;
     find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, &sT,
-                       &sAbove);  // ends with a barrier: s_nc / s_na are zero
-    int* above_l = reinterpret_cast<int*>(S.bm);
+                       &sAbove);
+    unsigned na = 0, nc = 0;
+    unsigned key[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int s = s0 + u * 1024 + (int)threadIdx.x;
-      if (s < nv) {
-        const unsigned key = score_key(v[u]);
-        const int bin = (int)(key >> 20);
-        if (bin > T) {
-          const unsigned p = atomicAdd(&s_na, 1u);  // < above < k <= kAboveCap
-          if (p < (unsigned)kAboveCap) above_l[p] = s;
-        } else if (bin == T) {
-          const unsigned p = atomicAdd(&s_nc, 1u);
-          if (p < (unsigned)kLocalCap) S.cand[p] = make_uint2(key, (unsigned)s);
-        }
+      key[u] = score_key(v[u]);
+      const int bin = (int)(key[u] >> 20);
+      const bool vis = sb + u < nv;
+      na += (vis && bin > T) ? 1u : 0u;
+      nc += (vis && bin == T) ? 1u : 0u;
+    }
+    // one scan of both counts (each total <= kChunk < 2^16)
+    unsigned tot;
+    const unsigned x = block_exclusive_scan(na | (nc << 16), sh.scan, &tot);
+    unsigned pa = x & 0xFFFFu, pc = x >> 16;
+    int* ab = ws.above + ((size_t)r * nch + c) * k;
+    uint2* cd = ws.cand + ((size_t)r * nch + c) * kLocalCap;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (sb + u >= nv) continue;
+      const int bin = (int)(key[u] >> 20);
+      if (bin > T) {
+        if (pa < (unsigned)k) ab[pa] = sb + u;  // a chunk holds fewer than k
+        ++pa;
+      } else if (bin == T) {
+        if (pc < (unsigned)kLocalCap) cd[pc] = make_uint2(key[u], (unsigned)(sb + u));
+        ++pc;
       }
     }
-    __syncthreads();
-    const unsigned na = min(s_na, (unsigned)kAboveCap), nc = s_nc;
-    if (threadIdx.x == 0) {
-      s_ba = na ? atomicAdd(&ws.cnt[2 * r + 1], na) : 0u;
-      // an overflowing chunk pushes the query's count past the capacity
-      s_bc = nc ? atomicAdd(&ws.cnt[2 * r], nc > (unsigned)kLocalCap ? (unsigned)kCandCap + 1u : nc)
-                : 0u;
-    }
-    __syncthreads();
-    for (unsigned i = threadIdx.x; i < na; i += blockDim.x)
-      if (s_ba + i < (unsigned)kAboveCap) ws.above[(size_t)r * kAboveCap + s_ba + i] = above_l[i];
-    if (nc <= (unsigned)kLocalCap)
-      for (unsigned i = threadIdx.x; i < nc; i += blockDim.x)
-        if (s_bc + i < (unsigned)kCandCap) ws.cand[(size_t)r * kCandCap + s_bc + i] = S.cand[i];
+    if (threadIdx.x == 0) ws.ccnt[(size_t)r * nch + c] = make_uint2(tot & 0xFFFFu, tot >> 16);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned prev = atomicAdd(&ws.done[r], 1u);
-    s_last = prev == gridDim.y - 1;
+    s_last = prev == (unsigned)nch - 1;
   }
   __syncthreads();
   if (!s_last) return;
@@ -437,7 +449,10 @@ __global__ void __launch_bounds__(1024) topk_select_final(
     write_all_visible(sc, nv, k, out, sout);
     return;
   }
-  finalize_query(sc, nv, k, r, T, above, ws, out, sout, S, sh);
+  const bool ok = finalize_query(sc, k, r, nch, T, above, ws, out, sout, S, sh);
+  if (threadIdx.x == 0) s_exact = !ok;
+  __syncthreads();
+  if (s_exact) radix_select_block(sc, nv, k, out, sout, sh);
 }
 
 // ------------------------------------------------------------------ host --
@@ -451,11 +466,11 @@ __global__ void index_plan(const int32_t* q_pos, int G, int ngroups, int m, int 
                            unsigned* zero_words, size_t nzero);
 
 static bool use_multi_topk(int R, int N, int k) {
-  return R <= 64 && N >= 4096 && k <= kAboveCap;
+  return R <= 64 && N >= 4096 && k <= kAboveCap && (N + kChunk - 1) / kChunk <= kMaxChunks;
 }
 
 struct IdxWsLayout {
-  size_t scores = 0, plan = 0, ghist = 0, cnt = 0, done = 0, above = 0, cand = 0, total = 0;
+  size_t scores = 0, plan = 0, ghist = 0, done = 0, ccnt = 0, above = 0, cand = 0, total = 0;
 };
 
 static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
@@ -465,16 +480,17 @@ static IdxWsLayout idx_ws_layout(const csa_params& p, int B, int Q, int N) {
   L.plan = off;
   off += align_up((R + 1) * sizeof(int), 256);
   if (use_multi_topk((int)R, N, p.topk)) {
-    L.ghist = off;  // ghist, cnt and done are contiguous (zeroed together)
+    const size_t nch = (N + kChunk - 1) / kChunk;
+    L.ghist = off;  // ghist and done are contiguous (zeroed together)
     off += R * kBins * 4;
-    L.cnt = off;
-    off += R * 2 * 4;
     L.done = off;
     off = align_up(off + R * 4, 256);
+    L.ccnt = off;
+    off += align_up(R * nch * sizeof(uint2), 256);
     L.above = off;
-    off += align_up(R * kAboveCap * sizeof(int), 256);
+    off += align_up(R * nch * p.topk * sizeof(int), 256);
     L.cand = off;
-    off += align_up(R * kCandCap * sizeof(uint2), 256);
+    off += align_up(R * nch * kLocalCap * sizeof(uint2), 256);
   }
   L.total = off;
   return L;
@@ -524,9 +540,9 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
   MultiTopkWs mw{};
   size_t nzero = 0;
   if (multi) {
-    mw = MultiTopkWs{(unsigned*)(base + L.ghist), (unsigned*)(base + L.cnt),
-                     (unsigned*)(base + L.done), (int*)(base + L.above), (uint2*)(base + L.cand)};
-    nzero = (L.above - L.ghist) / 4;  // ghist, cnt and done
+    mw = MultiTopkWs{(unsigned*)(base + L.ghist), (unsigned*)(base + L.done),
+                     (uint2*)(base + L.ccnt), (int*)(base + L.above), (uint2*)(base + L.cand)};
+    nzero = (L.ccnt - L.ghist) / 4;  // ghist and done
   }
   bool hist_done = false;
   if (index_tc_supported(p)) {

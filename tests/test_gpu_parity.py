@@ -111,6 +111,9 @@ ATTN_CASES = [
     ("csa_fp8_decode", "csa", "bf16", "fp8mix", 2, 1, 1500, 32, 512, 64, 4, 96, 128, "decode"),
     ("csa_f32_prefill", "csa", "f32", "f32", 1, 200, 64, 8, 128, 32, 4, 16, 16, "prefill"),
     ("csa_bf16_prefill_many", "csa", "bf16", "bf16", 1, 700, 300, 16, 512, 64, 4, 32, 128, "prefill"),
+    # few queries at random positions: key slices of a cluster that hold no keys
+    ("csa_bf16_split_ragged", "csa", "bf16", "bf16", 2, 3, 600, 16, 512, 64, 4, 64, 128, "prefill"),
+    ("csa_fp8_split_ragged", "csa", "bf16", "fp8mix", 1, 5, 900, 64, 512, 64, 4, 128, 128, "prefill"),
     ("hca_bf16_decode", "hca", "bf16", "bf16", 2, 1, 300, 16, 512, 64, 128, 0, 128, "decode"),
     ("hca_f32_prefill", "hca", "f32", "f32", 1, 150, 20, 4, 128, 32, 8, 0, 16, "prefill"),
     ("hca_fp8_decode", "hca", "bf16", "fp8mix", 2, 1, 260, 16, 512, 64, 128, 0, 128, "decode"),
