@@ -292,18 +292,16 @@ __global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
     const float4* src = reinterpret_cast<const float4*>(a.ws_o + ((size_t)r * a.n_h + head) * c) + e / 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     int s = 0;
-    for (; s + 4 <= S; s += 4) {
-      float4 v0 = src[(size_t)s * stride], v1 = src[(size_t)(s + 1) * stride];
-      float4 v2 = src[(size_t)(s + 2) * stride], v3 = src[(size_t)(s + 3) * stride];
-      const float f0 = wsp[s], f1 = wsp[s + 1], f2 = wsp[s + 2], f3 = wsp[s + 3];
-      acc.x = fmaf(f0, v0.x, acc.x); acc.y = fmaf(f0, v0.y, acc.y);
-      acc.z = fmaf(f0, v0.z, acc.z); acc.w = fmaf(f0, v0.w, acc.w);
-      acc.x = fmaf(f1, v1.x, acc.x); acc.y = fmaf(f1, v1.y, acc.y);
-      acc.z = fmaf(f1, v1.z, acc.z); acc.w = fmaf(f1, v1.w, acc.w);
-      acc.x = fmaf(f2, v2.x, acc.x); acc.y = fmaf(f2, v2.y, acc.y);
-      acc.z = fmaf(f2, v2.z, acc.z); acc.w = fmaf(f2, v2.w, acc.w);
-      acc.x = fmaf(f3, v3.x, acc.x); acc.y = fmaf(f3, v3.y, acc.y);
-      acc.z = fmaf(f3, v3.z, acc.z); acc.w = fmaf(f3, v3.w, acc.w);
+    for (; s + 8 <= S; s += 8) {  // eight partials in flight
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (size_t)(s + u) * stride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float f = wsp[s + u];
+        acc.x = fmaf(f, v[u].x, acc.x); acc.y = fmaf(f, v[u].y, acc.y);
+        acc.z = fmaf(f, v[u].z, acc.z); acc.w = fmaf(f, v[u].w, acc.w);
+      }
     }
     for (; s < S; ++s) {
       const float4 v = src[(size_t)s * stride];

@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
 constexpr int kBins = 4096;
 constexpr int kChunk = 8192;     // entries per CTA in (1) and (2)
 constexpr int kPer = kChunk / 1024;
-constexpr int kMaxChunks = 1024; // one chunk per finalize thread
+constexpr int kMaxChunks = 512;  // chunks of one query (counts fit one packed scan)
 constexpr int kCandCap = 4096;   // candidates per query in (3)
 constexpr int kAboveCap = 4096;  // largest k of this path
 constexpr int kLocalCap = 2048;  // candidate slots per chunk
@@ -266,10 +266,15 @@ __device__ bool finalize_query(const float* __restrict__ sc, int k, int r, int n
   // chunk counts -> offsets of each chunk's lists in the query's lists
   uint2 cc = make_uint2(0u, 0u);
   if (t < nch) cc = __ldcg(ws.ccnt + (size_t)r * nch + t);
-  const int bad = __syncthreads_or(t < nch && cc.y > (unsigned)kLocalCap);
-  unsigned na, ncand;
-  const unsigned xa = block_exclusive_scan(cc.x, sh.scan, &na);
-  const unsigned xc = block_exclusive_scan(min(cc.y, (unsigned)kLocalCap), sh.scan, &ncand);
+  // a chunk whose candidates filled its slots takes the exact select
+  const int bad = __syncthreads_or(t < nch && cc.y >= (unsigned)kLocalCap);
+  // one scan of both counts: above entries < k <= 4096 in bits 20..31,
+  // candidates (< kLocalCap per chunk, kMaxChunks chunks: < 2^20) below
+  const unsigned cy = min(cc.y, (unsigned)kLocalCap - 1u);
+  unsigned tot2;
+  const unsigned x2 = block_exclusive_scan((min(cc.x, 4095u) << 20) | cy, sh.scan, &tot2);
+  const unsigned xa = x2 >> 20, xc = x2 & 0xFFFFFu;
+  unsigned na = tot2 >> 20, ncand = tot2 & 0xFFFFFu;
   if (t < nch) {
     S.oa[t] = xa;
     S.oc[t] = xc;
@@ -326,38 +331,33 @@ __device__ bool finalize_query(const float* __restrict__ sc, int k, int r, int n
   }
   const unsigned K = prefix;  // exact key of the k-th largest score
   // candidates kept: keys above K, and the `remaining` lowest indices with
-  // key K.  Thread t owns the four consecutive candidates 4t .. 4t+3.
-  unsigned keq = 0;
+  // key K.  Thread t owns the four consecutive candidates 4t .. 4t+3; one
+  // scan of (greater, equal) counts gives every kept candidate its place.
+  unsigned kgt = 0, keq = 0;
   uint2 cv[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const unsigned j = 4u * t + u;
     cv[u] = j < ncand ? S.c[j] : make_uint2(0u, 0u);
+    kgt += (j < ncand && cv[u].x > K) ? 1u : 0u;
     keq += (j < ncand && cv[u].x == K) ? 1u : 0u;
   }
-  unsigned teq;
-  unsigned req = block_exclusive_scan(keq, sh.scan, &teq);
-  unsigned keep = 0, kmask = 0;
+  unsigned tge;
+  const unsigned xge = block_exclusive_scan((kgt << 16) | keq, sh.scan, &tge);
+  unsigned ngt = xge >> 16, neq = xge & 0xFFFFu;  // before this thread's candidates
+  const unsigned nkeep = (tge >> 16) + min(tge & 0xFFFFu, remaining);
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const unsigned j = 4u * t + u;
-    bool kp = false;
-    if (j < ncand) {
-      if (cv[u].x > K) {
-        kp = true;
-      } else if (cv[u].x == K) {
-        kp = req < remaining;
-        ++req;
-      }
+    if (j >= ncand) continue;
+    if (cv[u].x > K) {
+      S.cs[ngt + min(neq, remaining)] = (int)cv[u].y;
+      ++ngt;
+    } else if (cv[u].x == K) {
+      if (neq < remaining) S.cs[ngt + neq] = (int)cv[u].y;
+      ++neq;
     }
-    kmask |= (kp ? 1u : 0u) << u;
-    keep += kp ? 1u : 0u;
   }
-  unsigned nkeep;
-  unsigned pk = block_exclusive_scan(keep, sh.scan, &nkeep);
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    if ((kmask >> u) & 1u) S.cs[pk++] = (int)cv[u].y;
   __syncthreads();
   // merge the two ascending lists: position = own rank + rank in the other
   for (unsigned j = t; j < na; j += 1024) {
@@ -402,8 +402,15 @@ __global__ void __launch_bounds__(1024) topk_select_final(
     // threshold is found)
     const int sb = c * kChunk + (int)threadIdx.x * kPer;
     float v[kPer];
+    if ((N & 3) == 0 && sb + kPer <= nv) {  // two 16-byte loads
+      const float4 a0 = __ldcg(reinterpret_cast<const float4*>(sc + sb));
+      const float4 a1 = __ldcg(reinterpret_cast<const float4*>(sc + sb + 4));
+      v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+      v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+    } else {
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) v[u] = sb + u < nv ? __ldcg(sc + sb + u) : 0.f;
+      for (int u = 0; u < kPer; ++u) v[u] = sb + u < nv ? __ldcg(sc + sb + u) : 0.f;
+    }
     find_threshold_bin(ws.ghist + (size_t)r * kBins, (unsigned)k, sh.scan, &T, &above, &sT,
                        &sAbove);
     unsigned na = 0, nc = 0;
