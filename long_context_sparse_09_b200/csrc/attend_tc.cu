@@ -154,15 +154,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const int hb = (item % per_r) / a.nsplit;
   const int sp = item % a.nsplit;
   const int b = r / a.Q;
-  const int t0 = a.q_pos[r];
-  const int nv = n_visible(t0, a.m, a.N);
-  const int lo = t0 - a.n_win + 1 > 0 ? t0 - a.n_win + 1 : 0;
-  const int nwin_q = (a.n_win > 0 && t0 >= 0) ? t0 - lo + 1 : 0;
-  const int n_main = a.dense ? nv : a.topk;
-  const int nk = n_main + nwin_q;
-  const int j_begin = sp * a.keys_per_split;
-  const int j_end = min(nk, j_begin + a.keys_per_split);
-  const int ntiles = j_end > j_begin ? (j_end - j_begin + kAtKeys - 1) / kAtKeys : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
@@ -186,6 +177,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tbase_sm;
   const size_t rb = FP8 ? 576 : 1024;  // stored row bytes
+  // the set-up above may overlap the previous kernel; inputs are read below
+  pdl_wait();
+  const int t0 = a.q_pos[r];
+  const int nv = n_visible(t0, a.m, a.N);
+  const int lo = t0 - a.n_win + 1 > 0 ? t0 - a.n_win + 1 : 0;
+  const int nwin_q = (a.n_win > 0 && t0 >= 0) ? t0 - lo + 1 : 0;
+  const int n_main = a.dense ? nv : a.topk;
+  const int nk = n_main + nwin_q;
+  const int j_begin = sp * a.keys_per_split;
+  const int j_end = min(nk, j_begin + a.keys_per_split);
+  const int ntiles = j_end > j_begin ? (j_end - j_begin + kAtKeys - 1) / kAtKeys : 0;
 
   if (ntiles > 0) {
     if (!FP8 && warp < 4) {
@@ -636,7 +638,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
               tma_store_2d(&km.o_ws, stage + bx * box_bytes, bx * 32, row0);
           }
           bulk_commit();
-          bulk_wait_all();
+          bulk_wait_read();
         }
         if (split && hl < brows && half == 0) {  // natural-log max for the combine
           const size_t slot = ((size_t)sp * a.R + r) * a.n_h + head;
@@ -829,22 +831,27 @@ static cudaError_t launch_attend_kernel(unsigned items, int smem, int cluster, c
   if (cudaFuncSetAttribute(attend_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return cudaErrorInvalidValue;
-  if (cluster <= 1) {
-    attend_tc<FP8><<<items, kAtThreads, smem, st>>>(tmQ, km, a);
-    return cudaGetLastError();
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(items);
   cfg.blockDim = dim3(kAtThreads);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (kPdlAttend) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, attend_tc<FP8>, tmQ, km, a);
 }
 

@@ -32,6 +32,16 @@ void prof_end(int slot, cudaStream_t st);
     ::csa::count_launch();                   \
   } while (0)
 
+// Programmatic dependent launch: a kernel launched with it may be scheduled
+// while the previous kernel of the stream still runs; it calls pdl_wait()
+// before it reads anything earlier stream work wrote (a no-op otherwise).
+// A kernel calls pdl_trigger() to let its dependent be scheduled early.
+constexpr bool kPdlAttend = true;  // attention after the top-k
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Device error word of the current GPU (set with atomicOr from kernels).
 unsigned int* device_error_word();
 

@@ -390,6 +390,7 @@ __global__ void __launch_bounds__(1024) topk_select_final(
   __shared__ int sT;
   __shared__ unsigned sAbove;
   __shared__ int s_last, s_exact;
+  pdl_trigger();  // the attention kernel may take the SMs this grid frees
   const int r = blockIdx.x, c = blockIdx.y, nch = gridDim.y;
   const int nv = n_visible(q_pos[r], m, N);
   const float* sc = scores + (size_t)r * N;
