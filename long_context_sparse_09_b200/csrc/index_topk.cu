@@ -145,11 +145,145 @@ __device__ __forceinline__ void write_all_visible(const float* sc, int nv, int k
   }
 }
 
+// Top-k of one query with at most kFastMax visible entries, all in one
+// pass of loads (1024 threads x 8 consecutive entries in registers): a
+// histogram of the top 12 key bits gives the bin T of the k-th key; the keys
+// of bin T are listed and a two-digit radix select over their low 20 bits
+// gives the exact k-th key K; one scan of (key > K, key == K) counts then
+// places every selected entry in index order, the lowest indices first
+// among keys equal to K.  Returns false, before writing any output, when bin
+// T holds more than kFastCand keys.
+constexpr int kFastMax = 8192;
+constexpr int kFastCand = 2048;
+struct FastTopkSmem {
+  unsigned hist[4096];
+  uint2 cand[kFastCand];
+};
+
+__device__ bool topk_block_fast(const float* __restrict__ sc, int nv, int k,
+                                int32_t* __restrict__ out, float* __restrict__ sout,
+                                FastTopkSmem& F, RadixShared& sh) {
+  __shared__ unsigned s_nc;
+  __shared__ int sT;
+  __shared__ unsigned sAbove;
+  const int t = threadIdx.x;
+  const int sb = t * 8;
+  float v[8];
+  if ((((uintptr_t)sc) & 15) == 0 && sb + 8 <= nv) {
+    const float4 a0 = __ldg(reinterpret_cast<const float4*>(sc + sb));
+    const float4 a1 = __ldg(reinterpret_cast<const float4*>(sc + sb + 4));
+    v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+    v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = sb + u < nv ? __ldg(sc + sb + u) : 0.f;
+  }
+  unsigned key[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) key[u] = score_key(v[u]);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) F.hist[4 * t + j] = 0;
+  if (t == 0) s_nc = 0;
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    if (sb + u < nv) atomicAdd(&F.hist[key[u] >> 20], 1u);
+  __syncthreads();
+  // bin T of the k-th key: thread t owns bins 4(1023 - t) .. +3
+  {
+    const int rt = 1023 - t;
+    unsigned c[4], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      c[j] = F.hist[4 * rt + j];
+      sum += c[j];
+    }
+    unsigned tot;
+    unsigned above = block_exclusive_scan(sum, sh.scan, &tot);
+#pragma unroll
+    for (int j = 3; j >= 0; --j) {
+      if (above < (unsigned)k && above + c[j] >= (unsigned)k) {
+        sT = 4 * rt + j;
+        sAbove = above;
+      }
+      above += c[j];
+    }
+  }
+  __syncthreads();
+  const int T = sT;
+  const unsigned above = sAbove;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    if (sb + u < nv && (int)(key[u] >> 20) == T) {
+      const unsigned p = atomicAdd(&s_nc, 1u);
+      if (p < (unsigned)kFastCand) F.cand[p] = make_uint2(key[u], 0u);
+    }
+  __syncthreads();
+  const unsigned nc = s_nc;
+  if (nc > (unsigned)kFastCand) return false;
+  // exact k-th key among the candidates (keys only: ties are settled below)
+  unsigned remaining = (unsigned)k - above;
+  unsigned prefix = (unsigned)T << 20, mask = 0xFFF00000u;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    sh.hist[t] = 0;
+    __syncthreads();
+    for (unsigned j = t; j < nc; j += 1024) {
+      const unsigned kk = F.cand[j].x;
+      if ((kk & mask) == prefix) atomicAdd(&sh.hist[(kk >> shift) & 1023u], 1u);
+    }
+    __syncthreads();
+    const int bin = 1023 - t;
+    const unsigned hc = sh.hist[bin];
+    unsigned tot;
+    const unsigned higher = block_exclusive_scan(hc, sh.scan, &tot);
+    if (higher < remaining && higher + hc >= remaining) {
+      sh.digit = (unsigned)bin;
+      sh.remaining = remaining - higher;
+    }
+    __syncthreads();
+    prefix |= sh.digit << shift;
+    mask |= 1023u << shift;
+    remaining = sh.remaining;
+  }
+  const unsigned K = prefix;
+  // one scan of (key > K, key == K) counts: positions in index order
+  unsigned ngt = 0, neq = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const bool vis = sb + u < nv;
+    ngt += (vis && key[u] > K) ? 1u : 0u;
+    neq += (vis && key[u] == K) ? 1u : 0u;
+  }
+  unsigned tge;
+  const unsigned x = block_exclusive_scan((ngt << 16) | neq, sh.scan, &tge);
+  unsigned bg = x >> 16, be = x & 0xFFFFu;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    if (sb + u >= nv) continue;
+    int pos = -1;
+    if (key[u] > K) {
+      pos = (int)(bg + min(be, remaining));
+      ++bg;
+    } else if (key[u] == K) {
+      if (be < remaining) pos = (int)(bg + be);
+      ++be;
+    }
+    if (pos >= 0 && pos < k) {
+      out[pos] = sb + u;
+      if (sout) sout[pos] = v[u];
+    }
+  }
+  return true;
+}
+
 // One CTA per query (used when there are many queries).
-__global__ void __launch_bounds__(kTopkThreads) topk_radix(
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_radix(
     const float* __restrict__ scores, int N, const int32_t* __restrict__ q_pos,
     int m, int k, int32_t* __restrict__ idx_out, float* __restrict__ score_out) {
+  extern __shared__ __align__(16) uint8_t topk_fast_smem[];
   __shared__ RadixShared sh;
+  __shared__ int s_ok;
   const int r = blockIdx.x;
   const int nv = n_visible(q_pos[r], m, N);
   const float* sc = scores + (size_t)r * N;
@@ -158,6 +292,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix(
   if (nv <= k) {
     write_all_visible(sc, nv, k, out, sout);
     return;
+  }
+  if (nv <= kFastMax) {
+    const bool ok = topk_block_fast(sc, nv, k, out, sout,
+                                    *reinterpret_cast<FastTopkSmem*>(topk_fast_smem), sh);
+    if (threadIdx.x == 0) s_ok = ok;
+    __syncthreads();
+    if (s_ok) return;
   }
   radix_select_block(sc, nv, k, out, sout, sh);
 }
@@ -576,8 +717,12 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
     CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select_final<<<grid, 1024, smem, st>>>(
                                        scores, N, q_pos, p.m, p.topk, mw, idx_out, score_out));
   } else {
-    CSA_LAUNCH(KK_TOPK, st, topk_radix<<<R, kTopkThreads, 0, st>>>(scores, N, q_pos, p.m,
-                                                                   p.topk, idx_out, score_out));
+    const int smem = (int)sizeof(FastTopkSmem);
+    if (cudaFuncSetAttribute(topk_radix, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return CSA_ERR_CUDA;
+    CSA_LAUNCH(KK_TOPK, st, topk_radix<<<R, kTopkThreads, smem, st>>>(scores, N, q_pos, p.m,
+                                                                      p.topk, idx_out, score_out));
   }
   return last_launch_status();
 }

@@ -76,7 +76,7 @@ def test_index_topk_parity(case):
         check_topk(idx[rows].cpu().numpy(), sco[rows].cpu().numpy(), sref, nv, k, tol, name)
 
 
-@pytest.mark.parametrize("nh,N", [(8, 1000), (64, 20000)])
+@pytest.mark.parametrize("nh,N", [(8, 1000), (8, 3000), (64, 20000)])
 def test_index_topk_all_ties_take_lowest_indices(nh, N):
     """w = 0: every score is 0, the selection is 0..k-1 (lower index wins);
     the long case overflows the multi-CTA candidate list on purpose."""
@@ -89,6 +89,36 @@ def test_index_topk_all_ties_take_lowest_indices(nh, N):
     idx = torch.empty(2, 100, dtype=torch.int32, device=DEV)
     bd.csa_index_topk(p, pos, qI, w, kI, idx)
     assert torch.equal(idx.cpu(), torch.arange(100, dtype=torch.int32).repeat(2, 1))
+
+
+@pytest.mark.parametrize("B,Q,N,k", [(1, 200, 2000, 64), (2, 1, 20000, 300)])
+def test_index_topk_integer_scores_exact(B, Q, N, k):
+    """Small-integer q^I, K^I and w: every score is exact in fp32, so many
+    scores tie at the k-th value and the selection must equal the oracle's
+    (ties to the lower index) element for element.  Covers the per-query
+    and the multi-CTA top-k."""
+    wl = BASE.with_(n_hI=16, c_I=64, topk=k)
+    p = bd.params_for(wl)
+    g = _gen(B * 1000 + N)
+    qI = torch.randint(0, 2, (B * Q, 16, 64), generator=g).to(torch.bfloat16)
+    kI = torch.randint(-2, 3, (B, N, 64), generator=g).to(torch.bfloat16)
+    w = torch.randint(1, 3, (B * Q, 16), generator=g).float() * 0.5
+    pos = torch.full((B * Q,), 4 * N, dtype=torch.int32)
+    if Q > 1:
+        pos = torch.randint(4 * k, 4 * N, (B * Q,), generator=g, dtype=torch.int32)
+    idx = torch.empty(B * Q, k, dtype=torch.int32, device=DEV)
+    sco = torch.empty(B * Q, k, dtype=torch.float32, device=DEV)
+    bd.csa_index_topk(p, pos.to(DEV), qI.to(DEV), w.to(DEV), kI.to(DEV), idx, sco)
+    torch.cuda.synchronize()
+    for b in range(B):
+        rows = slice(b * Q, (b + 1) * Q)
+        sref = oracle.index_scores(pos[rows].numpy(), wl.m, qI[rows], w[rows], kI[b])
+        nv = np.array([oracle.nvis(t, wl.m, N) for t in pos[rows].numpy()], np.int32)
+        ref_idx, _ = oracle.topk(sref, nv, k)
+        assert np.array_equal(idx[rows].cpu().numpy(), ref_idx), f"b{b}: selection differs"
+        got = sco[rows].cpu().numpy()
+        exp = np.take_along_axis(sref, np.maximum(ref_idx, 0), axis=1)
+        assert np.array_equal(got[ref_idx >= 0], exp[ref_idx >= 0]), f"b{b}: scores differ"
 
 
 # ---------------------------------------------------------------- attend --
