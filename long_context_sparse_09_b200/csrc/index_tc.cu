@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
   unsigned* shist = (unsigned*)((uint8_t*)bars + 512);  // [kHistBins] when G == 1
   int* s_prefix = (int*)((uint8_t*)bars + 512 + (G == 1 ? kHistBins * 4 : 0));  // [65]
+  float* s_w = (float*)(s_prefix + 80);  // [G * 64] head weights of the group (G > 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // as many TMEM accumulators as fit (up to 8): more products in flight
@@ -287,7 +288,21 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
       int an = 0, hist_r = cur.g;
       float wreg[G == 1 ? 64 : 1];
       int w_r = -1;
+      constexpr int NQM = (NE == 4 || kAlt) ? G : G / 2;  // queries of this warp
+      int nvq[NQM];  // visible entries of those queries (current group)
+      int grp_r = -1;
       for (int i = 0; i < count; ++i) {
+        if (cur.g != grp_r) {  // group changed: its visible counts (and weights)
+#pragma unroll
+          for (int qq = 0; qq < NQM; ++qq)
+            nvq[qq] = n_visible(__ldg(a.q_pos + cur.g * G + q0 + qq), a.m, a.N);
+          if (G > 1 && a.nhI == 64) {
+            named_bar(2, 32 * NE);  // every epilogue warp is done with the old weights
+            for (int j = et; j < G * 64; j += 32 * NE) s_w[j] = __ldg(a.w + (size_t)cur.g * G * 64 + j);
+            named_bar(2, 32 * NE);
+          }
+          grp_r = cur.g;
+        }
         if (hist && cur.g != hist_r) {  // query changed: flush its histogram
           named_bar(2, 32 * NE);
           for (int bin = et; bin < kHistBins; bin += 32 * NE) {
@@ -335,6 +350,29 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
             for (int j = 0; j < 16; ++j)
               part[q4] = fmaf(wreg[16 * q4 + j], fmaxf(v[q4][j], 0.f), part[q4]);
           sc[0] = (part[0] + part[1]) + (part[2] + part[3]);
+        } else if (a.nhI == 64) {
+          // 64 heads per query: weights of the group in shared memory
+#pragma unroll
+          for (int qq = 0; qq < NQM; ++qq) {
+            const int qi = q0 + qq;
+            float v[4][16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(trow + qi * 64 + q4 * 16, v[q4]);
+            tmem_wait_ld();
+            const float4* w4 = reinterpret_cast<const float4*>(s_w + qi * 64);
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 ww = w4[q4 * 4 + j4];
+                part[q4] = fmaf(ww.x, fmaxf(v[q4][4 * j4 + 0], 0.f), part[q4]);
+                part[q4] = fmaf(ww.y, fmaxf(v[q4][4 * j4 + 1], 0.f), part[q4]);
+                part[q4] = fmaf(ww.z, fmaxf(v[q4][4 * j4 + 2], 0.f), part[q4]);
+                part[q4] = fmaf(ww.w, fmaxf(v[q4][4 * j4 + 3], 0.f), part[q4]);
+              }
+            sc[qq] = (part[0] + part[1]) + (part[2] + part[3]);
+          }
         } else {
         for (int qq = 0; qq < nq_mine; ++qq) {
           const int qi = q0 + qq;
@@ -369,10 +407,10 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
-        for (int qq = 0; qq < nq_mine; ++qq) {
+#pragma unroll
+        for (int qq = 0; qq < NQM; ++qq) {
           const int r = cur.g * G + q0 + qq;
-          const int nv = n_visible(__ldg(a.q_pos + r), a.m, a.N);
-          if (s < nv) {
+          if (s < nvq[qq]) {
             a.scores[(size_t)r * a.N + s] = sc[qq];
             if (hist) atomicAdd(&shist[score_key(sc[qq]) >> 20], 1u);
           }
@@ -474,7 +512,7 @@ static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
   using Cfg = IdxTcCfg<G, KB, S, NE, NQ>;
   const int NROWS = G * a.nhI;
   size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + NQ * (size_t)KB * NROWS * 128 + 512 +
-                (G == 1 ? kHistBins * 4 : 0) + (kInlineGroups + 1) * 4;
+                (G == 1 ? kHistBins * 4 : 0) + 80 * 4 + G * 64 * 4;
   auto kern = index_scores_tc<G, KB, S, NE, NQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)

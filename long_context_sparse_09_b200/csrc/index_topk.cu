@@ -278,7 +278,7 @@ __device__ bool topk_block_fast(const float* __restrict__ sc, int nv, int k,
 }
 
 // One CTA per query (used when there are many queries).
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_radix(
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_radix(
     const float* __restrict__ scores, int N, const int32_t* __restrict__ q_pos,
     int m, int k, int32_t* __restrict__ idx_out, float* __restrict__ score_out) {
   extern __shared__ __align__(16) uint8_t topk_fast_smem[];
