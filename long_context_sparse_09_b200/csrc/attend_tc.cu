@@ -73,6 +73,7 @@ constexpr int kKBytes = 64 * 1024;
 constexpr int kPBytes = 8 * 1024;
 constexpr float kLazyRescale = 8.0f;  // log2 units: rescale when the max grows 256x
 constexpr int kMaxSlices = 8;         // key slices of one (query, head block): one cluster
+constexpr bool kAsyncGather = true;   // bf16 selected rows by cp.async (else via registers)
 
 template <bool FP8>
 struct AtLayout {
@@ -257,6 +258,20 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             tma_load_2d(dstK + t * 8192, mode == 1 ? &km.c_box : &km.w_box, &kfull[s], t * 64,
                         s_row0);
           if (t != 0) mbar_arrive(&kfull[s]);
+        } else if (kAsyncGather) {
+          // selected rows: 32 asynchronous 16-byte copies per thread straight
+          // into the swizzled tile (absent rows are zero-filled); the barrier
+          // completes when they land, so the next tile's copies can follow
+#pragma unroll 8
+          for (int u = 0; u < 32; ++u) {
+            const int idx = u * 128 + t;
+            const int key = idx >> 6, ch = idx & 63;
+            const int kb = ch >> 3, c = ch & 7;
+            const uint8_t* src = row_sm[key];
+            cp_async16(dstK + kb * 8192 + key * 128 + ((c ^ (key & 7)) << 4),
+                       src ? src + ch * 16 : a.ckv, src ? 16u : 0u);
+          }
+          cp_async_arrive(&kfull[s]);
         } else {
 #pragma unroll 1
           for (int it0 = 0; it0 < 32; it0 += 16) {
