@@ -485,13 +485,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         // logits in base-2 units; absent keys get a huge negative logit
         const unsigned long long vmask = meta_mask[s];
         const float* scl = meta_scale + s * 64;
-        float mt = kMasked;
+        float mq[4] = {kMasked, kMasked, kMasked, kMasked};  // four short chains
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           const float z = ((vmask >> j) & 1ull) ? a.scale2 * sv[j] : kMasked;
           sv[j] = z;
-          mt = fmaxf(mt, z);
+          mq[j & 3] = fmaxf(mq[j & 3], z);
         }
+        const float mt = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
         float alpha = 1.f;
         int resc = 0;
         if (mt > 0.5f * kMasked) {  // the tile has a present key
@@ -523,13 +524,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           tmem_wait_st();
           tc_fence_before();
         }
-        float lsum = 0.f;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           const float p = sv[j] > 0.5f * kMasked ? fast_exp2(sv[j] - m_used) : 0.f;
-          lsum += p;
+          ls[j & 3] += p;
           sv[j] = p;
         }
+        const float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
         l = l * alpha + lsum;
         l = __shfl_sync(0xffffffffu, l, src);
         // P buffer bb was read by the P V of tile i-2
