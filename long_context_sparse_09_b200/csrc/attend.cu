@@ -263,6 +263,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
   __shared__ float wsp[256];
   __shared__ float s_den;
+  pdl_wait();  // partials of the attention kernel
   const int r = blockIdx.x, head = blockIdx.y;
   const size_t R = gridDim.x;
   const int c = a.c;
@@ -416,8 +417,11 @@ csa_status launch_attend(const csa_params& p, bool dense, int B, int Q,
                                     win_scale, W, win_pos0, sink, out, a.ws_o, a.ws_ml,
                                     a.nsplit, a.keys_per_split, cluster, st);
     if (s != CSA_OK || a.nsplit <= 1 || cluster) return s;
-    CSA_LAUNCH(KK_COMBINE, st, attend_combine<__nv_bfloat16><<<dim3(R, a.n_h), 128, 0, st>>>(a));
-    return last_launch_status();
+    cudaError_t e = cudaSuccess;
+    CSA_LAUNCH(KK_COMBINE, st,
+               e = launch_maybe_pdl(kPdlCombine, attend_combine<__nv_bfloat16>, dim3(R, a.n_h),
+                                    dim3(128), 0, st, a));
+    return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
   }
   if (p.act == CSA_F32) {
     if (p.kv == CSA_F32) return launch_attn_c<float, CSA_F32>(a, R, st);

@@ -802,6 +802,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     const uint64_t t0w = globaltimer();
     while (globaltimer() - t0w < 200000ull) __nanosleep(1000);
   }
+  pdl_trigger();  // the slice combine may be scheduled as this grid retires
   if (warp == 4) tmem_dealloc(tbase, 512);
 }
 

@@ -36,7 +36,25 @@ void prof_end(int slot, cudaStream_t st);
 // while the previous kernel of the stream still runs; it calls pdl_wait()
 // before it reads anything earlier stream work wrote (a no-op otherwise).
 // A kernel calls pdl_trigger() to let its dependent be scheduled early.
-constexpr bool kPdlAttend = true;  // attention after the top-k
+constexpr bool kPdlAttend = true;   // attention after the top-k
+constexpr bool kPdlTopk = false;    // top-k select after the scorer (measured slower)
+constexpr bool kPdlCombine = false; // slice combine after the attention (no gain)
+// launch with the programmatic-dependent attribute when `pdl` is set
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_maybe_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                                    size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -437,6 +437,7 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
     const uint64_t t0 = globaltimer();
     while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
   }
+  pdl_trigger();  // the top-k kernel may be scheduled as this grid retires
   if (warp == 1) tmem_dealloc(tbase, ncols_alloc);
 }
 

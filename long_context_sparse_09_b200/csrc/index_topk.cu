@@ -532,6 +532,7 @@ __global__ void __launch_bounds__(1024) topk_select_final(
   __shared__ unsigned sAbove;
   __shared__ int s_last, s_exact;
   pdl_trigger();  // the attention kernel may take the SMs this grid frees
+  pdl_wait();     // scores and histograms of the scoring kernel
   const int r = blockIdx.x, c = blockIdx.y, nch = gridDim.y;
   const int nv = n_visible(q_pos[r], m, N);
   const float* sc = scores + (size_t)r * N;
@@ -714,8 +715,12 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
     if (cudaFuncSetAttribute(topk_select_final, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return CSA_ERR_CUDA;
-    CSA_LAUNCH(KK_TOPK_SELECT, st, topk_select_final<<<grid, 1024, smem, st>>>(
-                                       scores, N, q_pos, p.m, p.topk, mw, idx_out, score_out));
+    cudaError_t e = cudaSuccess;
+    CSA_LAUNCH(KK_TOPK_SELECT, st,
+               e = launch_maybe_pdl(kPdlTopk && hist_done, topk_select_final, grid, dim3(1024),
+                                    (size_t)smem, st, (const float*)scores, N, q_pos, p.m,
+                                    p.topk, mw, idx_out, score_out));
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
   } else {
     const int smem = (int)sizeof(FastTopkSmem);
     if (cudaFuncSetAttribute(topk_radix, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
