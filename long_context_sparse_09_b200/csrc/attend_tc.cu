@@ -201,10 +201,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int wp0 = a.win ? a.win_pos0[b] : 0;
       const uint8_t* ckv = a.ckv + (size_t)b * a.N * rb;
       const uint8_t* win = a.win + (size_t)b * a.W * rb;
+      // the selected index of this thread's key in the next tile is loaded
+      // one tile ahead (its latency hides behind the current tile's copies)
+      auto sel_index = [&](int j) -> int {
+        return (t < kAtKeys && !a.dense && j < j_end && j < n_main)
+                   ? __ldg(a.idx + (size_t)r * a.topk + j) : 0;
+      };
+      int e_next = sel_index(j_begin + t);
       for (int i = 0; i < ntiles; ++i) {
         const int s = i & 1;
         if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
         const int j0 = j_begin + i * kAtKeys;
+        const int e_sel = e_next;
+        e_next = sel_index(j0 + kAtKeys + t);
         if (t < kAtKeys) {
           const int j = j0 + t;
           int valid = 0;
@@ -212,7 +221,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const uint8_t* row = nullptr;
           if (j < j_end) {
             if (j < n_main) {
-              const int e = a.dense ? j : a.idx[(size_t)r * a.topk + j];
+              const int e = a.dense ? j : e_sel;
               if (e >= 0) {
                 if (e < nv) {
                   valid = 1;
@@ -376,9 +385,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     } else if (warp == 4) {
       // ------------------------------------------------------------- MMA --
       if (lane == 0) {
+        // queries and outputs are touched once: keep the cached keys in L2
+        const uint64_t qo_pol = l2_evict_first_policy();
         mbar_expect_tx(qfull, kQBytes);
         for (int kb = 0; kb < 8; ++kb)
-          tma_load_2d(sQ + kb * 8192, &tmQ, qfull, kb * 64, r * a.n_h + hb * 64);
+          tma_load_2d_hint(sQ + kb * 8192, &tmQ, qfull, kb * 64, r * a.n_h + hb * 64, qo_pol);
         const uint32_t idesc_qk = idesc_bf16(64, 64, false);
         const uint32_t qb = smem_u32(sQ);
         bool ok = mbar_wait(qfull, 0, abort_sm);
@@ -648,7 +659,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           if (!split) {
             const int row0 = r * a.n_h + hb * 64;
             for (int bx = 0; bx < 8; ++bx)
-              tma_store_2d(&km.o_out, stage + bx * box_bytes, bx * 64, row0);
+              tma_store_2d_hint(&km.o_out, stage + bx * box_bytes, bx * 64, row0,
+                                l2_evict_first_policy());
           } else {
             const int row0 = (sp * a.R + r) * a.n_h + hb * 64;
             for (int bx = 0; bx < 16; ++bx)
