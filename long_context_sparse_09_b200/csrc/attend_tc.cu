@@ -66,23 +66,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-constexpr int kAtKeys = 64;       // keys per tile
 constexpr int kAtThreads = 288;   // 9 warps
 constexpr int kQBytes = 64 * 1024;
-constexpr int kKBytes = 64 * 1024;
 constexpr int kPBytes = 8 * 1024;
 constexpr float kLazyRescale = 8.0f;  // log2 units: rescale when the max grows 256x
 constexpr int kMaxSlices = 8;         // key slices of one (query, head block): one cluster
 constexpr bool kAsyncGather = true;   // bf16 selected rows by cp.async (else via registers)
 
-template <bool FP8>
+// KT keys per tile, NS key-tile stages: FP8-mixed caches use 64-key tiles in
+// 2 stages (its P needs two buffers per parity), bf16 caches 48-key tiles in
+// 3 stages (a tile can load while the two before it are in use).
+template <bool FP8, int KT, int NS>
 struct AtLayout {
   static constexpr int NP = FP8 ? 2 : 1;  // P buffers per tile parity
+  static constexpr int KSTAGE = KT * 1024;  // a key tile: 8 k-blocks of KT rows x 128 B
   static constexpr int q = 0;
   static constexpr int k = kQBytes;
-  static constexpr int p = k + 2 * kKBytes;
+  static constexpr int p = k + NS * KSTAGE;
   static constexpr int meta = p + 2 * NP * kPBytes;
-  static constexpr int bars = meta + 1024;
+  static constexpr int bars = meta + 896;  // key scales [NS][64] fp32, masks [NS] u64
   static constexpr int total = bars + 256;
 };
 
@@ -119,33 +121,35 @@ struct KeyMaps {
   CUtensorMap c_box, c_row, w_box, w_row, o_out, o_ws;
 };
 
-template <bool FP8>
+template <bool FP8, int KT, int NS>
 __global__ void __launch_bounds__(kAtThreads, 1)
     attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ KeyMaps km,
               AttnTcArgs a) {
-  using L = AtLayout<FP8>;
+  using L = AtLayout<FP8, KT, NS>;
+  static_assert(KT % 16 == 0 && KT <= 64 && (!FP8 || KT == 64), "key tile");
+  constexpr int KBS = KT * 128;  // k-block stride of a key tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = sm + L::q;
   uint8_t* sK = sm + L::k;
   uint8_t* sP = sm + L::p;
-  float* meta_scale = (float*)(sm + L::meta);                       // [2][64]
-  unsigned long long* meta_mask = (unsigned long long*)(sm + L::meta + 512);  // [2]
+  float* meta_scale = (float*)(sm + L::meta);                        // [NS][64]
+  unsigned long long* meta_mask = (unsigned long long*)(sm + L::meta + 768);  // [NS]
   uint64_t* bars = (uint64_t*)(sm + L::bars);
   uint64_t* qfull = bars;
-  uint64_t* kfull = bars + 1;
-  uint64_t* kempty = bars + 3;
-  uint64_t* sfull = bars + 5;
-  uint64_t* sfree = bars + 7;
-  uint64_t* pfull = bars + 9;
-  uint64_t* pvdone = bars + 11;
-  uint32_t* tbase_sm = (uint32_t*)(bars + 13);
+  uint64_t* kfull = bars + 1;       // [NS]
+  uint64_t* kempty = kfull + NS;    // [NS]
+  uint64_t* sfull = kempty + NS;    // [2]
+  uint64_t* sfree = sfull + 2;      // [2]
+  uint64_t* pfull = sfree + 2;      // [2]
+  uint64_t* pvdone = pfull + 2;     // [2]
+  uint32_t* tbase_sm = (uint32_t*)(pvdone + 2);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
   int& valid_sm = *(int*)(tbase_sm + 2);  // the slice had keys (cluster combine)
   // slice max (base 2) and sum per head for the cluster combine; written
   // after the last tile, when the per-tile key scales are no longer read
   float2* ml_sm = (float2*)meta_scale;  // [64]
-  __shared__ const uint8_t* row_sm[kAtKeys];
+  __shared__ const uint8_t* row_sm[KT];
   __shared__ float rope_tab[64];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -158,9 +162,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qfull, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&kfull[i], 128);
       mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&sfree[i], 4);
       mbar_init(&pfull[i], 4);
@@ -188,10 +194,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const int nk = n_main + nwin_q;
   const int j_begin = sp * a.keys_per_split;
   const int j_end = min(nk, j_begin + a.keys_per_split);
-  const int ntiles = j_end > j_begin ? (j_end - j_begin + kAtKeys - 1) / kAtKeys : 0;
+  const int ntiles = j_end > j_begin ? (j_end - j_begin + KT - 1) / KT : 0;
 
   if (ntiles > 0) {
-    if (!FP8 && warp < 4) {
+    if (warp < 4) {
+     if constexpr (!FP8) {
       // ----------------------------------------------------- key loads (bf16) --
       // Contiguous 64-key runs (HCA entries, window rows) come in as TMA
       // boxes; selected rows are gathered with 16-byte loads, 16 in flight
@@ -204,22 +211,22 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       // the selected index of this thread's key in the next tile is loaded
       // one tile ahead (its latency hides behind the current tile's copies)
       auto sel_index = [&](int j) -> int {
-        return (t < kAtKeys && !a.dense && j < j_end && j < n_main)
+        return (t < KT && !a.dense && j < j_end && j < n_main)
                    ? __ldg(a.idx + (size_t)r * a.topk + j) : 0;
       };
       int e_next = sel_index(j_begin + t);
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i & 1;
-        if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
-        const int j0 = j_begin + i * kAtKeys;
+        const int s = i % NS;
+        if (!mbar_wait(&kempty[s], ((i / NS) & 1) ^ 1, abort_sm)) break;
+        const int j0 = j_begin + i * KT;
         const int e_sel = e_next;
-        e_next = sel_index(j0 + kAtKeys + t);
-        if (t < kAtKeys) {
+        e_next = sel_index(j0 + KT + t);
+        if (t < 64) {  // warps 0-1: key t of the tile (t < KT)
           const int j = j0 + t;
           int valid = 0;
           const int inwin = j >= n_main;
           const uint8_t* row = nullptr;
-          if (j < j_end) {
+          if (t < KT && j < j_end) {
             if (j < n_main) {
               const int e = a.dense ? j : e_sel;
               if (e >= 0) {
@@ -240,8 +247,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
               }
             }
           }
-          row_sm[t] = row;
-          meta_scale[s * 64 + t] = 1.f;
+          if (t < KT) {
+            row_sm[t] = row;
+            meta_scale[s * 64 + t] = 1.f;
+          }
           const unsigned vb = __ballot_sync(0xffffffffu, valid);
           if ((t & 31) == 0) reinterpret_cast<unsigned*>(&meta_mask[s])[t >> 5] = vb;
           (void)inwin;
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (t == 0) {
           // whole tile contiguous in one tensor? (entries: dense; window)
           bool ent = true, wnd = true;
-          for (int u = 0; u < kAtKeys; ++u) {
+          for (int u = 0; u < KT; ++u) {
             const int j = j0 + u;
             if (j >= n_main) ent = false; else wnd = false;
           }
@@ -258,13 +267,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           s_row0 = s_mode == 1 ? b * a.N + j0 : b * a.W + lo + (j0 - n_main) - wp0;
         }
         named_bar(1, 128);
-        uint8_t* dstK = sK + s * kKBytes;
+        uint8_t* dstK = sK + s * L::KSTAGE;
         const int mode = s_mode;
         if (mode != 0) {
-          if (t == 0) mbar_expect_tx(&kfull[s], kKBytes);
+          if (t == 0) mbar_expect_tx(&kfull[s], (uint32_t)L::KSTAGE);
           __syncwarp();
           if (t < 8)
-            tma_load_2d(dstK + t * 8192, mode == 1 ? &km.c_box : &km.w_box, &kfull[s], t * 64,
+            tma_load_2d(dstK + t * KBS, mode == 1 ? &km.c_box : &km.w_box, &kfull[s], t * 64,
                         s_row0);
           if (t != 0) mbar_arrive(&kfull[s]);
         } else if (kAsyncGather) {
@@ -272,32 +281,33 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           // into the swizzled tile (absent rows are zero-filled); the barrier
           // completes when they land, so the next tile's copies can follow
 #pragma unroll 8
-          for (int u = 0; u < 32; ++u) {
+          for (int u = 0; u < KT / 2; ++u) {
             const int idx = u * 128 + t;
             const int key = idx >> 6, ch = idx & 63;
             const int kb = ch >> 3, c = ch & 7;
             const uint8_t* src = row_sm[key];
-            cp_async16(dstK + kb * 8192 + key * 128 + ((c ^ (key & 7)) << 4),
+            cp_async16(dstK + kb * KBS + key * 128 + ((c ^ (key & 7)) << 4),
                        src ? src + ch * 16 : a.ckv, src ? 16u : 0u);
           }
           cp_async_arrive(&kfull[s]);
         } else {
 #pragma unroll 1
-          for (int it0 = 0; it0 < 32; it0 += 16) {
+          for (int it0 = 0; it0 < KT / 2; it0 += 16) {
             uint4 v[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
               const int idx = (it0 + u) * 128 + t;
               const int key = idx >> 6, ch = idx & 63;
-              const uint8_t* src = row_sm[key];
+              const uint8_t* src = it0 + u < KT / 2 ? row_sm[key] : nullptr;
               v[u] = src ? __ldg(reinterpret_cast<const uint4*>(src + ch * 16)) : zero4();
             }
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
+              if (it0 + u >= KT / 2) continue;
               const int idx = (it0 + u) * 128 + t;
               const int key = idx >> 6, ch = idx & 63;
               const int kb = ch >> 3, c = ch & 7;
-              st_shared16(dstK + kb * 8192 + key * 128 + ((c ^ (key & 7)) << 4), v[u]);
+              st_shared16(dstK + kb * KBS + key * 128 + ((c ^ (key & 7)) << 4), v[u]);
             }
           }
           fence_proxy_async_smem();
@@ -305,18 +315,18 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
         named_bar(1, 128);  // row_sm and the mode are rewritten by the next tile
       }
-    } else if (FP8 && warp < 4) {
+     } else {
       // ------------------------------------------- key gather (FP8-mixed) --
       const int t = threadIdx.x;
       const uint8_t* ckv = a.ckv + (size_t)b * a.N * rb;
       const uint8_t* win = a.win + (size_t)b * a.W * rb;
       const int wp0 = a.win ? a.win_pos0[b] : 0;
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i & 1;
-        if (!mbar_wait(&kempty[s], ((i >> 1) & 1) ^ 1, abort_sm)) break;
+        const int s = i % NS;
+        if (!mbar_wait(&kempty[s], ((i / NS) & 1) ^ 1, abort_sm)) break;
         float sc_reg = 1.f;
-        if (t < kAtKeys) {
-          const int j = j_begin + i * kAtKeys + t;
+        if (t < KT) {
+          const int j = j_begin + i * KT + t;
           int valid = 0;
           const uint8_t* row = nullptr;
           float sc = 1.f;
@@ -349,7 +359,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           if ((t & 31) == 0) reinterpret_cast<unsigned*>(&meta_mask[s])[t >> 5] = bits;
         }
         named_bar(1, 128);
-        uint8_t* dstK = sK + s * kKBytes;
+        uint8_t* dstK = sK + s * L::KSTAGE;
         // all 18 loads in flight, then widen and store
         uint4 v[18];
 #pragma unroll
@@ -370,18 +380,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             widen_e4m3(v[u], lo4, hi4);
             const int d0 = 2 * ch;  // destination chunk of dims 16ch..16ch+7
             const int kb = d0 >> 3, c0 = d0 & 7;
-            st_shared16(rowp + kb * 8192 + ((c0 ^ sw) << 4), lo4);
-            st_shared16(rowp + kb * 8192 + (((c0 + 1) ^ sw) << 4), hi4);
+            st_shared16(rowp + kb * KBS + ((c0 ^ sw) << 4), lo4);
+            st_shared16(rowp + kb * KBS + (((c0 + 1) ^ sw) << 4), hi4);
           } else {
             const int c = ch - 28;  // dims 448 + 8c .. : K-block 7
-            st_shared16(rowp + 7 * 8192 + ((c ^ sw) << 4), v[u]);
+            st_shared16(rowp + 7 * KBS + ((c ^ sw) << 4), v[u]);
           }
         }
-        if (t < kAtKeys) meta_scale[s * 64 + t] = sc_reg;
+        if (t < KT) meta_scale[s * 64 + t] = sc_reg;
         fence_proxy_async_smem();
         mbar_arrive(&kfull[s]);
         named_bar(1, 128);  // row_sm is rewritten by the next tile
       }
+     }
     } else if (warp == 4) {
       // ------------------------------------------------------------- MMA --
       if (lane == 0) {
@@ -390,18 +401,18 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         mbar_expect_tx(qfull, kQBytes);
         for (int kb = 0; kb < 8; ++kb)
           tma_load_2d_hint(sQ + kb * 8192, &tmQ, qfull, kb * 64, r * a.n_h + hb * 64, qo_pol);
-        const uint32_t idesc_qk = idesc_bf16(64, 64, false);
+        const uint32_t idesc_qk = idesc_bf16(64, KT, false);
         const uint32_t qb = smem_u32(sQ);
         bool ok = mbar_wait(qfull, 0, abort_sm);
         // S(i) = Q K(i)^T into S buffer i&1 (waits for the tile and the buffer)
         auto issue_qk = [&](int i) -> bool {
-          const int s = i & 1, bb = i & 1;
-          if (!mbar_wait(&kfull[s], (i >> 1) & 1, abort_sm)) return false;
+          const int s = i % NS, bb = i & 1;
+          if (!mbar_wait(&kfull[s], (i / NS) & 1, abort_sm)) return false;
           fence_proxy_async_smem();  // cp.async-written tile -> tensor-core reads
           if (!mbar_wait(&sfree[bb], ((i >> 1) & 1) ^ 1, abort_sm)) return false;
           tc_fence_after();
           const uint32_t sacc = tbase + ((uint32_t)(16 * bb) << 16) + 256;
-          const uint32_t kbase = smem_u32(sK + s * kKBytes);
+          const uint32_t kbase = smem_u32(sK + s * L::KSTAGE);
 #pragma unroll
           for (int kb = 0; kb < 8; ++kb) {
             const bool rope_blk = FP8 && kb == 7;
@@ -410,7 +421,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             for (int j = 0; j < 4; ++j) {
               const bool first = j == 0 && (kb == 0 || rope_blk);
               mma_bf16(d, sdesc_k_sw128(qb + kb * 8192 + j * 32),
-                       sdesc_k_sw128(kbase + kb * 8192 + j * 32), idesc_qk, first ? 0u : 1u);
+                       sdesc_k_sw128(kbase + kb * KBS + j * 32), idesc_qk, first ? 0u : 1u);
             }
           }
           mma_commit(&sfull[bb]);
@@ -418,36 +429,36 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         };
         if (ok) ok = issue_qk(0);
         for (int i = 0; ok && i < ntiles; ++i) {
-          const int s = i & 1, bb = i & 1;
+          const int s = i % NS, bb = i & 1;
           // QK(i+1) early only if its tile and S buffer are already there;
           // P V(i) must not wait behind a late tile
           bool qk_next = false;
-          if (i + 1 < ntiles && mbar_try_wait(&kfull[(i + 1) & 1], ((i + 1) >> 1) & 1) &&
+          if (i + 1 < ntiles && mbar_try_wait(&kfull[(i + 1) % NS], ((i + 1) / NS) & 1) &&
               mbar_try_wait(&sfree[(i + 1) & 1], (((i + 1) >> 1) & 1) ^ 1)) {
             if (!issue_qk(i + 1)) break;
             qk_next = true;
           }
           if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort_sm)) break;
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sK + s * kKBytes);
+          const uint32_t kbase = smem_u32(sK + s * L::KSTAGE);
           const uint32_t pb = smem_u32(sP + bb * L::NP * kPBytes);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < KT / 16; ++j) {
             const uint32_t acc = (i > 0 || j > 0) ? 1u : 0u;
             const uint32_t vb = kbase + j * 2048;  // 16 keys of the tile
-            if (!FP8) {
-              mma_bf16(tbase, sdesc_k_sw128(pb + j * 32), sdesc_mn_sw128(vb, 8192, 1024),
+            if constexpr (!FP8) {
+              mma_bf16(tbase, sdesc_k_sw128(pb + j * 32), sdesc_mn_sw128(vb, KBS, 1024),
                        idesc_bf16(64, 256, true), acc);
               mma_bf16(tbase + (16u << 16), sdesc_k_sw128(pb + j * 32),
-                       sdesc_mn_sw128(vb + 4 * 8192, 8192, 1024), idesc_bf16(64, 256, true), acc);
+                       sdesc_mn_sw128(vb + 4 * KBS, KBS, 1024), idesc_bf16(64, 256, true), acc);
             } else {
               const uint32_t ps = pb, p1 = pb + kPBytes;  // p*scale, p
-              mma_bf16(tbase, sdesc_k_sw128(ps + j * 32), sdesc_mn_sw128(vb, 8192, 1024),
+              mma_bf16(tbase, sdesc_k_sw128(ps + j * 32), sdesc_mn_sw128(vb, KBS, 1024),
                        idesc_bf16(64, 256, true), acc);
               mma_bf16(tbase + (16u << 16), sdesc_k_sw128(ps + j * 32),
-                       sdesc_mn_sw128(vb + 4 * 8192, 8192, 1024), idesc_bf16(64, 192, true), acc);
+                       sdesc_mn_sw128(vb + 4 * KBS, KBS, 1024), idesc_bf16(64, 192, true), acc);
               mma_bf16(tbase + (16u << 16) + 192, sdesc_k_sw128(p1 + j * 32),
-                       sdesc_mn_sw128(vb + 7 * 8192, 8192, 1024), idesc_bf16(64, 64, true), acc);
+                       sdesc_mn_sw128(vb + 7 * KBS, KBS, 1024), idesc_bf16(64, 64, true), acc);
             }
           }
           mma_commit(&kempty[s]);
@@ -465,19 +476,19 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       float m_used = kMasked, l = 0.f;  // running max (base 2) and sum
       bool ok = true;
       for (int i = 0; i < ntiles; ++i) {
-        const int bb = i & 1, s = i & 1;
+        const int bb = i & 1, s = i % NS;  // S / P buffer, key stage
         const bool mine = half == bb;
         if (!mbar_wait(&sfull[bb], (i >> 1) & 1, abort_sm)) { ok = false; break; }
         tc_fence_after();
-        float sv[64];
+        float sv[KT];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < KT / 16; ++c) {
           float v[16];
           tmem_ld16(trow + 256 + c * 16, v);
 #pragma unroll
           for (int u = 0; u < 16; ++u) sv[c * 16 + u] = v[u];
         }
-        if (FP8) {  // logit = scale_j * (q . codes_j) + q_rope . rope_j, 16 keys at a time
+        if constexpr (FP8) {  // logit = scale_j * (q . codes_j) + q_rope . rope_j, 16 keys at a time
           tmem_wait_ld();
           const float* scl0 = meta_scale + s * 64;
 #pragma unroll
@@ -498,7 +509,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const float* scl = meta_scale + s * 64;
         float mq[4] = {kMasked, kMasked, kMasked, kMasked};  // four short chains
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < KT; ++j) {
           const float z = ((vmask >> j) & 1ull) ? a.scale2 * sv[j] : kMasked;
           sv[j] = z;
           mq[j & 3] = fmaxf(mq[j & 3], z);
@@ -537,7 +548,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < KT; ++j) {
           const float p = sv[j] > 0.5f * kMasked ? fast_exp2(sv[j] - m_used) : 0.f;
           ls[j & 3] += p;
           sv[j] = p;
@@ -550,12 +561,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         if (mine) {
           uint8_t* prow = sP + bb * L::NP * kPBytes + hl * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < KT / 8; ++c) {
             const int off = ((c ^ (hl & 7)) << 4);
             const float* x = sv + 8 * c;
             const uint4 w1 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
                                         pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-            if (FP8) {
+            if constexpr (FP8) {
               const float* y = scl + 8 * c;
               const uint4 ws = make_uint4(pack_bf16(x[0] * y[0], x[1] * y[1]),
                                           pack_bf16(x[2] * y[2], x[3] * y[3]),
@@ -834,19 +845,25 @@ bool attend_tc_supported(const csa_params& p) {
 // Key slices per (query, head block): at most one wave of CTAs (148 SMs, one
 // CTA each).  Up to kMaxSlices slices are launched as a cluster and combined
 // in the kernel; more slices write partials for attend_combine.
+// keys per tile of the kernel instance that serves these parameters
+constexpr int kKtFp8 = 64, kNsFp8 = 2;   // FP8-mixed cache
+constexpr int kKtBf16 = 48, kNsBf16 = 3;  // bf16 cache
+static int tile_keys(const csa_params& p) { return p.kv == CSA_KV_FP8MIX ? kKtFp8 : kKtBf16; }
+
 void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps,
                     int* cluster) {
   const int hbn = (p.n_h + 63) / 64;
   const int base = R * hbn;
   const int nk_max = (dense ? N : p.topk) + p.n_win;
-  const int ntiles = (nk_max + kAtKeys - 1) / kAtKeys;
+  const int KT = tile_keys(p);
+  const int ntiles = (nk_max + KT - 1) / KT;
   int s = base >= 148 ? 1 : 148 / base;
   if (s > ntiles) s = ntiles;
   if (s > 256) s = 256;
   if (s < 1) s = 1;
   int k = (nk_max + s - 1) / s;
-  k = (k + kAtKeys - 1) / kAtKeys * kAtKeys;
-  if (k < kAtKeys) k = kAtKeys;
+  k = (k + KT - 1) / KT * KT;
+  if (k < KT) k = KT;
   *kps = k;
   *nsplit = nk_max > 0 ? (nk_max + k - 1) / k : 1;
   *cluster = *nsplit > 1 && *nsplit <= kMaxSlices;
@@ -854,11 +871,11 @@ void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, 
 
 // one CTA per (query, head block, key slice); the slices of one (query, head
 // block) are launched as a cluster
-template <bool FP8>
+template <bool FP8, int KT, int NS>
 static cudaError_t launch_attend_kernel(unsigned items, int smem, int cluster, cudaStream_t st,
                                         const CUtensorMap& tmQ, const KeyMaps& km,
                                         const AttnTcArgs& a) {
-  if (cudaFuncSetAttribute(attend_tc<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  if (cudaFuncSetAttribute(attend_tc<FP8, KT, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
@@ -882,7 +899,7 @@ static cudaError_t launch_attend_kernel(unsigned items, int smem, int cluster, c
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attend_tc<FP8>, tmQ, km, a);
+  return cudaLaunchKernelEx(&cfg, attend_tc<FP8, KT, NS>, tmQ, km, a);
 }
 
 csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
@@ -917,9 +934,9 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
     const uint64_t crows = N > 0 ? (uint64_t)B * N : (uint64_t)B * W;
     const uint64_t wrows = (W > 0 && win) ? (uint64_t)B * W : (uint64_t)B * N;
     if (crows == 0 || wrows == 0) return CSA_ERR_UNSUPPORTED;
-    if (!make_tmap_bf16(&km.c_box, cbase, crows, 512, 64) ||
+    if (!make_tmap_bf16(&km.c_box, cbase, crows, 512, kKtBf16) ||
         !make_tmap_bf16(&km.c_row, cbase, crows, 512, 1) ||
-        !make_tmap_bf16(&km.w_box, wbase, wrows, 512, 64) ||
+        !make_tmap_bf16(&km.w_box, wbase, wrows, 512, kKtBf16) ||
         !make_tmap_bf16(&km.w_row, wbase, wrows, 512, 1))
       return CSA_ERR_CUDA;
     a.R_rows_c = (int)crows;
@@ -936,11 +953,13 @@ csa_status launch_attend_tc(const csa_params& p, bool dense, int B, int Q,
   cudaError_t e;
   if (p.kv == CSA_KV_FP8MIX)
     CSA_LAUNCH(KK_ATTN, st,
-               e = launch_attend_kernel<true>((unsigned)items, AtLayout<true>::total + 1024,
+               e = launch_attend_kernel<true, kKtFp8, kNsFp8>(
+                   (unsigned)items, AtLayout<true, kKtFp8, kNsFp8>::total + 1024,
                                               cl, st, tmQ, km, a));
   else
     CSA_LAUNCH(KK_ATTN, st,
-               e = launch_attend_kernel<false>((unsigned)items, AtLayout<false>::total + 1024,
+               e = launch_attend_kernel<false, kKtBf16, kNsBf16>(
+                   (unsigned)items, AtLayout<false, kKtBf16, kNsBf16>::total + 1024,
                                                cl, st, tmQ, km, a));
   return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
