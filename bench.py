@@ -150,18 +150,19 @@ class DecodeStep:
         self.ws_a = torch.empty(max(bd.attend_workspace_bytes(self.p, B, 1, N), 1),
                                 dtype=torch.uint8, device=device)
 
-    def run(self, q=None, qI=None, w=None):
+    def run(self, q=None, qI=None, w=None, q_pos=None):
         i, wl = self.inp, self.wl
         q = i["q"] if q is None else q
+        q_pos = i["q_pos"] if q_pos is None else q_pos
         if wl.variant == "csa":
-            bd.csa_index_topk(self.p, i["q_pos"], i["qI"] if qI is None else qI,
+            bd.csa_index_topk(self.p, q_pos, i["qI"] if qI is None else qI,
                               i["w"] if w is None else w, i["kI"], self.idx,
                               workspace=self.ws_i)
-            bd.csa_attend(self.p, i["q_pos"], q, self.idx, i["ckv"], i["ckv_scale"], i["win"],
+            bd.csa_attend(self.p, q_pos, q, self.idx, i["ckv"], i["ckv_scale"], i["win"],
                           i["win_scale"], i["win_pos0"], i["sink"], self.out,
                           workspace=self.ws_a)
         else:
-            bd.hca_attend(self.p, i["q_pos"], q, i["ckv"], i["ckv_scale"], i["win"],
+            bd.hca_attend(self.p, q_pos, q, i["ckv"], i["ckv_scale"], i["win"],
                           i["win_scale"], i["win_pos0"], i["sink"], self.out,
                           workspace=self.ws_a)
 
@@ -262,14 +263,15 @@ class PrefillStep:
         self.ws_a = torch.empty(max(bd.attend_workspace_bytes(self.p, B, T, nE), 1),
                                 dtype=torch.uint8, device=device)
 
-    def run(self, H=None, q=None, qI=None, w=None):
+    def run(self, H=None, q=None, qI=None, w=None, q_pos=None):
         i = self.inp
         H = i["H"] if H is None else H
+        q_pos = i["q_pos"] if q_pos is None else q_pos
         bd.csa_compress(self.p, H, self.packed, self.ckv, None, self.kI, self.win, None,
                         workspace=self.ws_c)
-        bd.csa_index_topk(self.p, i["q_pos"], i["qI"] if qI is None else qI,
+        bd.csa_index_topk(self.p, q_pos, i["qI"] if qI is None else qI,
                           i["w"] if w is None else w, self.kI, self.idx, workspace=self.ws_i)
-        bd.csa_attend(self.p, i["q_pos"], i["q"] if q is None else q, self.idx, self.ckv, None,
+        bd.csa_attend(self.p, q_pos, i["q"] if q is None else q, self.idx, self.ckv, None,
                       self.win, None, self.win_pos0, i["sink"], self.out, workspace=self.ws_a)
 
     def step_inputs(self):
@@ -362,30 +364,47 @@ def run_ours(args, world, rank, local):
     value = units / (ms / 1e3)
     assert bd.device_status() == 0, "device error word set during the timed steps"
 
-    # end to end through the public API: pinned host inputs -> device, step,
-    # result -> pinned host, every step
+    # end to end through the public API: every step copies its inputs from
+    # pinned host memory to the device, runs the library calls eagerly and
+    # reads the result back to pinned host memory.  The copies of step k+1 run
+    # on a copy stream while step k computes (two input buffers), as a serving
+    # loop would; every copy of every timed step lies inside the timed region.
     host_in = {k: v.cpu().pin_memory() for k, v in step.step_inputs().items()}
-    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
-    host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host_in.items()} for _ in range(2)]
+    host_out = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    copy_stream = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_free:
+        e.record(stream)
 
-    def e2e_step():
-        for k, v in host_in.items():
-            dev_in[k].copy_(v, non_blocking=True)
-        kw = {"q": dev_in["q"], "qI": dev_in.get("qI"), "w": dev_in.get("w")}
-        if "H" in dev_in:
-            kw["H"] = dev_in["H"]
+    def e2e_step(k):
+        bsel = k & 1
+        copy_stream.wait_event(ev_free[bsel])  # the buffers' previous step has run
+        with torch.cuda.stream(copy_stream):
+            for name, v in host_in.items():
+                dev_in[bsel][name].copy_(v, non_blocking=True)
+            ev_in[bsel].record(copy_stream)
+        stream.wait_event(ev_in[bsel])
+        d = dev_in[bsel]
+        kw = {"q": d["q"], "qI": d.get("qI"), "w": d.get("w"), "q_pos": d["q_pos"]}
+        if "H" in d:
+            kw["H"] = d["H"]
         step.run(**kw)
-        host_out.copy_(step.out, non_blocking=True)
+        host_out[bsel].copy_(step.out, non_blocking=True)
+        ev_free[bsel].record(stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for k in range(args.warmup):
+        e2e_step(k)
     torch.cuda.synchronize()
     _barrier(world)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    for e in ev_free:
+        e.record(stream)  # the first copies start inside the timed region
+    for k in range(args.steps):
+        e2e_step(k)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)

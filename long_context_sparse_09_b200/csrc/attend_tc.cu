@@ -875,9 +875,7 @@ template <bool FP8, int KT, int NS>
 static cudaError_t launch_attend_kernel(unsigned items, int smem, int cluster, cudaStream_t st,
                                         const CUtensorMap& tmQ, const KeyMaps& km,
                                         const AttnTcArgs& a) {
-  if (cudaFuncSetAttribute(attend_tc<FP8, KT, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
-    return cudaErrorInvalidValue;
+  if (!set_kernel_smem((const void*)attend_tc<FP8, KT, NS>, smem)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(items);
   cfg.blockDim = dim3(kAtThreads);

@@ -60,6 +60,13 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Host-side caches (csa_abi.cu): SM count of the current device; a kernel's
+// dynamic shared-memory limit set once per (kernel, device, size); its
+// resident CTAs per SM queried once per (kernel, device, threads, size).
+int sm_count();
+bool set_kernel_smem(const void* kern, int smem);
+int kernel_occupancy(const void* kern, int threads, int smem);
+
 // Device error word of the current GPU (set with atomicOr from kernels).
 unsigned int* device_error_word();
 

@@ -77,6 +77,59 @@ unsigned int* device_error_word() {
   return addr[dev];
 }
 
+// ---------------------------------------------------- per-device launch caches
+// Kernel attributes and device properties persist for the process, so they
+// are set / queried once per (kernel, device) instead of on every call.
+namespace {
+struct KernelFacts {
+  const void* kern;
+  int dev, smem, threads;
+  int occupancy;  // resident CTAs per SM at (threads, smem); -1: not asked yet
+};
+std::mutex g_facts_mu;
+std::vector<KernelFacts> g_facts;
+KernelFacts* find_facts(const void* kern, int dev, int smem, int threads) {
+  for (auto& f : g_facts)
+    if (f.kern == kern && f.dev == dev && f.smem == smem && f.threads == threads) return &f;
+  return nullptr;
+}
+}  // namespace
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+int sm_count() {
+  static int cnt[64] = {0};
+  const int dev = current_device();
+  if (dev < 0 || dev >= 64) return 0;
+  if (cnt[dev] == 0) cudaDeviceGetAttribute(&cnt[dev], cudaDevAttrMultiProcessorCount, dev);
+  return cnt[dev];
+}
+
+bool set_kernel_smem(const void* kern, int smem) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_facts_mu);
+  if (find_facts(kern, dev, smem, 0)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return false;
+  g_facts.push_back({kern, dev, smem, 0, -1});
+  return true;
+}
+
+int kernel_occupancy(const void* kern, int threads, int smem) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(g_facts_mu);
+  if (KernelFacts* f = find_facts(kern, dev, smem, threads)) return f->occupancy;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess)
+    occ = 0;
+  g_facts.push_back({kern, dev, smem, threads, occ});
+  return occ;
+}
+
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 static csa_status check_params(const csa_params* p, bool need_indexer) {

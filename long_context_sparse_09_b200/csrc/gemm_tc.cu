@@ -178,12 +178,8 @@ csa_status launch_gemm_tc(const void* A, const void* B, float* C, int M, int N, 
   if (a.err == nullptr) return CSA_ERR_CUDA;
   a.tiles = ((M + kGm - 1) / kGm) * a.tiles_n;
   const int smem = 1024 + kGStages * (kGAStage + kGBStage) + 256;
-  if (cudaFuncSetAttribute(gemm_bf16_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
-    return CSA_ERR_CUDA;
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (!set_kernel_smem((const void*)gemm_bf16_tc, smem)) return CSA_ERR_CUDA;
+  const int sms = sm_count();
   const int grid = a.tiles < sms ? a.tiles : sms;
   CSA_LAUNCH(KK_GEMM, st, gemm_bf16_tc<<<grid, kGThreads, smem, st>>>(tmA, tmB, a));
   return last_launch_status();

@@ -460,10 +460,67 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps are cached per host thread (direct-mapped on the
+// pointer and shape): a decode step re-encodes the same maps every call.
+namespace {
+struct TmapKey {
+  const void* base;
+  uint64_t rows, cols;
+  uint32_t box_rows, dtype;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && box_rows == o.box_rows &&
+           dtype == o.dtype;
+  }
+};
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+constexpr int kTmapCache = 64;
+thread_local TmapEntry t_tmaps[kTmapCache];
+TmapEntry& tmap_slot(const TmapKey& k) {
+  uint64_t h = (uint64_t)(uintptr_t)k.base * 0x9E3779B97F4A7C15ull;
+  h ^= (k.rows * 31 + k.cols) * 0xC2B2AE3D27D4EB4Full + k.box_rows * 131 + k.dtype;
+  return t_tmaps[(h >> 40) % kTmapCache];
+}
+}  // namespace
+
+static bool encode_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_rows);
+static bool encode_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows);
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  const TmapKey k{base, rows, cols, box_rows, 2};
+  TmapEntry& e = tmap_slot(k);
+  if (e.valid && e.key == k) {
+    *m = e.map;
+    return true;
+  }
+  if (!encode_bf16(m, base, rows, cols, box_rows)) return false;
+  e = TmapEntry{k, *m, true};
+  return true;
+}
+
+bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  const TmapKey k{base, rows, cols, box_rows, 4};
+  TmapEntry& e = tmap_slot(k);
+  if (e.valid && e.key == k) {
+    *m = e.map;
+    return true;
+  }
+  if (!encode_f32(m, base, rows, cols, box_rows)) return false;
+  e = TmapEntry{k, *m, true};
+  return true;
+}
+
 // 2-D bf16 tensor [rows][cols] (cols contiguous), boxes of 64 x box_rows with
 // the 128-byte swizzle.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                           uint32_t box_rows) {
+static bool encode_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -477,8 +534,8 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 }
 
 // fp32 rows of `cols` floats; boxes of 32 columns (128 bytes) x box_rows rows
-bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                   uint32_t box_rows) {
+static bool encode_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -515,13 +572,9 @@ static csa_status launch_tc_t(const CUtensorMap& tmK, const CUtensorMap& tmQ,
   size_t smem = 1024 + (size_t)S * Cfg::kStageBytes + NQ * (size_t)KB * NROWS * 128 + 512 +
                 (G == 1 ? kHistBins * 4 : 0) + 80 * 4 + G * 64 * 4;
   auto kern = index_scores_tc<G, KB, S, NE, NQ>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return CSA_ERR_CUDA;
-  int dev = 0, sms = 0, occ = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
+  if (!set_kernel_smem((const void*)kern, (int)smem)) return CSA_ERR_CUDA;
+  const int sms = sm_count();
+  const int occ = kernel_occupancy((const void*)kern, Cfg::kThreads, (int)smem);
   if (occ < 1) return CSA_ERR_UNSUPPORTED;
   const int grid = sms * occ;
   CSA_LAUNCH(KK_SCORES, st, kern<<<grid, Cfg::kThreads, smem, st>>>(tmK, tmQ, a));

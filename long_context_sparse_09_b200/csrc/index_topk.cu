@@ -712,9 +712,7 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
       CSA_LAUNCH(KK_TOPK_HIST, st, topk_hist<<<grid, 1024, 0, st>>>(scores, N, q_pos, p.m, p.topk,
                                                                     mw.ghist));
     const int smem = (int)sizeof(SelectSmem);
-    if (cudaFuncSetAttribute(topk_select_final, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return CSA_ERR_CUDA;
+    if (!set_kernel_smem((const void*)topk_select_final, smem)) return CSA_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     CSA_LAUNCH(KK_TOPK_SELECT, st,
                e = launch_maybe_pdl(kPdlTopk && hist_done, topk_select_final, grid, dim3(1024),
@@ -723,9 +721,7 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   } else {
     const int smem = (int)sizeof(FastTopkSmem);
-    if (cudaFuncSetAttribute(topk_radix, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return CSA_ERR_CUDA;
+    if (!set_kernel_smem((const void*)topk_radix, smem)) return CSA_ERR_CUDA;
     CSA_LAUNCH(KK_TOPK, st, topk_radix<<<R, kTopkThreads, smem, st>>>(scores, N, q_pos, p.m,
                                                                       p.topk, idx_out, score_out));
   }
