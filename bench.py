@@ -150,20 +150,21 @@ class DecodeStep:
         self.ws_a = torch.empty(max(bd.attend_workspace_bytes(self.p, B, 1, N), 1),
                                 dtype=torch.uint8, device=device)
 
-    def run(self, q=None, qI=None, w=None, q_pos=None):
+    def run(self, q=None, qI=None, w=None, q_pos=None, out=None):
         i, wl = self.inp, self.wl
         q = i["q"] if q is None else q
+        out = self.out if out is None else out
         q_pos = i["q_pos"] if q_pos is None else q_pos
         if wl.variant == "csa":
             bd.csa_index_topk(self.p, q_pos, i["qI"] if qI is None else qI,
                               i["w"] if w is None else w, i["kI"], self.idx,
                               workspace=self.ws_i)
             bd.csa_attend(self.p, q_pos, q, self.idx, i["ckv"], i["ckv_scale"], i["win"],
-                          i["win_scale"], i["win_pos0"], i["sink"], self.out,
+                          i["win_scale"], i["win_pos0"], i["sink"], out,
                           workspace=self.ws_a)
         else:
             bd.hca_attend(self.p, q_pos, q, i["ckv"], i["ckv_scale"], i["win"],
-                          i["win_scale"], i["win_pos0"], i["sink"], self.out,
+                          i["win_scale"], i["win_pos0"], i["sink"], out,
                           workspace=self.ws_a)
 
     # per-step host<->device traffic of the end-to-end leg
@@ -263,16 +264,17 @@ class PrefillStep:
         self.ws_a = torch.empty(max(bd.attend_workspace_bytes(self.p, B, T, nE), 1),
                                 dtype=torch.uint8, device=device)
 
-    def run(self, H=None, q=None, qI=None, w=None, q_pos=None):
+    def run(self, H=None, q=None, qI=None, w=None, q_pos=None, out=None):
         i = self.inp
         H = i["H"] if H is None else H
+        out = self.out if out is None else out
         q_pos = i["q_pos"] if q_pos is None else q_pos
         bd.csa_compress(self.p, H, self.packed, self.ckv, None, self.kI, self.win, None,
                         workspace=self.ws_c)
         bd.csa_index_topk(self.p, q_pos, i["qI"] if qI is None else qI,
                           i["w"] if w is None else w, self.kI, self.idx, workspace=self.ws_i)
         bd.csa_attend(self.p, q_pos, i["q"] if q is None else q, self.idx, self.ckv, None,
-                      self.win, None, self.win_pos0, i["sink"], self.out, workspace=self.ws_a)
+                      self.win, None, self.win_pos0, i["sink"], out, workspace=self.ws_a)
 
     def step_inputs(self):
         i = self.inp
@@ -366,45 +368,59 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API: every step copies its inputs from
     # pinned host memory to the device, runs the library calls eagerly and
-    # reads the result back to pinned host memory.  The copies of step k+1 run
-    # on a copy stream while step k computes (two input buffers), as a serving
-    # loop would; every copy of every timed step lies inside the timed region.
+    # copies the result back to pinned host memory.  The copies run on two
+    # copy streams (in, out) with double buffers, so that step k+1's inputs
+    # and step k's read-back overlap the compute, as a serving loop would;
+    # every copy of every timed step lies inside the timed region.
     host_in = {k: v.cpu().pin_memory() for k, v in step.step_inputs().items()}
     dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host_in.items()} for _ in range(2)]
+    dev_out = [torch.empty_like(step.out) for _ in range(2)]
     host_out = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = host_out[0].numel() * host_out[0].element_size()
-    copy_stream = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_free = [torch.cuda.Event() for _ in range(2)]
-    for e in ev_free:
-        e.record(stream)
+    copy_stream = torch.cuda.Stream(device=dev)  # host -> device
+    back_stream = torch.cuda.Stream(device=dev)  # device -> host
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b copied
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # step on buffer b computed
+    ev_read = [torch.cuda.Event() for _ in range(2)]   # result of buffer b read back
 
     def e2e_step(k):
         bsel = k & 1
-        copy_stream.wait_event(ev_free[bsel])  # the buffers' previous step has run
         with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(ev_used[bsel])  # inputs of step k-2 no longer needed
             for name, v in host_in.items():
                 dev_in[bsel][name].copy_(v, non_blocking=True)
             ev_in[bsel].record(copy_stream)
         stream.wait_event(ev_in[bsel])
+        stream.wait_event(ev_read[bsel])  # result of step k-2 read back
         d = dev_in[bsel]
-        kw = {"q": d["q"], "qI": d.get("qI"), "w": d.get("w"), "q_pos": d["q_pos"]}
+        kw = {"q": d["q"], "qI": d.get("qI"), "w": d.get("w"), "q_pos": d["q_pos"],
+              "out": dev_out[bsel]}
         if "H" in d:
             kw["H"] = d["H"]
         step.run(**kw)
-        host_out[bsel].copy_(step.out, non_blocking=True)
-        ev_free[bsel].record(stream)
+        ev_used[bsel].record(stream)
+        with torch.cuda.stream(back_stream):
+            back_stream.wait_event(ev_used[bsel])
+            host_out[bsel].copy_(dev_out[bsel], non_blocking=True)
+            ev_read[bsel].record(back_stream)
 
+    def arm():  # the events of both buffers start out complete
+        for bsel in range(2):
+            ev_used[bsel].record(stream)
+            ev_read[bsel].record(stream)
+
+    arm()
     for k in range(args.warmup):
         e2e_step(k)
     torch.cuda.synchronize()
     _barrier(world)
     e0.record(stream)
-    for e in ev_free:
-        e.record(stream)  # the first copies start inside the timed region
+    arm()  # the first copies start inside the timed region
     for k in range(args.steps):
         e2e_step(k)
+    for bsel in range(2):
+        stream.wait_event(ev_read[bsel])  # the last results are on the host
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
