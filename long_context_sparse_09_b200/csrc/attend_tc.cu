@@ -850,6 +850,44 @@ constexpr int kKtFp8 = 64, kNsFp8 = 2;   // FP8-mixed cache
 constexpr int kKtBf16 = 48, kNsBf16 = 3;  // bf16 cache
 static int tile_keys(const csa_params& p) { return p.kv == CSA_KV_FP8MIX ? kKtFp8 : kKtBf16; }
 
+template <bool FP8, int KT, int NS>
+static int max_active_clusters_t(int csize) {
+  const int smem = AtLayout<FP8, KT, NS>::total + 1024;
+  if (!set_kernel_smem((const void*)attend_tc<FP8, KT, NS>, smem)) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(csize * 148);
+  cfg.blockDim = dim3(kAtThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attend_tc<FP8, KT, NS>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
+}
+
+// clusters of `csize` attention CTAs that fit on the current GPU at once
+static int max_active_clusters(bool fp8, int csize) {
+  static int cache[64][2][kMaxSlices + 1];
+  static bool have[64][2][kMaxSlices + 1];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || csize < 1 || csize > kMaxSlices) return 0;
+  if (!have[dev][fp8][csize]) {
+    cache[dev][fp8][csize] = fp8 ? max_active_clusters_t<true, kKtFp8, kNsFp8>(csize)
+                                 : max_active_clusters_t<false, kKtBf16, kNsBf16>(csize);
+    have[dev][fp8][csize] = true;
+  }
+  return cache[dev][fp8][csize];
+}
+
 void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps,
                     int* cluster) {
   const int hbn = (p.n_h + 63) / 64;
@@ -866,7 +904,10 @@ void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, 
   if (k < KT) k = KT;
   *kps = k;
   *nsplit = nk_max > 0 ? (nk_max + k - 1) / k : 1;
-  *cluster = *nsplit > 1 && *nsplit <= kMaxSlices;
+  // clusters only if all of them fit on the GPU at once (clusters of CTAs
+  // this large are placed whole within a GPC: 16 clusters of 8 took two waves)
+  *cluster = *nsplit > 1 && *nsplit <= kMaxSlices &&
+             base <= max_active_clusters(p.kv == CSA_KV_FP8MIX, *nsplit);
 }
 
 // one CTA per (query, head block, key slice); the slices of one (query, head
