@@ -144,6 +144,8 @@ ATTN_CASES = [
     # few queries at random positions: key slices of a cluster that hold no keys
     ("csa_bf16_split_ragged", "csa", "bf16", "bf16", 2, 3, 600, 16, 512, 64, 4, 64, 128, "prefill"),
     ("csa_fp8_split_ragged", "csa", "bf16", "fp8mix", 1, 5, 900, 64, 512, 64, 4, 128, 128, "prefill"),
+    # two head blocks of 64 (bf16 48-key tiles, clusters of slices)
+    ("csa_bf16_h128_decode", "csa", "bf16", "bf16", 2, 1, 3000, 128, 512, 64, 4, 256, 128, "decode"),
     ("hca_bf16_decode", "hca", "bf16", "bf16", 2, 1, 300, 16, 512, 64, 128, 0, 128, "decode"),
     ("hca_f32_prefill", "hca", "f32", "f32", 1, 150, 20, 4, 128, 32, 8, 0, 16, "prefill"),
     ("hca_fp8_decode", "hca", "bf16", "fp8mix", 2, 1, 260, 16, 512, 64, 128, 0, 128, "decode"),
