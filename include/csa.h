@@ -135,6 +135,42 @@ csa_status hca_compress(const csa_params* p, int B, int T, int d,
                         void* workspace, size_t ws_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_decode_append: the compressor one token at a time (decode; the same
+ * arithmetic as csa_compress, [N] eq. 9-12, 2.5.1-2.5.3).  For each sequence
+ * b the new token h_b at position t[b] (tokens 0..t[b]-1 appended before) is
+ * projected with the packed weights into row t[b] % R of the sequence's ring
+ * of the last R tokens' projections (R = 2m); when t[b] closes block
+ * i = t[b] / m (t[b] % m == m-1) entry i is folded from the ring, normalised,
+ * rotated at m*i and stored as ckv[b][i] and kI[b][i]; the window row of the
+ * token (RMSNorm + RoPE(t[b]) of C^a_t) is stored as win[b][t[b]-win_pos0[b]].
+ *   H        [B][d]               act dtype, d a multiple of 8 (bf16) or 4
+ *   t        [B] int32            positions of the new tokens
+ *   packed   from csa_pack_weights (same d)
+ *   tail     [B][R][ncols] fp32   the ring (csa_decode_tail_bytes): caller
+ *                                 owned state between calls; its rows are
+ *                                 written before they are read
+ *   ckv      [B][N][row], ckv_scale [B][N] (CSA_KV_FP8MIX, else NULL)
+ *   kI       [B][N][c_I]          act dtype
+ *   win      [B][W][row], win_scale [B][W] (CSA_KV_FP8MIX, else NULL),
+ *            win_pos0 [B] int32   position of window row 0; NULL win skips
+ * An entry index >= N or a window row outside [0, W) is skipped and raises
+ * CSA_DEV_BAD_INDEX / CSA_DEV_BAD_WINDOW in the device error word.
+ * hca_decode_append is the same with overlap = 0 (R = m, [N] eq. 20-23) and no
+ * indexer keys.
+ * ------------------------------------------------------------------------- */
+size_t csa_decode_tail_bytes(const csa_params* p, int B, int d);
+csa_status csa_decode_append(const csa_params* p, int B, int d, const void* H,
+                             const int32_t* t, const void* packed, float* tail,
+                             void* ckv, float* ckv_scale, int N, void* kI,
+                             void* win, float* win_scale, const int32_t* win_pos0,
+                             int W, csa_stream_t stream);
+csa_status hca_decode_append(const csa_params* p, int B, int d, const void* H,
+                             const int32_t* t, const void* packed, float* tail,
+                             void* ckv, float* ckv_scale, int N,
+                             void* win, float* win_scale, const int32_t* win_pos0,
+                             int W, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * csa_index_topk: Lightning-Indexer scores and top-k selection ([N] eq. 16-17,
  * [P] 2.2):  I[r][s] = sum_h w[r][h] * ReLU(qI[r][h] . kI[b][s])  for every
  * visible s, then the topk largest.  Ties are broken towards the lower index.

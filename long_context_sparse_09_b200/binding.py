@@ -60,6 +60,11 @@ _SIGS = {
     "csa_compress_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_compress": (C.c_int, [_P, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "hca_compress": (C.c_int, [_P, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "csa_decode_tail_bytes": (_sz, [_P, _i, _i]),
+    "csa_decode_append": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp,
+                                    _vp, _vp, _i, _vp]),
+    "hca_decode_append": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp,
+                                    _vp, _i, _vp]),
     "csa_index_topk_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_noalloc": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
@@ -182,6 +187,36 @@ def hca_compress(p: CsaParams, H, packed, ckv, ckv_scale, win, win_scale,
     st = lib().hca_compress(C.byref(p), B, T, d, _p(H), _p(packed), _p(ckv), _p(ckv_scale),
                             _p(win), _p(win_scale), _p(ws), wsb, _stream(stream))
     _check("hca_compress", st)
+
+
+# ------------------------------------------------------ decode: append --
+def decode_tail_bytes(p: CsaParams, B, d) -> int:
+    return lib().csa_decode_tail_bytes(C.byref(p), B, d)
+
+
+def csa_decode_append(p: CsaParams, H, t, packed, tail, ckv, ckv_scale, kI, win, win_scale,
+                      win_pos0, stream=None):
+    """H [B][d] new tokens at positions t [B]; tail from decode_tail_bytes;
+    ckv [B][N][row] (ckv_scale [B][N]), kI [B][N][c_I], win [B][W][row]
+    (win_scale [B][W]), win_pos0 [B]."""
+    B, d = H.shape
+    N = ckv.shape[1]
+    W = win.shape[1] if win is not None else 0
+    st = lib().csa_decode_append(C.byref(p), B, d, _p(H), _p(t), _p(packed), _p(tail), _p(ckv),
+                                 _p(ckv_scale), N, _p(kI), _p(win), _p(win_scale), _p(win_pos0),
+                                 W, _stream(stream))
+    _check("csa_decode_append", st)
+
+
+def hca_decode_append(p: CsaParams, H, t, packed, tail, ckv, ckv_scale, win, win_scale,
+                      win_pos0, stream=None):
+    B, d = H.shape
+    N = ckv.shape[1]
+    W = win.shape[1] if win is not None else 0
+    st = lib().hca_decode_append(C.byref(p), B, d, _p(H), _p(t), _p(packed), _p(tail), _p(ckv),
+                                 _p(ckv_scale), N, _p(win), _p(win_scale), _p(win_pos0), W,
+                                 _stream(stream))
+    _check("hca_decode_append", st)
 
 
 # --------------------------------------------------------- index / top-k --

@@ -151,31 +151,35 @@ __global__ void __launch_bounds__(256) gemm_nt_simt(const T* __restrict__ A,
 // ------------------------------------------------------------ fold / store --
 // One channel of entry i: softmax over the a rows m*i..m*i+m-1 (logit Z^a +
 // B^a) and, when overlapping and i > 0, the b rows m*(i-1)..m*i-1 (Z^b + B^b);
-// returns sum S * C over the same rows.
+// returns sum S * C over the same rows.  Token j's projections are row j of
+// Pb, or row j % ring of a ring of the last `ring` tokens (ring > 0).
 __device__ float fold_channel(const float* __restrict__ Pb, int ncols, int m,
                               int i, bool use_b, int cCa, int cZa, int cCb,
                               int cZb, const float* __restrict__ bias, int nb,
-                              int bA, int bB, int ch) {
+                              int bA, int bB, int ch, int ring = 0) {
+  auto row_of = [&](int tok) -> size_t {
+    return (size_t)(ring > 0 ? tok % ring : tok) * ncols;
+  };
   float mx = -INFINITY;
   for (int r = 0; r < m; ++r) {
-    float z = Pb[(size_t)(m * i + r) * ncols + cZa + ch] + bias[r * nb + bA + ch];
+    float z = Pb[row_of(m * i + r) + cZa + ch] + bias[r * nb + bA + ch];
     mx = fmaxf(mx, z);
   }
   if (use_b)
     for (int r = 0; r < m; ++r) {
-      float z = Pb[(size_t)(m * (i - 1) + r) * ncols + cZb + ch] + bias[r * nb + bB + ch];
+      float z = Pb[row_of(m * (i - 1) + r) + cZb + ch] + bias[r * nb + bB + ch];
       mx = fmaxf(mx, z);
     }
   float den = 0.f, num = 0.f;
   for (int r = 0; r < m; ++r) {
-    size_t row = (size_t)(m * i + r) * ncols;
+    const size_t row = row_of(m * i + r);
     float e = expf(Pb[row + cZa + ch] + bias[r * nb + bA + ch] - mx);
     den += e;
     num = fmaf(e, Pb[row + cCa + ch], num);
   }
   if (use_b)
     for (int r = 0; r < m; ++r) {
-      size_t row = (size_t)(m * (i - 1) + r) * ncols;
+      const size_t row = row_of(m * (i - 1) + r);
       float e = expf(Pb[row + cZb + ch] + bias[r * nb + bB + ch] - mx);
       den += e;
       num = fmaf(e, Pb[row + cCb + ch], num);
@@ -337,6 +341,163 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
       launch_fold<__nv_bfloat16, CSA_BF16>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
     else
       launch_fold<__nv_bfloat16, CSA_KV_FP8MIX>(p, L, P, bias, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+  }
+  return last_launch_status();
+}
+
+// ------------------------------------------------------ decode: append --
+// One new token per sequence.  Its projections P_t = h_t W (all packed
+// columns) go to row t % R of the sequence's ring of the last R tokens
+// (R = 2m with the overlapped two-window compressor, m without); when t
+// closes block i = t / m the entry i is folded from the ring exactly as in
+// the prefill (same fold, RMSNorm and RoPE at m*i, same storage); the window
+// row of token t (RMSNorm + RoPE(t) of C^a_t, or C_t) is written every step.
+
+// P_t for B tokens: warp w of a CTA computes packed column blockIdx.x*8+w for
+// every token, 16-byte loads along d (the weight row is read once).
+template <typename TA, int kMaxB>
+__global__ void __launch_bounds__(256) append_project(
+    const TA* __restrict__ H, const TA* __restrict__ Wp, int B, int d, int ncols,
+    const int32_t* __restrict__ t, float* __restrict__ tail, int R) {
+  constexpr int V = 16 / sizeof(TA);  // elements per 16-byte load
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int col = blockIdx.x * 8 + warp;
+  if (col >= ncols) return;
+  float acc[kMaxB];
+#pragma unroll
+  for (int b = 0; b < kMaxB; ++b) acc[b] = 0.f;
+  const TA* w = Wp + (size_t)col * d;
+  for (int k = lane * V; k < d; k += 32 * V) {
+    const uint4 wr = *reinterpret_cast<const uint4*>(w + k);
+    const TA* wv = reinterpret_cast<const TA*>(&wr);
+#pragma unroll
+    for (int b = 0; b < kMaxB; ++b) {
+      if (b >= B) break;
+      const uint4 hr = __ldg(reinterpret_cast<const uint4*>(H + (size_t)b * d + k));
+      const TA* hv = reinterpret_cast<const TA*>(&hr);
+#pragma unroll
+      for (int u = 0; u < V; ++u) acc[b] = fmaf(to_f32(hv[u]), to_f32(wv[u]), acc[b]);
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < kMaxB; ++b) {
+    if (b >= B) break;
+    float v = acc[b];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) tail[((size_t)b * R + (t[b] % R)) * ncols + col] = v;
+  }
+}
+
+// blockIdx.y: 0 the entry closed by token t (if any), 1 its indexer key,
+// 2 the window row of token t.
+template <typename TA, int kKV>
+__global__ void __launch_bounds__(256) append_fold(
+    const float* __restrict__ tail, int R, int ncols, const float* __restrict__ bias, int nb,
+    PackLayout L, const int32_t* __restrict__ tpos, int m, int overlap, int c, int rd, int cI,
+    float eps, double base, void* __restrict__ ckv, float* __restrict__ ckv_scale, int N,
+    TA* __restrict__ kI, void* __restrict__ win, float* __restrict__ win_scale,
+    const int32_t* __restrict__ win_pos0, int W, unsigned* __restrict__ err) {
+  extern __shared__ float xs[];  // c floats
+  __shared__ float red[32];
+  const int b = blockIdx.x, part = blockIdx.y;
+  const int t = tpos[b];
+  const float* Pb = tail + (size_t)b * R * ncols;
+  const size_t rowb = kv_row_bytes(kKV, c, rd);
+  if (part == 2) {  // window row of token t
+    if (win == nullptr) return;
+    const int wr = t - win_pos0[b];
+    if (wr < 0 || wr >= W) {
+      if (threadIdx.x == 0) atomicOr(err, CSA_DEV_BAD_WINDOW);
+      return;
+    }
+    for (int ch = threadIdx.x; ch < c; ch += blockDim.x)
+      xs[ch] = Pb[(size_t)(t % R) * ncols + L.col_Ca + ch];
+    __syncthreads();
+    norm_rope_shared(xs, c, rd, eps, (double)t, base, red);
+    const size_t e = (size_t)b * W + wr;
+    store_kv_row<kKV>(xs, c, rd, (char*)win + e * rowb, win_scale ? win_scale + e : nullptr,
+                      red);
+    return;
+  }
+  if (t % m != m - 1) return;  // no block closed by this token
+  const int i = t / m;
+  if (i >= N) {
+    if (threadIdx.x == 0) atomicOr(err, CSA_DEV_BAD_INDEX);
+    return;
+  }
+  const bool use_b = overlap && i > 0;
+  const size_t e = (size_t)b * N + i;
+  if (part == 0) {
+    for (int ch = threadIdx.x; ch < c; ch += blockDim.x)
+      xs[ch] = fold_channel(Pb, ncols, m, i, use_b, L.col_Ca, L.col_Za, L.col_Cb, L.col_Zb,
+                            bias, nb, L.b_Ba, L.b_Bb, ch, R);
+    __syncthreads();
+    norm_rope_shared(xs, c, rd, eps, (double)m * i, base, red);
+    store_kv_row<kKV>(xs, c, rd, (char*)ckv + e * rowb, ckv_scale ? ckv_scale + e : nullptr,
+                      red);
+  } else if (kI != nullptr) {
+    for (int ch = threadIdx.x; ch < cI; ch += blockDim.x)
+      kI[e * cI + ch] = from_f32<TA>(fold_channel(Pb, ncols, m, i, use_b, L.col_CIa, L.col_ZIa,
+                                                  L.col_CIb, L.col_ZIb, bias, nb, L.b_BIa,
+                                                  L.b_BIb, ch, R));
+  }
+}
+
+constexpr int kAppendMaxB = 8;  // tokens per launch of append_project
+
+int append_ring(const csa_params& p) { return p.overlap ? 2 * p.m : p.m; }
+
+size_t decode_tail_bytes(const csa_params& p, int B, int d) {
+  return (size_t)B * append_ring(p) * pack_layout(p, d).ncols * sizeof(float);
+}
+
+template <typename TA, int kKV>
+static void launch_append_fold(const csa_params& p, const PackLayout& L, int B, const float* tail,
+                               const float* bias, const int32_t* t, void* ckv, float* ckv_scale,
+                               int N, void* kI, void* win, float* win_scale,
+                               const int32_t* win_pos0, int W, cudaStream_t st) {
+  const size_t smem = (size_t)p.c * sizeof(float);
+  CSA_LAUNCH(KK_FOLD, st, append_fold<TA, kKV><<<dim3(B, 3), 256, smem, st>>>(
+      tail, append_ring(p), L.ncols, bias, L.nb, L, t, p.m, p.overlap, p.c, p.rope_dims, p.c_I,
+      p.rms_eps, (double)p.rope_base, ckv, ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W,
+      device_error_word()));
+}
+
+csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H,
+                                const int32_t* t, const void* packed, float* tail, void* ckv,
+                                float* ckv_scale, int N, void* kI, void* win, float* win_scale,
+                                const int32_t* win_pos0, int W, cudaStream_t st) {
+  const PackLayout L = pack_layout(p, d);
+  const int R = append_ring(p);
+  const float* bias = (const float*)((const char*)packed + L.bias_off);
+  if (device_error_word() == nullptr) return CSA_ERR_CUDA;
+  for (int b0 = 0; b0 < B; b0 += kAppendMaxB) {  // the projections, 8 tokens per launch
+    const int nb = B - b0 < kAppendMaxB ? B - b0 : kAppendMaxB;
+    const dim3 grid((L.ncols + 7) / 8);
+    if (p.act == CSA_F32)
+      CSA_LAUNCH(KK_GEMM, st, append_project<float, kAppendMaxB><<<grid, 256, 0, st>>>(
+          (const float*)H + (size_t)b0 * d, (const float*)packed, nb, d, L.ncols, t + b0,
+          tail + (size_t)b0 * R * L.ncols, R));
+    else
+      CSA_LAUNCH(KK_GEMM, st, append_project<__nv_bfloat16, kAppendMaxB><<<grid, 256, 0, st>>>(
+          (const __nv_bfloat16*)H + (size_t)b0 * d, (const __nv_bfloat16*)packed, nb, d,
+          L.ncols, t + b0, tail + (size_t)b0 * R * L.ncols, R));
+  }
+  if (p.act == CSA_F32) {
+    if (p.kv == CSA_F32)
+      launch_append_fold<float, CSA_F32>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+    else if (p.kv == CSA_BF16)
+      launch_append_fold<float, CSA_BF16>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+    else
+      launch_append_fold<float, CSA_KV_FP8MIX>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+  } else {
+    if (p.kv == CSA_F32)
+      launch_append_fold<__nv_bfloat16, CSA_F32>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+    else if (p.kv == CSA_BF16)
+      launch_append_fold<__nv_bfloat16, CSA_BF16>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+    else
+      launch_append_fold<__nv_bfloat16, CSA_KV_FP8MIX>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
   }
   return last_launch_status();
 }

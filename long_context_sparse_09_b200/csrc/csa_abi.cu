@@ -275,6 +275,48 @@ static csa_status compress_common(const csa_params* p, bool csa_variant, int B, 
                          workspace, S(stream));
 }
 
+size_t csa_decode_tail_bytes(const csa_params* p, int B, int d) {
+  if (check_params(p, p && p->overlap == 1) != CSA_OK || B <= 0 || d <= 0) return 0;
+  return decode_tail_bytes(*p, B, d);
+}
+
+static csa_status append_common(const csa_params* p, bool csa_variant, int B, int d,
+                                const void* H, const int32_t* t, const void* packed,
+                                float* tail, void* ckv, float* ckv_scale, int N, void* kI,
+                                void* win, float* win_scale, const int32_t* win_pos0, int W,
+                                csa_stream_t stream) {
+  csa_status st = check_params(p, csa_variant);
+  if (st != CSA_OK) return st;
+  if ((p->overlap == 1) != csa_variant) return CSA_ERR_ARG;
+  if (B <= 0 || d <= 0 || N < 0 || W < 0) return CSA_ERR_SHAPE;
+  if (d % (p->act == CSA_F32 ? 4 : 8) != 0) return CSA_ERR_SHAPE;
+  if (!H || !t || !packed || !tail || !ckv) return CSA_ERR_ARG;
+  if (csa_variant != (kI != nullptr)) return CSA_ERR_ARG;
+  const bool fp8 = p->kv == CSA_KV_FP8MIX;
+  if (fp8 && !ckv_scale) return CSA_ERR_ARG;
+  if (win && (!win_pos0 || (fp8 && !win_scale))) return CSA_ERR_ARG;
+  if (!fp8 && (ckv_scale || win_scale)) return CSA_ERR_ARG;
+  if (!aligned16(H) || !aligned16(packed) || !aligned16(tail)) return CSA_ERR_ALIGN;
+  return launch_decode_append(*p, B, d, H, t, packed, tail, ckv, ckv_scale, N, kI, win,
+                              win_scale, win_pos0, W, S(stream));
+}
+
+csa_status csa_decode_append(const csa_params* p, int B, int d, const void* H,
+                             const int32_t* t, const void* packed, float* tail, void* ckv,
+                             float* ckv_scale, int N, void* kI, void* win, float* win_scale,
+                             const int32_t* win_pos0, int W, csa_stream_t stream) {
+  return append_common(p, true, B, d, H, t, packed, tail, ckv, ckv_scale, N, kI, win,
+                       win_scale, win_pos0, W, stream);
+}
+
+csa_status hca_decode_append(const csa_params* p, int B, int d, const void* H,
+                             const int32_t* t, const void* packed, float* tail, void* ckv,
+                             float* ckv_scale, int N, void* win, float* win_scale,
+                             const int32_t* win_pos0, int W, csa_stream_t stream) {
+  return append_common(p, false, B, d, H, t, packed, tail, ckv, ckv_scale, N, nullptr, win,
+                       win_scale, win_pos0, W, stream);
+}
+
 csa_status csa_compress(const csa_params* p, int B, int T, int d, const void* H,
                         const void* packed, void* ckv, float* ckv_scale, void* kI,
                         void* win, float* win_scale, void* workspace, size_t ws_bytes,

@@ -103,6 +103,31 @@ def test_argument_errors_return_before_launch(lib):
     assert st == 4
 
 
+def test_decode_append_argument_errors(lib):
+    wl = WORKLOADS["pro_csa_decode_1m"]
+    p = bd.params_for(wl)
+    fake = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    d = wl.d
+    assert lib.csa_decode_tail_bytes(C.byref(p), 4, d) == 4 * 2 * wl.m * (4 * wl.c + 4 * wl.c_I) * 4
+    # indexer keys missing for the CSA variant
+    st = lib.csa_decode_append(C.byref(p), 4, d, fake, fake, fake, fake, fake, fake, 16, None,
+                               None, None, None, 0, None)
+    assert st == 1
+    # d not a multiple of 8 bf16 elements
+    st = lib.csa_decode_append(C.byref(p), 4, d + 4, fake, fake, fake, fake, fake, fake, 16, fake,
+                               None, None, None, 0, None)
+    assert st == 2
+    # the HCA call with CSA parameters
+    st = lib.hca_decode_append(C.byref(p), 4, d, fake, fake, fake, fake, fake, fake, 16, None,
+                               None, None, 0, None)
+    assert st == 1
+    # a window without its base positions
+    ph = bd.params_for(WORKLOADS["hca_decode_1m"])
+    st = lib.hca_decode_append(C.byref(ph), 2, wl.d, fake, fake, fake, fake, fake, None, 16, fake,
+                               None, None, 128, None)
+    assert st == 1
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(bd, "_lib", None)
     monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "libcsa.so"))

@@ -1,0 +1,106 @@
+"""Decode-time compressor (csa_decode_append / hca_decode_append) against
+the oracle: appending the tokens of a sequence one at a time must give the
+same entries, indexer keys and window rows as compressing the whole
+sequence ("DeepSeekV4技术报告阅读笔记" eq. 9-12 / 20-23, 2.5.1-2.5.3)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import pipeline as P
+from long_context_sparse_09_b200 import binding as bd, synth
+from long_context_sparse_09_b200.configs import WORKLOADS
+from gpu_util import DEV, act_dtype, alloc_kv, assert_close, kv_values, to_dev
+
+pytestmark = pytest.mark.gpu
+
+BASE = WORKLOADS["flash_csa_decode_64k"]
+
+APPEND_CASES = [
+    # name, variant, act, kv, B, T, d, c, rope, c_I, m
+    ("csa_bf16", "csa", "bf16", "bf16", 2, 42, 256, 512, 64, 128, 4),
+    ("csa_fp8", "csa", "bf16", "fp8mix", 2, 36, 128, 512, 64, 64, 4),
+    ("csa_f32", "csa", "f32", "f32", 1, 33, 96, 128, 32, 32, 4),
+    ("hca_bf16", "hca", "bf16", "bf16", 2, 50, 128, 128, 32, 0, 16),
+]
+
+
+@pytest.fixture(autouse=True)
+def _clean_status(cuda_ok):
+    bd.device_status()
+    yield
+    torch.cuda.synchronize()
+    assert bd.device_status() == 0
+
+
+def _check_fp8(got, ref, scale, wl, what):
+    nf = wl.c - wl.rope_dims
+    tol = 0.125 * np.abs(ref[:, :nf]) + scale[:, None] * 2.0 ** -9 + 1e-6
+    assert np.all(np.abs(got[:, :nf] - ref[:, :nf]) <= tol), what
+    assert_close(got[:, nf:], ref[:, nf:], "bf16", what + " rope")
+
+
+@pytest.mark.parametrize("case", APPEND_CASES, ids=[c[0] for c in APPEND_CASES])
+def test_append_matches_whole_sequence(case):
+    name, variant, act, kv, B, T, d, c, rd, ci, m = case
+    wl = BASE.with_(variant=variant, act=act, kv=kv, d=d, c=c, rope_dims=rd, c_I=ci,
+                    n_hI=4 if ci else 0, m=m, T=T, B=B, seed=len(name) + 23)
+    p = bd.params_for(wl)
+    W = synth.weights(wl)
+    H = synth.prefill_inputs(wl)["H"]  # [B][T][d]
+    packed = bd.csa_pack_weights(p, to_dev(W))
+    nE = T // m
+    ckv, ckv_s = alloc_kv(wl, (B,), nE)
+    win, win_s = alloc_kv(wl, (B,), T)
+    kI = torch.empty(B, nE, ci, dtype=act_dtype(wl), device=DEV) if variant == "csa" else None
+    tail = torch.zeros(bd.decode_tail_bytes(p, B, d) // 4, dtype=torch.float32, device=DEV)
+    win_pos0 = torch.zeros(B, dtype=torch.int32, device=DEV)
+    Hd = H.to(DEV)
+    for t in range(T):
+        h = Hd[:, t, :].contiguous()
+        tt = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        if variant == "csa":
+            bd.csa_decode_append(p, h, tt, packed, tail, ckv, ckv_s, kI, win, win_s, win_pos0)
+        else:
+            bd.hca_decode_append(p, h, tt, packed, tail, ckv, ckv_s, win, win_s, win_pos0)
+    torch.cuda.synchronize()
+    got_kv = kv_values(wl, ckv, ckv_s)
+    got_win = kv_values(wl, win, win_s)
+    for b in range(B):
+        ref_kv, ref_kI, ref_win = P.compress_seq(wl, W, H[b])
+        if kv == "fp8mix":
+            raw = oracle.norm_rope_rows(
+                oracle.compress(H[b], m, W["Wkv_a"], W["Wz_a"], W["B_a"], W["Wkv_b"], W["Wz_b"],
+                                W["B_b"]), rd, wl.rope_base, wl.rms_eps, 0.0, float(m))
+            _check_fp8(got_kv[b], raw, ckv_s[b].cpu().numpy(), wl, f"{name} kv")
+            raw_w = oracle.norm_rope_rows(oracle.matmul(H[b], W["Wkv_a"]), rd, wl.rope_base,
+                                          wl.rms_eps, 0.0, 1.0)
+            _check_fp8(got_win[b], raw_w, win_s[b].cpu().numpy(), wl, f"{name} win")
+        else:
+            fmt = wl.act if kv != "bf16" else "bf16"
+            assert_close(got_kv[b], ref_kv, fmt, f"{name} kv")
+            assert_close(got_win[b], ref_win, fmt, f"{name} win")
+        if kI is not None:
+            assert_close(kI[b].double().cpu().numpy(), ref_kI, wl.act, f"{name} kI")
+
+
+def test_append_flags_out_of_range_rows():
+    """An entry past the cache or a window row outside it is skipped and
+    reported in the device error word."""
+    wl = BASE.with_(d=64, c=128, rope_dims=32, c_I=32, n_hI=4, m=4, T=8, B=1)
+    p = bd.params_for(wl)
+    W = synth.weights(wl)
+    packed = bd.csa_pack_weights(p, to_dev(W))
+    ckv = torch.zeros(1, 1, 128, dtype=torch.bfloat16, device=DEV)
+    kI = torch.zeros(1, 1, 32, dtype=torch.bfloat16, device=DEV)
+    win = torch.zeros(1, 2, 128, dtype=torch.bfloat16, device=DEV)
+    tail = torch.zeros(bd.decode_tail_bytes(p, 1, 64) // 4, dtype=torch.float32, device=DEV)
+    h = torch.randn(1, 64, device=DEV).to(torch.bfloat16)
+    # token 7 closes block 1, but the cache holds one entry; window rows 0..1
+    tt = torch.full((1,), 7, dtype=torch.int32, device=DEV)
+    bd.csa_decode_append(p, h, tt, packed, tail, ckv, None, kI, win, None,
+                         torch.zeros(1, dtype=torch.int32, device=DEV))
+    torch.cuda.synchronize()
+    flags = bd.device_status()
+    assert flags & 0x1 and flags & 0x2
+    assert bd.device_status() == 0
