@@ -40,12 +40,14 @@ METRIC = "CSA decode query-tok/s @1M ctx & prefill tok/s; % of HBM / tensor roof
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
+L2_BYTES = 126 * 1000 * 1000  # B200 L2 capacity
+
 # ncu DRAM traffic per launch of the dominant kernel, with the hash of the
 # source file it was measured on (the value is dropped once the file changes).
 NCU_TRAFFIC = {
     # ncu --set full, pro_csa_decode_1m with 2 sequences (134.29 MB read +
     # 3.75 MB written), scaled by the units of a full launch (4 sequences)
-    "index_scores": (276.08e6, "9bec71653865"),
+    ("index_scores", "pro_csa_decode_1m"): (276.08e6, "9bec71653865"),
 }
 
 
@@ -175,6 +177,79 @@ class DecodeStep:
 
     def units(self):
         return self.wl.B  # queries per step
+
+    def time_append(self, steps, stream):
+        """Device time of the decode-time compressor for the step's tokens
+        (csa_decode_append / hca_decode_append at the workload's d; its own
+        small caches; every token closes a block, the costliest case).  One
+        graph holds one call per copy of the packed weights, the copies
+        together twice the L2, so every call streams its weights from HBM
+        and the graph launch is spread over many calls.  Returns (ms per
+        call, weight bytes per call, {kernel kind: ms per call})."""
+        wl, dev = self.wl, self.out.device
+        B, d = wl.B, wl.d
+        W = synth.weights(wl.with_(seed=wl.seed + 7), device=dev)
+        packed0 = bd.csa_pack_weights(self.p, W)
+        del W
+        ncols = (4 * wl.c + 4 * wl.c_I) if wl.variant == "csa" else 2 * wl.c
+        wbytes = ncols * d * 2
+        ncopy = max(2, min(32, -(-2 * L2_BYTES // wbytes)))
+        packs = [packed0] + [packed0.clone() for _ in range(ncopy - 1)]
+        H = torch.randn(B, d, device=dev).to(torch.bfloat16)
+        t = torch.full((B,), wl.m - 1, dtype=torch.int32, device=dev)
+        tail = torch.zeros(bd.decode_tail_bytes(self.p, B, d) // 4, dtype=torch.float32,
+                           device=dev)
+        rb = synth.kv_record_bytes(wl)
+        ckv = torch.empty(B, 1, rb, dtype=torch.uint8, device=dev)
+        win = torch.empty(B, 1, rb, dtype=torch.uint8, device=dev)
+        fp8 = wl.kv == "fp8mix"
+        ckv_s = torch.empty(B, 1, device=dev) if fp8 else None
+        win_s = torch.empty(B, 1, device=dev) if fp8 else None
+        wp0 = torch.full((B,), wl.m - 1, dtype=torch.int32, device=dev)
+        kI = torch.empty(B, 1, wl.c_I, dtype=torch.bfloat16, device=dev) if wl.variant == "csa" else None
+
+        def call(packed):
+            if wl.variant == "csa":
+                bd.csa_decode_append(self.p, H, t, packed, tail, ckv, ckv_s, kI, win, win_s, wp0)
+            else:
+                bd.hca_decode_append(self.p, H, t, packed, tail, ckv, ckv_s, win, win_s, wp0)
+
+        for pk in packs:
+            call(pk)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for pk in packs:
+                call(pk)
+        for _ in range(3):
+            g.replay()
+        reps = max(1, steps // ncopy)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / (reps * ncopy)
+        # per kernel: the same calls in a graph with the library's event pairs
+        # (an eager pass first fills the event pool, so capture creates none)
+        bd.profile_collect()
+        bd.profile_enable(True)
+        for pk in packs:
+            call(pk)
+        torch.cuda.synchronize()
+        bd.profile_collect()
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gp):
+            for pk in packs:
+                call(pk)
+        bd.profile_enable(False)
+        gp.replay()
+        torch.cuda.synchronize()
+        split = {k: round(v[0] / ncopy, 5) for k, v in bd.profile_collect().items() if v[1]}
+        assert bd.device_status() == 0, "device error word set by the decode append"
+        del g, gp, packs
+        return ms, wbytes, split
 
     def dominant(self):
         """(kernel kind, algorithmic bytes per launch, source file)."""
@@ -408,11 +483,27 @@ def run_ours(args, world, rank, local):
     # copy streams (in, out) with double buffers, so that step k+1's inputs
     # and step k's read-back overlap the compute, as a serving loop would;
     # every copy of every timed step lies inside the timed region.
-    host_in = {k: v.cpu().pin_memory() for k, v in step.step_inputs().items()}
-    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host_in.items()} for _ in range(2)]
+    # the step's inputs sit in one pinned staging buffer (each at a 256-byte
+    # offset), so that one copy per step carries them all
+    inputs = step.step_inputs()
+    offs, total = {}, 0
+    for k, v in inputs.items():
+        offs[k] = total
+        total += (v.numel() * v.element_size() + 255) // 256 * 256
+
+    def views(flat):
+        return {k: flat[offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+                for k, v in inputs.items()}
+
+    host_flat = torch.empty(total, dtype=torch.uint8).pin_memory()
+    host_in = views(host_flat)
+    for k, v in inputs.items():
+        host_in[k].copy_(v.cpu())
+    dev_flat = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dev_in = [views(f) for f in dev_flat]
     dev_out = [torch.empty_like(step.out) for _ in range(2)]
     host_out = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    h2d = total  # bytes copied per step, padding included
     d2h = host_out[0].numel() * host_out[0].element_size()
     copy_stream = torch.cuda.Stream(device=dev)  # host -> device
     back_stream = torch.cuda.Stream(device=dev)  # device -> host
@@ -424,8 +515,7 @@ def run_ours(args, world, rank, local):
         bsel = k & 1
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(ev_used[bsel])  # inputs of step k-2 no longer needed
-            for name, v in host_in.items():
-                dev_in[bsel][name].copy_(v, non_blocking=True)
+            dev_flat[bsel].copy_(host_flat, non_blocking=True)
             ev_in[bsel].record(copy_stream)
         stream.wait_event(ev_in[bsel])
         stream.wait_event(ev_read[bsel])  # result of step k-2 read back
@@ -462,6 +552,15 @@ def run_ours(args, world, rank, local):
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     assert bd.device_status() == 0, "device error word set during the timed steps"
 
+    append = None
+    if wl.mode == "decode":
+        # the decode-time compressor, timed on its own (not part of `value`)
+        a_ms, a_bytes, a_split = step.time_append(min(args.steps, 500), stream)
+        hbm0, _, _ = _peaks()
+        append = {"ms_per_call": round(a_ms, 5), "tokens": wl.B,
+                  "weight_bytes": a_bytes, "hbm_frac": round(a_bytes / (a_ms / 1e3) / 1e9 / hbm0, 4),
+                  "kernels_ms": a_split}
+
     kind, nbytes, src, bound = step.dominant()
     kms, kcnt = prof.get(kind, (0.0, 0))  # one replay: kcnt launches of the kernel
     hbm, tfl, peak_src = _peaks()
@@ -469,7 +568,7 @@ def run_ours(args, world, rank, local):
     if kcnt and bound == "hbm":
         per_launch_ms = kms / kcnt
         achieved = nbytes / (per_launch_ms / 1e3) / 1e9
-        tr = NCU_TRAFFIC.get(kind)
+        tr = NCU_TRAFFIC.get((kind, wl.name))
         traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
         roof = {"bound": bound, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": kind,
@@ -478,7 +577,7 @@ def run_ours(args, world, rank, local):
     elif kcnt:
         per_launch_ms = kms / kcnt
         achieved = nbytes / (per_launch_ms / 1e3) / 1e12
-        tr = NCU_TRAFFIC.get(kind)
+        tr = NCU_TRAFFIC.get((kind, wl.name))
         traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tfl, "unit": "TFLOP/s",
                 "frac": round(achieved / tfl, 4), "traffic": traffic, "kernel": kind,
@@ -524,6 +623,7 @@ def run_ours(args, world, rank, local):
             "ms_per_step_with_events": round(prof_ms, 5),
             "roofline": roof,
             "kernels": kernels,
+            "decode_append": append,
             "cpu_baseline": cpu,
             "clocks": clk,
         }

@@ -136,27 +136,32 @@ csa_status hca_compress(const csa_params* p, int B, int T, int d,
 
 /* ---------------------------------------------------------------------------
  * csa_decode_append: the compressor one token at a time (decode; the same
- * arithmetic as csa_compress, [N] eq. 9-12, 2.5.1-2.5.3).  For each sequence
- * b the new token h_b at position t[b] (tokens 0..t[b]-1 appended before) is
- * projected with the packed weights into row t[b] % R of the sequence's ring
- * of the last R tokens' projections (R = 2m); when t[b] closes block
- * i = t[b] / m (t[b] % m == m-1) entry i is folded from the ring, normalised,
+ * arithmetic as csa_compress, [N] eq. 9-12, 2.5.1-2.5.3, up to the order of
+ * the softmax sums).  For each sequence b the new token h_b at position t[b]
+ * (tokens 0..t[b]-1 appended before) is projected with the packed weights and
+ * folded into the running softmax of the entries it belongs to (entry
+ * t[b] / m, and entry t[b] / m + 1 through its b window): per channel the
+ * largest logit so far, the sum of exp(logit - largest) and the weighted sum
+ * of C, rescaled when a larger logit arrives.  When t[b] closes block
+ * i = t[b] / m (t[b] % m == m-1) entry i is num / den per channel, normalised,
  * rotated at m*i and stored as ckv[b][i] and kI[b][i]; the window row of the
  * token (RMSNorm + RoPE(t[b]) of C^a_t) is stored as win[b][t[b]-win_pos0[b]].
  *   H        [B][d]               act dtype, d a multiple of 8 (bf16) or 4
  *   t        [B] int32            positions of the new tokens
  *   packed   from csa_pack_weights (same d)
- *   tail     [B][R][ncols] fp32   the ring (csa_decode_tail_bytes): caller
- *                                 owned state between calls; its rows are
- *                                 written before they are read
+ *   tail     csa_decode_tail_bytes(p, B, d) bytes, fp32: caller-owned state
+ *            between calls, per sequence c floats (C^a of the last token)
+ *            then 2 slots (1 for HCA) of 3 x (c + c_I) floats (c for HCA);
+ *            entry i uses slot i % 2.  It needs no initialisation: a slot is
+ *            restarted by the first token that reaches its entry.
  *   ckv      [B][N][row], ckv_scale [B][N] (CSA_KV_FP8MIX, else NULL)
  *   kI       [B][N][c_I]          act dtype
  *   win      [B][W][row], win_scale [B][W] (CSA_KV_FP8MIX, else NULL),
  *            win_pos0 [B] int32   position of window row 0; NULL win skips
  * An entry index >= N or a window row outside [0, W) is skipped and raises
  * CSA_DEV_BAD_INDEX / CSA_DEV_BAD_WINDOW in the device error word.
- * hca_decode_append is the same with overlap = 0 (R = m, [N] eq. 20-23) and no
- * indexer keys.
+ * hca_decode_append is the same with overlap = 0 ([N] eq. 20-23, one open
+ * entry) and no indexer keys.
  * ------------------------------------------------------------------------- */
 size_t csa_decode_tail_bytes(const csa_params* p, int B, int d);
 csa_status csa_decode_append(const csa_params* p, int B, int d, const void* H,

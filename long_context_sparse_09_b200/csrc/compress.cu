@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -151,35 +152,31 @@ __global__ void __launch_bounds__(256) gemm_nt_simt(const T* __restrict__ A,
 // ------------------------------------------------------------ fold / store --
 // One channel of entry i: softmax over the a rows m*i..m*i+m-1 (logit Z^a +
 // B^a) and, when overlapping and i > 0, the b rows m*(i-1)..m*i-1 (Z^b + B^b);
-// returns sum S * C over the same rows.  Token j's projections are row j of
-// Pb, or row j % ring of a ring of the last `ring` tokens (ring > 0).
+// returns sum S * C over the same rows.
 __device__ float fold_channel(const float* __restrict__ Pb, int ncols, int m,
                               int i, bool use_b, int cCa, int cZa, int cCb,
                               int cZb, const float* __restrict__ bias, int nb,
-                              int bA, int bB, int ch, int ring = 0) {
-  auto row_of = [&](int tok) -> size_t {
-    return (size_t)(ring > 0 ? tok % ring : tok) * ncols;
-  };
+                              int bA, int bB, int ch) {
   float mx = -INFINITY;
   for (int r = 0; r < m; ++r) {
-    float z = Pb[row_of(m * i + r) + cZa + ch] + bias[r * nb + bA + ch];
+    float z = Pb[(size_t)(m * i + r) * ncols + cZa + ch] + bias[r * nb + bA + ch];
     mx = fmaxf(mx, z);
   }
   if (use_b)
     for (int r = 0; r < m; ++r) {
-      float z = Pb[row_of(m * (i - 1) + r) + cZb + ch] + bias[r * nb + bB + ch];
+      float z = Pb[(size_t)(m * (i - 1) + r) * ncols + cZb + ch] + bias[r * nb + bB + ch];
       mx = fmaxf(mx, z);
     }
   float den = 0.f, num = 0.f;
   for (int r = 0; r < m; ++r) {
-    const size_t row = row_of(m * i + r);
+    size_t row = (size_t)(m * i + r) * ncols;
     float e = expf(Pb[row + cZa + ch] + bias[r * nb + bA + ch] - mx);
     den += e;
     num = fmaf(e, Pb[row + cCa + ch], num);
   }
   if (use_b)
     for (int r = 0; r < m; ++r) {
-      const size_t row = row_of(m * (i - 1) + r);
+      size_t row = (size_t)(m * (i - 1) + r) * ncols;
       float e = expf(Pb[row + cZb + ch] + bias[r * nb + bB + ch] - mx);
       den += e;
       num = fmaf(e, Pb[row + cCb + ch], num);
@@ -346,63 +343,219 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
 }
 
 // ------------------------------------------------------ decode: append --
-// One new token per sequence.  Its projections P_t = h_t W (all packed
-// columns) go to row t % R of the sequence's ring of the last R tokens
-// (R = 2m with the overlapped two-window compressor, m without); when t
-// closes block i = t / m the entry i is folded from the ring exactly as in
-// the prefill (same fold, RMSNorm and RoPE at m*i, same storage); the window
+// One new token per sequence.  The softmax of an entry's fold is kept as a
+// running state instead of the rows it spans: per channel the largest logit
+// seen so far, the sum of exp(logit - largest) and the sum of that weight
+// times C, rescaled when a larger logit arrives.  Token t of block j = t / m
+// (row r = t % m) adds its a part (C^a, Z^a + B^a[r]) to entry j and, when
+// the windows overlap, its b part (C^b, Z^b + B^b[r]) to entry j + 1.  When t
+// closes block j (r == m-1) entry j is complete: num / den per channel, then
+// RMSNorm and RoPE at m*j and the same storage as the prefill.  The window
 // row of token t (RMSNorm + RoPE(t) of C^a_t, or C_t) is written every step.
+// Each token costs O(c) state work; nothing scales with m.
+//
+// State of one sequence (fp32): xrow[c] (C^a of the current token), then S
+// slots (S = 2 with overlap: entries j and j+1 are open at once; S = 1
+// without), each mx[nch] den[nch] num[nch] with nch = c + c_I (c without
+// indexer).  Entry i lives in slot i % S.
 
-// P_t for B tokens: warp w of a CTA computes packed column blockIdx.x*8+w for
-// every token, 16-byte loads along d (the weight row is read once).
-template <typename TA, int kMaxB>
+struct AppendState {
+  int c, cI, nch, S;
+  size_t per_seq;  // floats per sequence
+};
+
+static AppendState append_state(const csa_params& p) {
+  AppendState A;
+  A.c = p.c;
+  A.cI = p.overlap ? p.c_I : 0;
+  A.nch = A.c + A.cI;
+  A.S = p.overlap ? 2 : 1;
+  A.per_seq = (size_t)A.c + (size_t)A.S * 3 * A.nch;
+  return A;
+}
+
+// Fold one (C, z) pair into a slot's running state; `fresh` starts the entry.
+__device__ __forceinline__ void running_softmax_add(float* mx, float* den, float* num, float C,
+                                                    float z, bool fresh) {
+  if (fresh) {
+    *mx = z; *den = 1.f; *num = C;
+    return;
+  }
+  const float m0 = *mx, m1 = fmaxf(m0, z);
+  const float s0 = expf(m0 - m1), s1 = expf(z - m1);
+  *mx = m1;
+  *den = fmaf(*den, s0, s1);
+  *num = fmaf(*num, s0, s1 * C);
+}
+
+// A CTA owns 4 pairs, pair q = blockIdx.x*4 + p: the C and Z columns of one
+// channel of one part (a or b; main or indexer), computed for kB tokens (B
+// rounded up to a power of two; the rows past B are zeros and their results
+// are dropped).  d is walked in chunks of kChunk elements through a
+// kStages-deep cp.async pipeline in shared memory: each stage holds the
+// chunk of the CTA's 8 weight rows (the only HBM stream) and of the kB rows
+// of h, so several chunks are in flight while one is used.  Warps 2p and
+// 2p+1 take the even and odd halves of each chunk of pair p; the halves are
+// summed through shared memory and lane 0 of warp 2p updates the state.
+template <typename TA>
+struct AppendProj {
+  static constexpr int V = 16 / sizeof(TA);      // elements per 16-byte piece
+  static constexpr int kPieces = 64;             // 16-byte pieces per row of a chunk
+  static constexpr int kChunk = kPieces * V;     // elements of d per chunk
+  static constexpr int kStages = 3;
+  static constexpr int kThreads = 256;
+  __host__ __device__ static size_t stage_elems(int kB) { return (size_t)(8 + kB) * kChunk; }
+  static size_t smem(int kB) { return kStages * stage_elems(kB) * sizeof(TA); }
+};
+
+template <typename TA, int kB>
 __global__ void __launch_bounds__(256) append_project(
-    const TA* __restrict__ H, const TA* __restrict__ Wp, int B, int d, int ncols,
-    const int32_t* __restrict__ t, float* __restrict__ tail, int R) {
-  constexpr int V = 16 / sizeof(TA);  // elements per 16-byte load
+    const TA* __restrict__ H, const TA* __restrict__ Wp, int B, int d, PackLayout L,
+    const float* __restrict__ bias, int m, int overlap, int c, int cI,
+    const int32_t* __restrict__ tpos, float* __restrict__ state, size_t per_seq) {
+  using K = AppendProj<TA>;
+  constexpr int V = K::V, kPieces = K::kPieces, kChunk = K::kChunk, kStages = K::kStages;
+  extern __shared__ __align__(16) unsigned char append_smem[];
+  __shared__ float half_sum[4][kB][2];
+  // stage s: rows 0..7 the weight rows (row 2p the C row of pair p, 2p+1 its
+  // Z row), rows 8..8+kB-1 the rows of h; each row kChunk elements
+  TA* sm = reinterpret_cast<TA*>(append_smem);
+  constexpr size_t stage = (size_t)(8 + kB) * kChunk;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int col = blockIdx.x * 8 + warp;
-  if (col >= ncols) return;
-  float acc[kMaxB];
+  const int pp = warp >> 1, half = warp & 1;
+  const int q = blockIdx.x * 4 + pp;
+  // pair q -> (C column, Z column, bias column, state channel, part b?)
+  int colC = 0, colZ = 0, colB = 0, sch = 0;
+  bool partb = false, active = true;
+  if (q < c) {
+    colC = L.col_Ca + q; colZ = L.col_Za + q; colB = L.b_Ba + q; sch = q;
+  } else if (!overlap) {
+    active = false;
+  } else if (q < 2 * c) {
+    const int ch = q - c;
+    colC = L.col_Cb + ch; colZ = L.col_Zb + ch; colB = L.b_Bb + ch; sch = ch; partb = true;
+  } else if (q < 2 * c + cI) {
+    const int ch = q - 2 * c;
+    colC = L.col_CIa + ch; colZ = L.col_ZIa + ch; colB = L.b_BIa + ch; sch = c + ch;
+  } else if (q < 2 * c + 2 * cI) {
+    const int ch = q - 2 * c - cI;
+    colC = L.col_CIb + ch; colZ = L.col_ZIb + ch; colB = L.b_BIb + ch; sch = c + ch;
+    partb = true;
+  } else {
+    active = false;  // still takes part in the copies and barriers
+  }
+  // warp w copies weight row w: the C (even w) or Z (odd w) row of pair w/2
+  const TA* wrow = Wp + (size_t)(half ? colZ : colC) * d;
+  const int nchunk = (d + kChunk - 1) / kChunk;
+  // chunk ci into stage ci % kStages (zeros past d and past B); one group
+  auto load_chunk = [&](int ci) {
+    TA* st0 = sm + (size_t)(ci % kStages) * stage;
+    const int k0 = ci * kChunk;
 #pragma unroll
-  for (int b = 0; b < kMaxB; ++b) acc[b] = 0.f;
-  const TA* w = Wp + (size_t)col * d;
-  for (int k = lane * V; k < d; k += 32 * V) {
-    const uint4 wr = *reinterpret_cast<const uint4*>(w + k);
-    const TA* wv = reinterpret_cast<const TA*>(&wr);
+    for (int h = 0; h < 2; ++h) {
+      const int piece = lane + 32 * h;
+      const int k = k0 + piece * V;
+      const bool ok = active && k < d;
+      sm100::cp_async16(st0 + (size_t)warp * kChunk + piece * V,
+                        ok ? (const void*)(wrow + k) : (const void*)Wp, ok ? 16u : 0u);
+    }
 #pragma unroll
-    for (int b = 0; b < kMaxB; ++b) {
-      if (b >= B) break;
-      const uint4 hr = __ldg(reinterpret_cast<const uint4*>(H + (size_t)b * d + k));
-      const TA* hv = reinterpret_cast<const TA*>(&hr);
+    for (int i = threadIdx.x; i < kB * kPieces; i += K::kThreads) {
+      const int b = i / kPieces, piece = i - b * kPieces;
+      const int k = k0 + piece * V;
+      const bool ok = b < B && k < d;
+      sm100::cp_async16(st0 + (size_t)(8 + b) * kChunk + piece * V,
+                        ok ? (const void*)(H + (size_t)b * d + k) : (const void*)H,
+                        ok ? 16u : 0u);
+    }
+  };
 #pragma unroll
-      for (int u = 0; u < V; ++u) acc[b] = fmaf(to_f32(hv[u]), to_f32(wv[u]), acc[b]);
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < nchunk) load_chunk(s);
+    sm100::cp_async_commit();  // (empty groups keep the count uniform)
+  }
+  float accC[kB], accZ[kB];
+#pragma unroll
+  for (int b = 0; b < kB; ++b) accC[b] = accZ[b] = 0.f;
+  const int e0 = (lane + 32 * half) * V;  // this warp's piece of every chunk
+  for (int ci = 0; ci < nchunk; ++ci) {
+    sm100::cp_async_wait<kStages - 2>();  // chunk ci has landed (this thread's part)
+    __syncthreads();  // ... every thread's part; stage (ci-1) % kStages is free
+    if (ci + kStages - 1 < nchunk) load_chunk(ci + kStages - 1);
+    sm100::cp_async_commit();
+    if (active) {  // (past d the pieces are zeros)
+      const TA* st0 = sm + (size_t)(ci % kStages) * stage;
+      const uint4 rc = *reinterpret_cast<const uint4*>(st0 + (size_t)(2 * pp) * kChunk + e0);
+      const uint4 rz = *reinterpret_cast<const uint4*>(st0 + (size_t)(2 * pp + 1) * kChunk + e0);
+      uint4 hr[kB];
+#pragma unroll
+      for (int b = 0; b < kB; ++b)
+        hr[b] = *reinterpret_cast<const uint4*>(st0 + (size_t)(8 + b) * kChunk + e0);
+      const TA* cv = reinterpret_cast<const TA*>(&rc);
+      const TA* zv = reinterpret_cast<const TA*>(&rz);
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        const float wc = to_f32(cv[e]), wz = to_f32(zv[e]);
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          const float hx = to_f32(reinterpret_cast<const TA*>(&hr[b])[e]);
+          accC[b] = fmaf(hx, wc, accC[b]);
+          accZ[b] = fmaf(hx, wz, accZ[b]);
+        }
+      }
     }
   }
+  sm100::cp_async_wait<0>();  // (only empty groups remain)
 #pragma unroll
-  for (int b = 0; b < kMaxB; ++b) {
+  for (int b = 0; b < kB; ++b) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      accC[b] += __shfl_xor_sync(0xffffffffu, accC[b], o);
+      accZ[b] += __shfl_xor_sync(0xffffffffu, accZ[b], o);
+    }
+  }
+  if (half == 1 && lane == 0)
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      half_sum[pp][b][0] = accC[b];
+      half_sum[pp][b][1] = accZ[b];
+    }
+  __syncthreads();
+  if (!active || half == 1 || lane != 0) return;
+  const int nch = c + cI;
+  const int S = overlap ? 2 : 1;
+#pragma unroll
+  for (int b = 0; b < kB; ++b) {
     if (b >= B) break;
-    float v = acc[b];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) tail[((size_t)b * R + (t[b] % R)) * ncols + col] = v;
+    const float vC = accC[b] + half_sum[pp][b][0];
+    const float vZ = accZ[b] + half_sum[pp][b][1];
+    const int t = tpos[b];
+    const int j = t / m, r = t % m;
+    float* st = state + (size_t)b * per_seq;
+    if (q < c) st[q] = vC;  // C^a_t: the window row's source
+    // entry j (a part) or j + 1 (b part); a fresh entry starts at row 0
+    const int entry = partb ? j + 1 : j;
+    const bool fresh = r == 0 && (partb || !overlap || j == 0);
+    float* slot = st + c + (size_t)(entry % S) * 3 * nch;
+    running_softmax_add(slot + sch, slot + nch + sch, slot + 2 * nch + sch, vC,
+                        vZ + bias[r * L.nb + colB], fresh);
   }
 }
 
 // blockIdx.y: 0 the entry closed by token t (if any), 1 its indexer key,
 // 2 the window row of token t.
 template <typename TA, int kKV>
-__global__ void __launch_bounds__(256) append_fold(
-    const float* __restrict__ tail, int R, int ncols, const float* __restrict__ bias, int nb,
-    PackLayout L, const int32_t* __restrict__ tpos, int m, int overlap, int c, int rd, int cI,
-    float eps, double base, void* __restrict__ ckv, float* __restrict__ ckv_scale, int N,
-    TA* __restrict__ kI, void* __restrict__ win, float* __restrict__ win_scale,
-    const int32_t* __restrict__ win_pos0, int W, unsigned* __restrict__ err) {
+__global__ void __launch_bounds__(256) append_finish(
+    const float* __restrict__ state, size_t per_seq, const int32_t* __restrict__ tpos, int m,
+    int overlap, int c, int rd, int cI, float eps, double base, void* __restrict__ ckv,
+    float* __restrict__ ckv_scale, int N, TA* __restrict__ kI, void* __restrict__ win,
+    float* __restrict__ win_scale, const int32_t* __restrict__ win_pos0, int W,
+    unsigned* __restrict__ err) {
   extern __shared__ float xs[];  // c floats
   __shared__ float red[32];
   const int b = blockIdx.x, part = blockIdx.y;
   const int t = tpos[b];
-  const float* Pb = tail + (size_t)b * R * ncols;
+  const float* st = state + (size_t)b * per_seq;
   const size_t rowb = kv_row_bytes(kKV, c, rd);
   if (part == 2) {  // window row of token t
     if (win == nullptr) return;
@@ -411,8 +564,7 @@ __global__ void __launch_bounds__(256) append_fold(
       if (threadIdx.x == 0) atomicOr(err, CSA_DEV_BAD_WINDOW);
       return;
     }
-    for (int ch = threadIdx.x; ch < c; ch += blockDim.x)
-      xs[ch] = Pb[(size_t)(t % R) * ncols + L.col_Ca + ch];
+    for (int ch = threadIdx.x; ch < c; ch += blockDim.x) xs[ch] = st[ch];
     __syncthreads();
     norm_rope_shared(xs, c, rd, eps, (double)t, base, red);
     const size_t e = (size_t)b * W + wr;
@@ -426,41 +578,63 @@ __global__ void __launch_bounds__(256) append_fold(
     if (threadIdx.x == 0) atomicOr(err, CSA_DEV_BAD_INDEX);
     return;
   }
-  const bool use_b = overlap && i > 0;
+  const int nch = c + (overlap ? cI : 0);
+  const float* slot = st + c + (size_t)(overlap ? i % 2 : 0) * 3 * nch;
   const size_t e = (size_t)b * N + i;
   if (part == 0) {
     for (int ch = threadIdx.x; ch < c; ch += blockDim.x)
-      xs[ch] = fold_channel(Pb, ncols, m, i, use_b, L.col_Ca, L.col_Za, L.col_Cb, L.col_Zb,
-                            bias, nb, L.b_Ba, L.b_Bb, ch, R);
+      xs[ch] = slot[2 * nch + ch] / slot[nch + ch];
     __syncthreads();
     norm_rope_shared(xs, c, rd, eps, (double)m * i, base, red);
     store_kv_row<kKV>(xs, c, rd, (char*)ckv + e * rowb, ckv_scale ? ckv_scale + e : nullptr,
                       red);
-  } else if (kI != nullptr) {
+  } else if (kI != nullptr && overlap) {
     for (int ch = threadIdx.x; ch < cI; ch += blockDim.x)
-      kI[e * cI + ch] = from_f32<TA>(fold_channel(Pb, ncols, m, i, use_b, L.col_CIa, L.col_ZIa,
-                                                  L.col_CIb, L.col_ZIb, bias, nb, L.b_BIa,
-                                                  L.b_BIb, ch, R));
+      kI[e * cI + ch] = from_f32<TA>(slot[2 * nch + c + ch] / slot[nch + c + ch]);
   }
 }
 
-constexpr int kAppendMaxB = 8;  // tokens per launch of append_project
-
-int append_ring(const csa_params& p) { return p.overlap ? 2 * p.m : p.m; }
+constexpr int kAppendMaxB = 16;  // tokens per launch of append_project
 
 size_t decode_tail_bytes(const csa_params& p, int B, int d) {
-  return (size_t)B * append_ring(p) * pack_layout(p, d).ncols * sizeof(float);
+  (void)d;
+  return (size_t)B * append_state(p).per_seq * sizeof(float);
+}
+
+template <typename TA, int kB>
+static csa_status launch_append_project_kb(const csa_params& p, const PackLayout& L, int nb,
+                                           int d, const TA* H, const TA* packed,
+                                           const float* bias, const int32_t* t, float* sb,
+                                           const AppendState& A, dim3 grid, cudaStream_t st) {
+  const size_t smem = AppendProj<TA>::smem(kB);
+  if (!set_kernel_smem((const void*)append_project<TA, kB>, (int)smem)) return CSA_ERR_CUDA;
+  CSA_LAUNCH(KK_GEMM, st, append_project<TA, kB><<<grid, AppendProj<TA>::kThreads, smem, st>>>(
+      H, packed, nb, d, L, bias, p.m, p.overlap, A.c, A.cI, t, sb, A.per_seq));
+  return CSA_OK;
+}
+
+// kB = nb rounded up to a power of two (nb <= kAppendMaxB)
+template <typename TA>
+static csa_status launch_append_project(const csa_params& p, const PackLayout& L, int nb, int d,
+                                        const TA* H, const TA* packed, const float* bias,
+                                        const int32_t* t, float* sb, const AppendState& A,
+                                        dim3 grid, cudaStream_t st) {
+  if (nb <= 1) return launch_append_project_kb<TA, 1>(p, L, nb, d, H, packed, bias, t, sb, A, grid, st);
+  if (nb <= 2) return launch_append_project_kb<TA, 2>(p, L, nb, d, H, packed, bias, t, sb, A, grid, st);
+  if (nb <= 4) return launch_append_project_kb<TA, 4>(p, L, nb, d, H, packed, bias, t, sb, A, grid, st);
+  if (nb <= 8) return launch_append_project_kb<TA, 8>(p, L, nb, d, H, packed, bias, t, sb, A, grid, st);
+  return launch_append_project_kb<TA, 16>(p, L, nb, d, H, packed, bias, t, sb, A, grid, st);
 }
 
 template <typename TA, int kKV>
-static void launch_append_fold(const csa_params& p, const PackLayout& L, int B, const float* tail,
-                               const float* bias, const int32_t* t, void* ckv, float* ckv_scale,
-                               int N, void* kI, void* win, float* win_scale,
-                               const int32_t* win_pos0, int W, cudaStream_t st) {
+static void launch_append_finish(const csa_params& p, const AppendState& A, int B,
+                                 const float* state, const int32_t* t, void* ckv,
+                                 float* ckv_scale, int N, void* kI, void* win, float* win_scale,
+                                 const int32_t* win_pos0, int W, cudaStream_t st) {
   const size_t smem = (size_t)p.c * sizeof(float);
-  CSA_LAUNCH(KK_FOLD, st, append_fold<TA, kKV><<<dim3(B, 3), 256, smem, st>>>(
-      tail, append_ring(p), L.ncols, bias, L.nb, L, t, p.m, p.overlap, p.c, p.rope_dims, p.c_I,
-      p.rms_eps, (double)p.rope_base, ckv, ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W,
+  CSA_LAUNCH(KK_FOLD, st, append_finish<TA, kKV><<<dim3(B, 3), 256, smem, st>>>(
+      state, A.per_seq, t, p.m, p.overlap, p.c, p.rope_dims, A.cI, p.rms_eps,
+      (double)p.rope_base, ckv, ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W,
       device_error_word()));
 }
 
@@ -469,35 +643,37 @@ csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H
                                 float* ckv_scale, int N, void* kI, void* win, float* win_scale,
                                 const int32_t* win_pos0, int W, cudaStream_t st) {
   const PackLayout L = pack_layout(p, d);
-  const int R = append_ring(p);
+  const AppendState A = append_state(p);
   const float* bias = (const float*)((const char*)packed + L.bias_off);
   if (device_error_word() == nullptr) return CSA_ERR_CUDA;
-  for (int b0 = 0; b0 < B; b0 += kAppendMaxB) {  // the projections, 8 tokens per launch
+  const int npairs = L.ncols / 2;
+  const dim3 grid((npairs + 3) / 4);
+  for (int b0 = 0; b0 < B; b0 += kAppendMaxB) {  // the projections, kAppendMaxB tokens a launch
     const int nb = B - b0 < kAppendMaxB ? B - b0 : kAppendMaxB;
-    const dim3 grid((L.ncols + 7) / 8);
-    if (p.act == CSA_F32)
-      CSA_LAUNCH(KK_GEMM, st, append_project<float, kAppendMaxB><<<grid, 256, 0, st>>>(
-          (const float*)H + (size_t)b0 * d, (const float*)packed, nb, d, L.ncols, t + b0,
-          tail + (size_t)b0 * R * L.ncols, R));
-    else
-      CSA_LAUNCH(KK_GEMM, st, append_project<__nv_bfloat16, kAppendMaxB><<<grid, 256, 0, st>>>(
-          (const __nv_bfloat16*)H + (size_t)b0 * d, (const __nv_bfloat16*)packed, nb, d,
-          L.ncols, t + b0, tail + (size_t)b0 * R * L.ncols, R));
+    float* sb = tail + (size_t)b0 * A.per_seq;
+    const csa_status s = p.act == CSA_F32
+        ? launch_append_project<float>(p, L, nb, d, (const float*)H + (size_t)b0 * d,
+                                       (const float*)packed, bias, t + b0, sb, A, grid, st)
+        : launch_append_project<__nv_bfloat16>(p, L, nb, d,
+                                               (const __nv_bfloat16*)H + (size_t)b0 * d,
+                                               (const __nv_bfloat16*)packed, bias, t + b0, sb,
+                                               A, grid, st);
+    if (s != CSA_OK) return s;
   }
   if (p.act == CSA_F32) {
     if (p.kv == CSA_F32)
-      launch_append_fold<float, CSA_F32>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+      launch_append_finish<float, CSA_F32>(p, A, B, tail, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
     else if (p.kv == CSA_BF16)
-      launch_append_fold<float, CSA_BF16>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+      launch_append_finish<float, CSA_BF16>(p, A, B, tail, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
     else
-      launch_append_fold<float, CSA_KV_FP8MIX>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+      launch_append_finish<float, CSA_KV_FP8MIX>(p, A, B, tail, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
   } else {
     if (p.kv == CSA_F32)
-      launch_append_fold<__nv_bfloat16, CSA_F32>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+      launch_append_finish<__nv_bfloat16, CSA_F32>(p, A, B, tail, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
     else if (p.kv == CSA_BF16)
-      launch_append_fold<__nv_bfloat16, CSA_BF16>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+      launch_append_finish<__nv_bfloat16, CSA_BF16>(p, A, B, tail, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
     else
-      launch_append_fold<__nv_bfloat16, CSA_KV_FP8MIX>(p, L, B, tail, bias, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
+      launch_append_finish<__nv_bfloat16, CSA_KV_FP8MIX>(p, A, B, tail, t, ckv, ckv_scale, N, kI, win, win_scale, win_pos0, W, st);
   }
   return last_launch_status();
 }

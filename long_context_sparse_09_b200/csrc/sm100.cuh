@@ -178,6 +178,15 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
                "r"(src_bytes)
                : "memory");
 }
+// Close the group of cp.async copies issued so far by this thread; wait until
+// at most `kPending` of this thread's groups are still in flight.
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
 // Arrive on `bar` once all cp.async copies issued so far by this thread have
 // landed (the arrival counts towards the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {

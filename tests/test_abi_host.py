@@ -108,7 +108,8 @@ def test_decode_append_argument_errors(lib):
     p = bd.params_for(wl)
     fake = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
     d = wl.d
-    assert lib.csa_decode_tail_bytes(C.byref(p), 4, d) == 4 * 2 * wl.m * (4 * wl.c + 4 * wl.c_I) * 4
+    # per sequence: C^a of the last token, then two slots of (max, den, num) per channel
+    assert lib.csa_decode_tail_bytes(C.byref(p), 4, d) == 4 * (wl.c + 2 * 3 * (wl.c + wl.c_I)) * 4
     # indexer keys missing for the CSA variant
     st = lib.csa_decode_append(C.byref(p), 4, d, fake, fake, fake, fake, fake, fake, 16, None,
                                None, None, None, 0, None)

@@ -1,7 +1,8 @@
 """Decode-time compressor (csa_decode_append / hca_decode_append) against
 the oracle: appending the tokens of a sequence one at a time must give the
 same entries, indexer keys and window rows as compressing the whole
-sequence ("DeepSeekV4技术报告阅读笔记" eq. 9-12 / 20-23, 2.5.1-2.5.3)."""
+sequence ("DeepSeekV4技术报告阅读笔记" eq. 9-12 / 20-23, 2.5.1-2.5.3), up to
+the order of the softmax sums (a running maximum and rescaled sums)."""
 import numpy as np
 import pytest
 import torch
@@ -22,6 +23,10 @@ APPEND_CASES = [
     ("csa_fp8", "csa", "bf16", "fp8mix", 2, 36, 128, 512, 64, 64, 4),
     ("csa_f32", "csa", "f32", "f32", 1, 33, 96, 128, 32, 32, 4),
     ("hca_bf16", "hca", "bf16", "bf16", 2, 50, 128, 128, 32, 0, 16),
+    # more sequences than one projection launch takes (two launches)
+    ("csa_b18", "csa", "bf16", "bf16", 18, 13, 64, 128, 32, 32, 4),
+    # the heavy compression rate: entries span 128 tokens
+    ("hca_m128", "hca", "bf16", "bf16", 1, 300, 64, 128, 32, 0, 128),
 ]
 
 
@@ -53,7 +58,9 @@ def test_append_matches_whole_sequence(case):
     ckv, ckv_s = alloc_kv(wl, (B,), nE)
     win, win_s = alloc_kv(wl, (B,), T)
     kI = torch.empty(B, nE, ci, dtype=act_dtype(wl), device=DEV) if variant == "csa" else None
-    tail = torch.zeros(bd.decode_tail_bytes(p, B, d) // 4, dtype=torch.float32, device=DEV)
+    # the state needs no initialisation: every slot restarts at its entry's
+    # first token, so NaN left in it must never reach a result
+    tail = torch.full((bd.decode_tail_bytes(p, B, d) // 4,), float("nan"), device=DEV)
     win_pos0 = torch.zeros(B, dtype=torch.int32, device=DEV)
     Hd = H.to(DEV)
     for t in range(T):
