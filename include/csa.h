@@ -157,9 +157,16 @@ csa_status hca_compress(const csa_params* p, int B, int T, int d,
  *   ckv      [B][N][row], ckv_scale [B][N] (CSA_KV_FP8MIX, else NULL)
  *   kI       [B][N][c_I]          act dtype
  *   win      [B][W][row], win_scale [B][W] (CSA_KV_FP8MIX, else NULL),
- *            win_pos0 [B] int32   position of window row 0; NULL win skips
- * An entry index >= N or a window row outside [0, W) is skipped and raises
- * CSA_DEV_BAD_INDEX / CSA_DEV_BAD_WINDOW in the device error word.
+ *            win_pos0 [B] int32   position of window row 0 (device; read and
+ *                                 updated); NULL win skips the window row
+ * The window rolls: when token t[b] would land on row W (the rows are full)
+ * and W >= 2 (n_win - 1), rows W-n_win+1..W-1 move to rows 0..n_win-2,
+ * win_pos0[b] becomes t[b] - (n_win - 1) and the token's row is n_win - 1.
+ * So W = 2 n_win rows per sequence hold the window for any length, and the
+ * attention calls read the same win / win_pos0.
+ * An entry index >= N or a window row outside [0, W) that cannot be rolled
+ * is skipped and raises CSA_DEV_BAD_INDEX / CSA_DEV_BAD_WINDOW in the device
+ * error word.
  * hca_decode_append is the same with overlap = 0 ([N] eq. 20-23, one open
  * entry) and no indexer keys.
  * ------------------------------------------------------------------------- */
@@ -167,12 +174,12 @@ size_t csa_decode_tail_bytes(const csa_params* p, int B, int d);
 csa_status csa_decode_append(const csa_params* p, int B, int d, const void* H,
                              const int32_t* t, const void* packed, float* tail,
                              void* ckv, float* ckv_scale, int N, void* kI,
-                             void* win, float* win_scale, const int32_t* win_pos0,
+                             void* win, float* win_scale, int32_t* win_pos0,
                              int W, csa_stream_t stream);
 csa_status hca_decode_append(const csa_params* p, int B, int d, const void* H,
                              const int32_t* t, const void* packed, float* tail,
                              void* ckv, float* ckv_scale, int N,
-                             void* win, float* win_scale, const int32_t* win_pos0,
+                             void* win, float* win_scale, int32_t* win_pos0,
                              int W, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------

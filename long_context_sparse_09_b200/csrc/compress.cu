@@ -351,8 +351,11 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
 // the windows overlap, its b part (C^b, Z^b + B^b[r]) to entry j + 1.  When t
 // closes block j (r == m-1) entry j is complete: num / den per channel, then
 // RMSNorm and RoPE at m*j and the same storage as the prefill.  The window
-// row of token t (RMSNorm + RoPE(t) of C^a_t, or C_t) is written every step.
-// Each token costs O(c) state work; nothing scales with m.
+// row of token t (RMSNorm + RoPE(t) of C^a_t, or C_t) is written every step;
+// when the W window rows are full the last n_win - 1 of them move to the
+// front and win_pos0 advances, so W >= 2 (n_win - 1) rows per sequence
+// suffice for any length.  Each token costs O(c) state work; nothing scales
+// with m.
 //
 // State of one sequence (fp32): xrow[c] (C^a of the current token), then S
 // slots (S = 2 with overlap: entries j and j+1 are open at once; S = 1
@@ -542,14 +545,30 @@ __global__ void __launch_bounds__(256) append_project(
   }
 }
 
+// dst[0..n) = src[0..n) by the whole block (non-overlapping ranges), in the
+// widest words both addresses and n allow.
+__device__ void block_copy_bytes(char* dst, const char* src, size_t n) {
+  const uintptr_t al = (uintptr_t)dst | (uintptr_t)src | (uintptr_t)n;
+  if ((al & 15u) == 0) {
+    for (size_t i = threadIdx.x; i < n / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
+  } else if ((al & 3u) == 0) {
+    for (size_t i = threadIdx.x; i < n / 4; i += blockDim.x)
+      reinterpret_cast<uint32_t*>(dst)[i] = reinterpret_cast<const uint32_t*>(src)[i];
+  } else {
+    for (size_t i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src[i];
+  }
+}
+
 // blockIdx.y: 0 the entry closed by token t (if any), 1 its indexer key,
-// 2 the window row of token t.
+// 2 the window row of token t (rolling the window first when its rows are
+// full).
 template <typename TA, int kKV>
 __global__ void __launch_bounds__(256) append_finish(
     const float* __restrict__ state, size_t per_seq, const int32_t* __restrict__ tpos, int m,
     int overlap, int c, int rd, int cI, float eps, double base, void* __restrict__ ckv,
     float* __restrict__ ckv_scale, int N, TA* __restrict__ kI, void* __restrict__ win,
-    float* __restrict__ win_scale, const int32_t* __restrict__ win_pos0, int W,
+    float* __restrict__ win_scale, int32_t* __restrict__ win_pos0, int W, int n_win,
     unsigned* __restrict__ err) {
   extern __shared__ float xs[];  // c floats
   __shared__ float red[32];
@@ -559,7 +578,21 @@ __global__ void __launch_bounds__(256) append_finish(
   const size_t rowb = kv_row_bytes(kKV, c, rd);
   if (part == 2) {  // window row of token t
     if (win == nullptr) return;
-    const int wr = t - win_pos0[b];
+    int wr = t - win_pos0[b];
+    const int keep = n_win > 1 ? n_win - 1 : 0;  // earlier rows the window still needs
+    if (wr == W && W >= 2 * keep && W > 0) {
+      // the rows are full: roll the window.  Rows W-keep..W-1 (positions
+      // t-keep..t-1) move to rows 0..keep-1 (the ranges do not overlap) and
+      // row 0 becomes position t - keep.
+      char* wb = (char*)win + (size_t)b * W * rowb;
+      block_copy_bytes(wb, wb + (size_t)(W - keep) * rowb, (size_t)keep * rowb);
+      if (win_scale != nullptr)
+        for (int i = threadIdx.x; i < keep; i += blockDim.x)
+          win_scale[(size_t)b * W + i] = win_scale[(size_t)b * W + W - keep + i];
+      __syncthreads();  // every thread has read win_pos0 and copied its share
+      if (threadIdx.x == 0) win_pos0[b] = t - keep;
+      wr = keep;
+    }
     if (wr < 0 || wr >= W) {
       if (threadIdx.x == 0) atomicOr(err, CSA_DEV_BAD_WINDOW);
       return;
@@ -630,18 +663,18 @@ template <typename TA, int kKV>
 static void launch_append_finish(const csa_params& p, const AppendState& A, int B,
                                  const float* state, const int32_t* t, void* ckv,
                                  float* ckv_scale, int N, void* kI, void* win, float* win_scale,
-                                 const int32_t* win_pos0, int W, cudaStream_t st) {
+                                 int32_t* win_pos0, int W, cudaStream_t st) {
   const size_t smem = (size_t)p.c * sizeof(float);
   CSA_LAUNCH(KK_FOLD, st, append_finish<TA, kKV><<<dim3(B, 3), 256, smem, st>>>(
       state, A.per_seq, t, p.m, p.overlap, p.c, p.rope_dims, A.cI, p.rms_eps,
-      (double)p.rope_base, ckv, ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W,
+      (double)p.rope_base, ckv, ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W, p.n_win,
       device_error_word()));
 }
 
 csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H,
                                 const int32_t* t, const void* packed, float* tail, void* ckv,
                                 float* ckv_scale, int N, void* kI, void* win, float* win_scale,
-                                const int32_t* win_pos0, int W, cudaStream_t st) {
+                                int32_t* win_pos0, int W, cudaStream_t st) {
   const PackLayout L = pack_layout(p, d);
   const AppendState A = append_state(p);
   const float* bias = (const float*)((const char*)packed + L.bias_off);

@@ -283,7 +283,7 @@ size_t csa_decode_tail_bytes(const csa_params* p, int B, int d) {
 static csa_status append_common(const csa_params* p, bool csa_variant, int B, int d,
                                 const void* H, const int32_t* t, const void* packed,
                                 float* tail, void* ckv, float* ckv_scale, int N, void* kI,
-                                void* win, float* win_scale, const int32_t* win_pos0, int W,
+                                void* win, float* win_scale, int32_t* win_pos0, int W,
                                 csa_stream_t stream) {
   csa_status st = check_params(p, csa_variant);
   if (st != CSA_OK) return st;
@@ -304,7 +304,7 @@ static csa_status append_common(const csa_params* p, bool csa_variant, int B, in
 csa_status csa_decode_append(const csa_params* p, int B, int d, const void* H,
                              const int32_t* t, const void* packed, float* tail, void* ckv,
                              float* ckv_scale, int N, void* kI, void* win, float* win_scale,
-                             const int32_t* win_pos0, int W, csa_stream_t stream) {
+                             int32_t* win_pos0, int W, csa_stream_t stream) {
   return append_common(p, true, B, d, H, t, packed, tail, ckv, ckv_scale, N, kI, win,
                        win_scale, win_pos0, W, stream);
 }
@@ -312,7 +312,7 @@ csa_status csa_decode_append(const csa_params* p, int B, int d, const void* H,
 csa_status hca_decode_append(const csa_params* p, int B, int d, const void* H,
                              const int32_t* t, const void* packed, float* tail, void* ckv,
                              float* ckv_scale, int N, void* win, float* win_scale,
-                             const int32_t* win_pos0, int W, csa_stream_t stream) {
+                             int32_t* win_pos0, int W, csa_stream_t stream) {
   return append_common(p, false, B, d, H, t, packed, tail, ckv, ckv_scale, N, nullptr, win,
                        win_scale, win_pos0, W, stream);
 }

@@ -35,7 +35,7 @@ size_t decode_tail_bytes(const csa_params& p, int B, int d);
 csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H,
                                 const int32_t* t, const void* packed, float* tail, void* ckv,
                                 float* ckv_scale, int N, void* kI, void* win, float* win_scale,
-                                const int32_t* win_pos0, int W, cudaStream_t st);
+                                int32_t* win_pos0, int W, cudaStream_t st);
 
 size_t index_topk_ws_bytes(const csa_params& p, int B, int Q, int N);
 csa_status launch_index_topk(const csa_params& p, int B, int Q,

@@ -11,7 +11,8 @@ import oracle
 from oracle import pipeline as P
 from long_context_sparse_09_b200 import binding as bd, synth
 from long_context_sparse_09_b200.configs import WORKLOADS
-from gpu_util import DEV, act_dtype, alloc_kv, assert_close, kv_values, to_dev
+from gpu_util import (DEV, act_dtype, alloc_kv, assert_close, check_topk, kv_values,
+                      score_tolerance, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -111,3 +112,84 @@ def test_append_flags_out_of_range_rows():
     flags = bd.device_status()
     assert flags & 0x1 and flags & 0x2
     assert bd.device_status() == 0
+
+
+@pytest.mark.parametrize("variant", ["csa", "hca"])
+def test_incremental_decode_rolls_the_window(variant):
+    """The self-contained decode step: append token t, then select and
+    attend for the query at t.  The window holds 2 n_win rows and rolls
+    several times; after each checked step the rows of positions
+    t-n_win+1..t equal the oracle's window rows, and the attention output
+    over the step's caches equals the oracle's."""
+    nwin, m = 6, 4
+    wl = BASE.with_(variant=variant, act="bf16", kv="bf16", d=64, c=128, rope_dims=32,
+                    c_I=32 if variant == "csa" else 0, n_hI=4 if variant == "csa" else 0,
+                    n_h=4, m=m, topk=4 if variant == "csa" else 0, n_win=nwin, T=44, B=2,
+                    seed=71)
+    p = bd.params_for(wl)
+    B, T, d = wl.B, wl.T, wl.d
+    W = synth.weights(wl)
+    H = synth.prefill_inputs(wl)["H"]
+    packed = bd.csa_pack_weights(p, to_dev(W))
+    nE = T // m
+    Wrows = 2 * nwin
+    ckv, _ = alloc_kv(wl, (B,), nE)
+    win, _ = alloc_kv(wl, (B,), Wrows)
+    ckv.zero_()
+    win.zero_()
+    kI = torch.zeros(B, nE, wl.c_I, dtype=torch.bfloat16, device=DEV) if variant == "csa" else None
+    tail = torch.full((bd.decode_tail_bytes(p, B, d) // 4,), float("nan"), device=DEV)
+    win_pos0 = torch.zeros(B, dtype=torch.int32, device=DEV)
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(T, B, wl.n_h, wl.c, generator=g).to(torch.bfloat16)
+    sink = torch.randn(wl.n_h, generator=g)
+    if variant == "csa":
+        qI = torch.randn(T, B, wl.n_hI, wl.c_I, generator=g).to(torch.bfloat16)
+        w = torch.randn(T, B, wl.n_hI, generator=g)
+    ref = [P.compress_seq(wl, W, H[b]) for b in range(B)]  # (kv, kI, win) per sequence
+    Hd = H.to(DEV)
+    checked = {0, 3, 5, 11, 12, 13, 19, 30, 31, 43}
+    for t in range(T):
+        tt = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        h = Hd[:, t, :].contiguous()
+        if variant == "csa":
+            bd.csa_decode_append(p, h, tt, packed, tail, ckv, None, kI, win, None, win_pos0)
+        else:
+            bd.hca_decode_append(p, h, tt, packed, tail, ckv, None, win, None, win_pos0)
+        if t not in checked:
+            continue
+        out = torch.empty(B, wl.n_h, wl.c, dtype=torch.bfloat16, device=DEV)
+        qd = q[t].to(DEV)
+        if variant == "csa":
+            idx = torch.empty(B, wl.topk, dtype=torch.int32, device=DEV)
+            sco = torch.empty(B, wl.topk, device=DEV)
+            bd.csa_index_topk(p, tt, qI[t].to(DEV), w[t].to(DEV), kI, idx, sco)
+            bd.csa_attend(p, tt, qd, idx, ckv, None, win, None, win_pos0, sink.to(DEV), out)
+        else:
+            bd.hca_attend(p, tt, qd, ckv, None, win, None, win_pos0, sink.to(DEV), out)
+        torch.cuda.synchronize()
+        wp0 = win_pos0.cpu().numpy()
+        for b in range(B):
+            lo = max(0, t - nwin + 1)
+            assert wp0[b] <= lo and t - wp0[b] < Wrows, (t, b, wp0[b])
+            got_w = kv_values(wl, win[b].cpu(), None)
+            assert_close(got_w[lo - wp0[b]: t - wp0[b] + 1], ref[b][2][lo: t + 1], "bf16",
+                         f"{variant} t{t} b{b} window")
+            kv_b = kv_values(wl, ckv[b].cpu(), None)
+            pos = np.array([t], dtype=np.int32)
+            if variant == "csa":
+                kIb = kI[b].cpu()
+                sref = oracle.index_scores(pos, m, qI[t, b:b + 1], w[t, b:b + 1], kIb)
+                tol = score_tolerance(qI[t, b:b + 1].double().numpy(), w[t, b:b + 1].numpy(),
+                                      kIb.double().numpy())
+                nv = np.array([oracle.nvis(t, m, nE)])
+                ig = idx[b:b + 1].cpu().numpy()
+                check_topk(ig, sco[b:b + 1].cpu().numpy(), sref, nv, wl.topk, tol,
+                           f"t{t} b{b}")
+                sel = ig[0][ig[0] >= 0]
+                oref, _ = oracle.attend(pos, q[t, b:b + 1], np.arange(len(sel), dtype=np.int32)[None],
+                                        m, kv_b[sel], nwin, got_w, int(wp0[b]), sink,
+                                        wl.rope_dims, wl.rope_base, wl.softmax_scale)
+            else:
+                oref, _ = P.attend_wl(wl, pos, q[t, b:b + 1], None, kv_b, got_w, int(wp0[b]), sink)
+            assert_close(out[b:b + 1].double().cpu().numpy(), oref, "bf16", f"{variant} t{t} b{b} out")
