@@ -39,6 +39,7 @@ void prof_end(int slot, cudaStream_t st);
 constexpr bool kPdlAttend = true;   // attention after the top-k
 constexpr bool kPdlTopk = false;    // top-k select after the scorer (measured slower)
 constexpr bool kPdlCombine = false; // slice combine after the attention (no gain)
+constexpr bool kPdlAppend = true;   // decode compressor: finish after the projection
 // launch with the programmatic-dependent attribute when `pdl` is set
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_maybe_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
@@ -114,6 +115,22 @@ __device__ __forceinline__ void rope_cs(double pos, int p, int rope_dims,
   sincos(pos * theta, &s, &c);
   *cs = (float)c;
   *sn = (float)s;
+}
+
+// Decode compressor: fold one (C, z) pair into an open entry's running
+// softmax (largest logit, denominator, weighted sum of C); `fresh` starts
+// the entry.
+__device__ __forceinline__ void running_softmax_add(float* mx, float* den, float* num, float C,
+                                                    float z, bool fresh) {
+  if (fresh) {
+    *mx = z; *den = 1.f; *num = C;
+    return;
+  }
+  const float m0 = *mx, m1 = fmaxf(m0, z);
+  const float s0 = expf(m0 - m1), s1 = expf(z - m1);
+  *mx = m1;
+  *den = fmaf(*den, s0, s1);
+  *num = fmaf(*num, s0, s1 * C);
 }
 
 // ------------------------------------------------------------ reductions --

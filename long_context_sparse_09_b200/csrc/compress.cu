@@ -377,20 +377,6 @@ static AppendState append_state(const csa_params& p) {
   return A;
 }
 
-// Fold one (C, z) pair into a slot's running state; `fresh` starts the entry.
-__device__ __forceinline__ void running_softmax_add(float* mx, float* den, float* num, float C,
-                                                    float z, bool fresh) {
-  if (fresh) {
-    *mx = z; *den = 1.f; *num = C;
-    return;
-  }
-  const float m0 = *mx, m1 = fmaxf(m0, z);
-  const float s0 = expf(m0 - m1), s1 = expf(z - m1);
-  *mx = m1;
-  *den = fmaf(*den, s0, s1);
-  *num = fmaf(*num, s0, s1 * C);
-}
-
 // A CTA owns 4 pairs, pair q = blockIdx.x*4 + p: the C and Z columns of one
 // channel of one part (a or b; main or indexer), computed for kB tokens (B
 // rounded up to a power of two; the rows past B are zeros and their results
@@ -572,6 +558,8 @@ __global__ void __launch_bounds__(256) append_finish(
     unsigned* __restrict__ err) {
   extern __shared__ float xs[];  // c floats
   __shared__ float red[32];
+  pdl_wait();     // launched as a programmatic dependent of the projection
+  pdl_trigger();  // a following dependent may set up meanwhile (it waits for us)
   const int b = blockIdx.x, part = blockIdx.y;
   const int t = tpos[b];
   const float* st = state + (size_t)b * per_seq;
@@ -665,10 +653,14 @@ static void launch_append_finish(const csa_params& p, const AppendState& A, int 
                                  float* ckv_scale, int N, void* kI, void* win, float* win_scale,
                                  int32_t* win_pos0, int W, cudaStream_t st) {
   const size_t smem = (size_t)p.c * sizeof(float);
-  CSA_LAUNCH(KK_FOLD, st, append_finish<TA, kKV><<<dim3(B, 3), 256, smem, st>>>(
-      state, A.per_seq, t, p.m, p.overlap, p.c, p.rope_dims, A.cI, p.rms_eps,
-      (double)p.rope_base, ckv, ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W, p.n_win,
-      device_error_word()));
+  cudaError_t e = cudaSuccess;
+  CSA_LAUNCH(KK_FOLD, st,
+             e = launch_maybe_pdl(kPdlAppend, append_finish<TA, kKV>, dim3(B, 3), dim3(256), smem,
+                                  st, (const float*)state, A.per_seq, t, p.m, p.overlap, p.c,
+                                  p.rope_dims, A.cI, p.rms_eps, (double)p.rope_base, ckv,
+                                  ckv_scale, N, (TA*)kI, win, win_scale, win_pos0, W, p.n_win,
+                                  device_error_word()));
+  (void)e;  // a failed launch is reported by last_launch_status()
 }
 
 csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H,
@@ -684,6 +676,13 @@ csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H
   for (int b0 = 0; b0 < B; b0 += kAppendMaxB) {  // the projections, kAppendMaxB tokens a launch
     const int nb = B - b0 < kAppendMaxB ? B - b0 : kAppendMaxB;
     float* sb = tail + (size_t)b0 * A.per_seq;
+    if (append_tc_supported(p, nb)) {  // bf16: the tensor-core projection
+      const csa_status s = launch_append_project_tc(
+          p, L, nb, d, (const __nv_bfloat16*)H + (size_t)b0 * d, packed, bias, t + b0, sb,
+          A.cI, A.per_seq, st);
+      if (s != CSA_OK) return s;
+      continue;
+    }
     const csa_status s = p.act == CSA_F32
         ? launch_append_project<float>(p, L, nb, d, (const float*)H + (size_t)b0 * d,
                                        (const float*)packed, bias, t + b0, sb, A, grid, st)

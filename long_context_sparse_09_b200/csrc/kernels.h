@@ -32,6 +32,12 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
                            float* win_scale, void* ws, cudaStream_t st);
 
 size_t decode_tail_bytes(const csa_params& p, int B, int d);
+// decode append, tensor-core projection (bf16, at most 16 tokens a launch)
+bool append_tc_supported(const csa_params& p, int nb);
+csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, int nb, int d,
+                                    const void* H, const void* packed, const float* bias,
+                                    const int32_t* t, float* state, int cI, size_t per_seq,
+                                    cudaStream_t st);
 csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H,
                                 const int32_t* t, const void* packed, float* tail, void* ckv,
                                 float* ckv_scale, int N, void* kI, void* win, float* win_scale,

@@ -147,6 +147,12 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
                : "memory");
   return v;
 }
+// (no memory clobber: used after a cluster barrier, between reads only)
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ float2 ld_dsmem_f2(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
