@@ -68,6 +68,8 @@ def _load():
                                 C.c_int, C.c_int, _dp, C.c_int, C.c_int, C.c_int,
                                 C.c_void_p, _dp, C.c_double, _dp, C.c_void_p]
     lib.ocsa_round_bf16.argtypes = [C.c_int, _dp, _dp]
+    lib.ocsa_group_out_proj.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                        _dp, _dp, _dp, C.c_int, _dp, _dp]
     lib.ocsa_e4m3_decode.restype = C.c_double
     lib.ocsa_e4m3_decode.argtypes = [C.c_uint8]
     lib.ocsa_e4m3_encode.restype = C.c_uint8
@@ -203,6 +205,21 @@ def attend(t0s, q, idx, m: int, kv, n_win: int, win, win_pos0: int, sink,
     if rc != 0:
         raise ValueError("attend: an index or a window row is out of range")
     return out, mass
+
+
+def group_out_proj(O, WG, WO, round_mid: bool = True):
+    """(Y [Q][g d_g], out [Q][d]) of the grouped output projection: O
+    [Q][n_h][c], WG [g][c n_h/g][d_g], WO [g d_g][d]."""
+    O, WG, WO = _f64(O), _f64(WG), _f64(WO)
+    Q, n_h, c = O.shape
+    g, Kg, d_g = WG.shape
+    d = WO.shape[1]
+    if Kg * g != n_h * c or WO.shape[0] != g * d_g or n_h % g:
+        raise ValueError("group_out_proj: shapes do not agree")
+    Y = np.empty((Q, g * d_g))
+    out = np.empty((Q, d))
+    _load().ocsa_group_out_proj(Q, n_h, c, g, d_g, d, O, WG, WO, 1 if round_mid else 0, Y, out)
+    return Y, out
 
 
 def round_bf16(x) -> np.ndarray:

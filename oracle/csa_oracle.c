@@ -405,3 +405,44 @@ void ocsa_fp8mix_decode(int n, int c, int rope_dims, const uint8_t* codes,
     }
   }
 }
+
+/* [N] 2.3.3 "Grouped Output Projection"; [P] 2.2.  The attention output o_t
+ * (n_h heads of c values) is cut into g groups of n_h / g consecutive heads;
+ * group i (c n_h / g values) times W^G_i ((c n_h / g) x d_g) gives o'_i
+ * (d_g values); the concatenation [o'_1; ...; o'_g] (g d_g values) times W^O
+ * ((g d_g) x d) gives the layer output (d values).  Reading: consecutive
+ * heads form a group; with round_mid the group outputs are rounded to bf16
+ * before W^O, as a bf16 model stores the activation between the two
+ * projections.
+ *   O   [Q][n_h][c]       WG [g][c n_h / g][d_g]       WO [g d_g][d]
+ *   Y   [Q][g d_g] (the group outputs, after rounding when asked)
+ *   out [Q][d] */
+void ocsa_group_out_proj(int Q, int n_h, int c, int g, int d_g, int d, const double* O,
+                         const double* WG, const double* WO, int round_mid, double* Y,
+                         double* out) {
+  const int Kg = c * (n_h / g);
+#pragma omp parallel for schedule(static)
+  for (int q = 0; q < Q; ++q) {
+    const double* o = O + (size_t)q * n_h * c;
+    double* y = Y + (size_t)q * g * d_g;
+    for (int i = 0; i < g; ++i) {
+      const double* oi = o + (size_t)i * Kg;  /* heads i n_h/g .. (i+1) n_h/g - 1 */
+      const double* wi = WG + (size_t)i * Kg * d_g;
+      double* yi = y + (size_t)i * d_g;
+      for (int j = 0; j < d_g; ++j) yi[j] = 0.0;
+      for (int k = 0; k < Kg; ++k) {
+        const double a = oi[k];
+        const double* w = wi + (size_t)k * d_g;
+        for (int j = 0; j < d_g; ++j) yi[j] += a * w[j];
+      }
+    }
+    if (round_mid) ocsa_round_bf16(g * d_g, y, y);
+    double* r = out + (size_t)q * d;
+    for (int j = 0; j < d; ++j) r[j] = 0.0;
+    for (int k = 0; k < g * d_g; ++k) {
+      const double a = y[k];
+      const double* w = WO + (size_t)k * d;
+      for (int j = 0; j < d; ++j) r[j] += a * w[j];
+    }
+  }
+}

@@ -119,6 +119,14 @@ void ocsa_fp8mix_decode(int n, int c, int rope_dims, const uint8_t* codes,
                         const uint16_t* rope_bf16_bits, const float* scale,
                         double* x);
 
+/* Grouped output projection ([N] 2.3.3, [P] 2.2): group i of n_h / g
+ * consecutive heads of O [Q][n_h][c] times WG[i] [c n_h/g][d_g] gives
+ * Y[q][i d_g .. (i+1) d_g); out [Q][d] = Y WO with WO [g d_g][d].  With
+ * round_mid, Y is rounded to bf16 before WO. */
+void ocsa_group_out_proj(int Q, int n_h, int c, int g, int d_g, int d, const double* O,
+                         const double* WG, const double* WO, int round_mid, double* Y,
+                         double* out);
+
 #ifdef __cplusplus
 }
 #endif

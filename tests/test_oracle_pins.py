@@ -468,3 +468,70 @@ def test_e2e_rope_shift_invariance(variant):
         out, _ = P.attend_wl(wl, t0s, q, idx, kv, win, 0, inp["sink"], rope_shift=shift)
         outs.append(out)
     np.testing.assert_allclose(outs[0], outs[1], atol=1e-9)
+
+
+# ------------------------------------------------ grouped output projection ---
+# "DeepSeekV4技术报告阅读笔记" 2.3.3 (Grouped Output Projection); PaperTrace 2.2.
+
+def _gop_inputs(Q=3, n_h=8, c=6, g=4, d_g=5, d=7, seed=41):
+    r = rng(seed)
+    O = r.standard_normal((Q, n_h, c))
+    WG = r.standard_normal((g, c * n_h // g, d_g))
+    WO = r.standard_normal((g * d_g, d))
+    return O, WG, WO
+
+
+def test_group_out_proj_one_group_is_two_matmuls():
+    O, WG, WO = _gop_inputs(g=1)
+    Y, out = oracle.group_out_proj(O, WG, WO, round_mid=False)
+    flat = O.reshape(O.shape[0], -1)
+    np.testing.assert_allclose(Y, flat @ WG[0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(out, (flat @ WG[0]) @ WO, rtol=1e-12, atol=1e-12)
+
+
+def test_group_out_proj_is_a_block_diagonal_projection():
+    """The notes' one-line summary: R^{c n_h} -> R^{d_g g} by a block-diagonal
+    matrix (one block per group of consecutive heads), then -> R^d."""
+    import scipy.linalg
+    O, WG, WO = _gop_inputs()
+    Y, out = oracle.group_out_proj(O, WG, WO, round_mid=False)
+    W_eff = scipy.linalg.block_diag(*WG) @ WO
+    flat = O.reshape(O.shape[0], -1)
+    np.testing.assert_allclose(Y, flat @ scipy.linalg.block_diag(*WG), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(out, flat @ W_eff, rtol=1e-10, atol=1e-10)
+
+
+def test_group_out_proj_groups_are_independent():
+    O, WG, WO = _gop_inputs()
+    g, d_g = WG.shape[0], WG.shape[2]
+    hpg = O.shape[1] // g
+    Y0, _ = oracle.group_out_proj(O, WG, WO, round_mid=False)
+    O2 = O.copy()
+    O2[:, 2 * hpg:3 * hpg] += 1.0  # the heads of group 2 only
+    Y1, _ = oracle.group_out_proj(O2, WG, WO, round_mid=False)
+    changed = np.any(Y0 != Y1, axis=0).reshape(g, d_g).any(axis=1)
+    assert changed.tolist() == [False, False, True, False]
+
+
+def test_group_out_proj_rounds_the_group_outputs():
+    O, WG, WO = _gop_inputs()
+    Yx, _ = oracle.group_out_proj(O, WG, WO, round_mid=False)
+    Y, out = oracle.group_out_proj(O, WG, WO, round_mid=True)
+    np.testing.assert_array_equal(Y, torch.from_numpy(Yx).to(torch.bfloat16).double().numpy())
+    np.testing.assert_allclose(out, Y @ WO, rtol=1e-12, atol=1e-12)
+
+
+def test_group_out_proj_parameter_counts_of_the_pages():
+    """PaperTrace 2.2: with V4-Pro's shapes (c = 512, n_h = 128, g = 16,
+    d_g = 1024, d = 7168) the grouped projection has about 180 million
+    parameters and a direct one about 470 million; the notes 2.3.3 count
+    c n_h d_g + d_g g d multiplications.  The oracle accepts exactly these
+    operand shapes."""
+    c, n_h, g, d_g, d = 512, 128, 16, 1024, 7168
+    grouped = g * (c * n_h // g) * d_g + (g * d_g) * d
+    assert grouped == c * n_h * d_g + d_g * g * d
+    assert abs(grouped / 1.8e8 - 1) < 0.03
+    assert abs(c * n_h * d / 4.7e8 - 1) < 0.01
+    O = np.zeros((1, 4, 2))
+    with pytest.raises(ValueError):
+        oracle.group_out_proj(O, np.zeros((2, 3, 5)), np.zeros((10, 3)))  # c n_h / g = 4
