@@ -251,6 +251,45 @@ class DecodeStep:
         del g, gp, packs
         return ms, wbytes, split
 
+    def time_out_proj(self, steps, stream):
+        """Device time of csa_out_proj on the step's attention output (the
+        grouped output projection of the workload's g and d_g; graph replays,
+        4 calls per graph; the weights, larger than twice the L2, stream from
+        HBM every call).  Returns (ms per call, packed weight bytes)."""
+        wl, dev = self.wl, self.out.device
+        g, d_g, d = wl.g_out, wl.d_g, wl.d
+        Kg = wl.c * wl.n_h // g
+        gen = torch.Generator(device=dev).manual_seed(wl.seed + 11)
+        WG = (torch.randn(g, Kg, d_g, device=dev, generator=gen) / Kg ** 0.5).to(torch.bfloat16)
+        WO = (torch.randn(g * d_g, d, device=dev, generator=gen) / (g * d_g) ** 0.5).to(
+            torch.bfloat16)
+        packed = bd.out_proj_pack(WG, WO)
+        del WG, WO
+        O = self.out.view(self.out.shape[0], wl.n_h, wl.c)
+        res = torch.empty(O.shape[0], d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(bd.out_proj_workspace_bytes(O.shape[0], wl.n_h, wl.c, g, d_g, d),
+                         dtype=torch.uint8, device=dev)
+        per_graph = 4
+        for _ in range(2):
+            bd.csa_out_proj(O, packed, g, d_g, res, workspace=ws)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for _ in range(per_graph):
+                bd.csa_out_proj(O, packed, g, d_g, res, workspace=ws)
+        gr.replay()
+        reps = max(1, steps // per_graph)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            gr.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert bd.device_status() == 0, "device error word set by the output projection"
+        nbytes = packed.numel()
+        del gr, packed
+        return e0.elapsed_time(e1) / (reps * per_graph), nbytes
+
     def dominant(self):
         """(kernel kind, algorithmic bytes per launch, source file)."""
         wl, B, N = self.wl, self.wl.B, self.N
@@ -561,6 +600,15 @@ def run_ours(args, world, rank, local):
                   "weight_bytes": a_bytes, "hbm_frac": round(a_bytes / (a_ms / 1e3) / 1e9 / hbm0, 4),
                   "kernels_ms": a_split}
 
+    out_proj = None
+    if wl.mode == "decode" and wl.act == "bf16":
+        # the grouped output projection after the step (timed on its own)
+        o_ms, o_bytes = step.time_out_proj(min(args.steps, 200), stream)
+        hbm0, _, _ = _peaks()
+        out_proj = {"ms_per_call": round(o_ms, 5), "tokens": wl.B, "g": wl.g_out, "d_g": wl.d_g,
+                    "weight_bytes": o_bytes,
+                    "hbm_frac": round(o_bytes / (o_ms / 1e3) / 1e9 / hbm0, 4)}
+
     kind, nbytes, src, bound = step.dominant()
     kms, kcnt = prof.get(kind, (0.0, 0))  # one replay: kcnt launches of the kernel
     hbm, tfl, peak_src = _peaks()
@@ -624,6 +672,7 @@ def run_ours(args, world, rank, local):
             "roofline": roof,
             "kernels": kernels,
             "decode_append": append,
+            "out_proj": out_proj,
             "cpu_baseline": cpu,
             "clocks": clk,
         }

@@ -183,6 +183,30 @@ csa_status hca_decode_append(const csa_params* p, int B, int d, const void* H,
                              int W, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_out_proj: the grouped output projection that follows the attention
+ * ([N] 2.3.3 "Grouped Output Projection"; [P] 2.2).  The n_h head outputs
+ * of a token (csa_attend's out row, [n_h][c]) are cut into g groups of n_h/g
+ * consecutive heads; group i (c n_h/g values) times W^G_i gives d_g values
+ * (stored as bf16: Y); the g d_g values times W^O give the d outputs.
+ * bf16 only; 16 tokens per pair of tensor-core launches (weights streamed
+ * once per 16 tokens: the decode form).
+ *   WG  [g][c n_h/g][d_g] bf16, WO [g d_g][d] bf16 (row-major, x W form)
+ *   packed  csa_out_proj_packed_bytes(...) bytes from csa_out_proj_pack
+ *           (W^G and W^O transposed to K-major rows)
+ *   O   [R][n_h][c] bf16    out [R][d] bf16
+ *   workspace  csa_out_proj_workspace_bytes(...) bytes (Y, [R][g d_g] bf16)
+ * Shapes: n_h % g == 0, (c n_h / g) % 64 == 0, d_g % 128 == 0; otherwise
+ * CSA_ERR_SHAPE (and 0 from the size queries).  Pointers 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+size_t csa_out_proj_packed_bytes(int n_h, int c, int g, int d_g, int d);
+csa_status csa_out_proj_pack(int n_h, int c, int g, int d_g, int d, const void* WG,
+                             const void* WO, void* packed, csa_stream_t stream);
+size_t csa_out_proj_workspace_bytes(int R, int n_h, int c, int g, int d_g, int d);
+csa_status csa_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void* O,
+                        const void* packed, void* out, void* workspace, size_t ws_bytes,
+                        csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * csa_index_topk: Lightning-Indexer scores and top-k selection ([N] eq. 16-17,
  * [P] 2.2):  I[r][s] = sum_h w[r][h] * ReLU(qI[r][h] . kI[b][s])  for every
  * visible s, then the topk largest.  Ties are broken towards the lower index.

@@ -65,6 +65,10 @@ _SIGS = {
                                     _vp, _vp, _i, _vp]),
     "hca_decode_append": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp,
                                     _vp, _i, _vp]),
+    "csa_out_proj_packed_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "csa_out_proj_pack": (C.c_int, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "csa_out_proj_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "csa_out_proj": (C.c_int, [_i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_noalloc": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
@@ -217,6 +221,36 @@ def hca_decode_append(p: CsaParams, H, t, packed, tail, ckv, ckv_scale, win, win
                                  _p(ckv_scale), N, _p(win), _p(win_scale), _p(win_pos0), W,
                                  _stream(stream))
     _check("hca_decode_append", st)
+
+
+# ------------------------------------------- grouped output projection --
+def out_proj_pack(WG, WO, stream=None) -> torch.Tensor:
+    """WG [g][c n_h/g][d_g], WO [g d_g][d] (bf16, device) -> the packed
+    buffer for csa_out_proj.  n_h and c enter only through c n_h / g, so the
+    packing takes n_h = g, c = c n_h / g."""
+    g, Kg, d_g = WG.shape
+    d = WO.shape[1]
+    nbytes = lib().csa_out_proj_packed_bytes(g, Kg, g, d_g, d)
+    if nbytes == 0:
+        raise CsaError("csa_out_proj_packed_bytes", 2, "unsupported shapes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=WG.device)
+    st = lib().csa_out_proj_pack(g, Kg, g, d_g, d, _p(WG), _p(WO), _p(packed), _stream(stream))
+    _check("csa_out_proj_pack", st)
+    return packed
+
+
+def out_proj_workspace_bytes(R, n_h, c, g, d_g, d) -> int:
+    return lib().csa_out_proj_workspace_bytes(R, n_h, c, g, d_g, d)
+
+
+def csa_out_proj(O, packed, g, d_g, out, workspace=None, stream=None):
+    """O [R][n_h][c] bf16 -> out [R][d] bf16 (grouped output projection)."""
+    R, n_h, c = O.shape
+    d = out.shape[1]
+    ws, wsb = _ws(out_proj_workspace_bytes(R, n_h, c, g, d_g, d), O.device, workspace)
+    st = lib().csa_out_proj(R, n_h, c, g, d_g, d, _p(O), _p(packed), _p(out), _p(ws), wsb,
+                            _stream(stream))
+    _check("csa_out_proj", st)
 
 
 # --------------------------------------------------------- index / top-k --

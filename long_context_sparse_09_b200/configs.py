@@ -5,7 +5,8 @@ entry dim c=512 with RoPE on the last 64 dims, m=4, a 64-head x 128-dim
 indexer, top-k 512, window 128) and V4-Pro (d=7168, 128 heads, top-k 1024,
 448 FP8 dims + 64 BF16 RoPE dims per entry); HCA groups m'=128 tokens
 ("02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文", sections 2.1-2.5; "DeepSeekV4
-技术报告阅读笔记", section 2.3-2.5).  This module holds sizes only, no arithmetic
+技术报告阅读笔记", section 2.3-2.5); the grouped output projection has g = 8
+(Flash) or 16 (Pro) groups of width d_g = 1024 (PaperTrace 2.2).  This module holds sizes only, no arithmetic
 of the method.
 """
 from __future__ import annotations
@@ -35,6 +36,8 @@ class Workload:
     seed: int
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
+    g_out: int = 8     # output-projection groups (V4-Flash 8, V4-Pro 16)
+    d_g: int = 1024    # width of each group's projection
 
     @property
     def overlap(self) -> int:
@@ -69,7 +72,7 @@ WORKLOADS = {
     "pro_csa_decode_1m": Workload(
         "pro_csa_decode_1m", "decode", "csa", B=4, T=1048576, d=7168,
         n_h=128, c=512, rope_dims=64, m=4, n_hI=64, c_I=128, d_c=1536,
-        topk=1024, n_win=128, act="bf16", kv="fp8mix", seed=3),
+        topk=1024, n_win=128, act="bf16", kv="fp8mix", seed=3, g_out=16),
     "hca_decode_1m": Workload(
         "hca_decode_1m", "decode", "hca", B=16, T=1048576, d=4096, n_h=64,
         c=512, rope_dims=64, m=128, n_hI=0, c_I=0, d_c=1024, topk=0,

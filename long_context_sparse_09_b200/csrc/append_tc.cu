@@ -1,7 +1,8 @@
-// append_tc.cu -- the decode-time compressor's projection on the 5th-
-// generation tensor cores ("DeepSeekV4技术报告阅读笔记" eq. 9-12 and 20-23 for
-// one new token per sequence; the running-softmax state of the open entries
-// is the one csa_decode_append keeps, see compress.cu).
+// append_tc.cu -- projections of a few tokens on the 5th-generation tensor
+// cores: the decode-time compressor's ("DeepSeekV4技术报告阅读笔记" eq. 9-12
+// and 20-23 for one new token per sequence; the running-softmax state of the
+// open entries is the one csa_decode_append keeps, see compress.cu) and the
+// grouped output projection (same notes 2.3.3; PaperTrace 2.2).
 //
 // D[128][16] = Wtile[128][d] . H[16][d]^T: the M side is one block of 64
 // channels of one part (a or b window, main or indexer) as its 64 C rows and
@@ -11,8 +12,10 @@
 // thread issues the MMAs into a 16-column fp32 TMEM accumulator, and the
 // epilogue stages it in shared memory.  The slices are summed in a fixed
 // order through distributed shared memory, and each CTA of the cluster folds
-// its share of the (channel, token) pairs into the state.  Every wait is
-// bounded.
+// its share of the (channel, token) pairs into the state.  The output
+// projection uses the same body with 128 consecutive output features as M
+// and a plain bf16 store of its share of the (feature, token) pairs.  Every
+// wait is bounded.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -40,11 +43,17 @@ struct ApArgs {
   unsigned* err;
   size_t per_seq;
   int nb, KB, kbs, nsplit, m, overlap, c, cI;
+  // plain-store form: out[b * ld_out + f] for features f < nfeat; the tile
+  // of features f0.. reads the tokens' columns from (f0 / rows_per_group) *
+  // x_per_group on
+  __nv_bfloat16* out;
+  int ld_out, nfeat, rows_per_group, x_per_group;
 };
 
-__global__ void __launch_bounds__(kApThreads, 1)
-    append_project_tc(const __grid_constant__ CUtensorMap tmW,
-                      const __grid_constant__ CUtensorMap tmH, ApArgs a) {
+// kMode 0: the compressor projection and state update; 1: a plain store.
+template <int kMode>
+__device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtensorMap* tmH,
+                                            const ApArgs& a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* dtile = (float*)(sm + kApStages * kApStage);  // [128 rows][16 tokens]
@@ -59,27 +68,41 @@ __global__ void __launch_bounds__(kApThreads, 1)
   const int split = (int)cluster_ctarank();
   const int tile = blockIdx.x / a.nsplit;
 
-  // tile -> part (0 a main, 1 b main, 2 a indexer, 3 b indexer) and block
-  const int nbc = (a.c + 63) / 64, nbi = (a.cI + 63) / 64;
-  int part, blk;
-  if (tile < nbc) {
-    part = 0; blk = tile;
-  } else if (tile < 2 * nbc) {
-    part = 1; blk = tile - nbc;
-  } else if (tile < 2 * nbc + nbi) {
-    part = 2; blk = tile - 2 * nbc;
-  } else {
-    part = 3; blk = tile - 2 * nbc - nbi;
-  }
+  // tile -> the two 64-row boxes of weights, the tokens' column offset and,
+  // for the compressor, part (0 a main, 1 b main, 2 a indexer, 3 b indexer)
+  int rowA0, rowB0, xoff = 0;
+  int part = 0, colB0 = 0, nvalid = 128, sch0 = 0, ch0 = 0;
+  bool partb = false;
   const PackLayout& L = a.L;
-  const int colC0 = part == 0 ? L.col_Ca : part == 1 ? L.col_Cb : part == 2 ? L.col_CIa : L.col_CIb;
-  const int colZ0 = part == 0 ? L.col_Za : part == 1 ? L.col_Zb : part == 2 ? L.col_ZIa : L.col_ZIb;
-  const int colB0 = part == 0 ? L.b_Ba : part == 1 ? L.b_Bb : part == 2 ? L.b_BIa : L.b_BIb;
-  const int nchan = part < 2 ? a.c : a.cI;
-  const int sch0 = part < 2 ? 0 : a.c;  // state channel of the part's channel 0
-  const bool partb = part == 1 || part == 3;
-  const int ch0 = blk * 64;
-  const int nvalid = nchan - ch0 < 64 ? nchan - ch0 : 64;
+  if constexpr (kMode == 0) {
+    const int nbc = (a.c + 63) / 64, nbi = (a.cI + 63) / 64;
+    int blk;
+    if (tile < nbc) {
+      part = 0; blk = tile;
+    } else if (tile < 2 * nbc) {
+      part = 1; blk = tile - nbc;
+    } else if (tile < 2 * nbc + nbi) {
+      part = 2; blk = tile - 2 * nbc;
+    } else {
+      part = 3; blk = tile - 2 * nbc - nbi;
+    }
+    const int colC0 = part == 0 ? L.col_Ca : part == 1 ? L.col_Cb : part == 2 ? L.col_CIa : L.col_CIb;
+    const int colZ0 = part == 0 ? L.col_Za : part == 1 ? L.col_Zb : part == 2 ? L.col_ZIa : L.col_ZIb;
+    colB0 = part == 0 ? L.b_Ba : part == 1 ? L.b_Bb : part == 2 ? L.b_BIa : L.b_BIb;
+    const int nchan = part < 2 ? a.c : a.cI;
+    sch0 = part < 2 ? 0 : a.c;  // state channel of the part's channel 0
+    partb = part == 1 || part == 3;
+    ch0 = blk * 64;
+    nvalid = nchan - ch0 < 64 ? nchan - ch0 : 64;
+    rowA0 = colC0 + ch0;
+    rowB0 = colZ0 + ch0;
+  } else {
+    const int f0 = tile * 128;
+    rowA0 = f0;
+    rowB0 = f0 + 64;
+    xoff = (f0 / a.rows_per_group) * a.x_per_group;
+    nvalid = a.nfeat - f0 < 128 ? a.nfeat - f0 : 128;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kApStages; ++i) {
@@ -95,8 +118,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
-    prefetch_tmap(&tmW);
-    prefetch_tmap(&tmH);
+    prefetch_tmap(tmW);
+    prefetch_tmap(tmH);
   }
   tc_fence_before();
   __syncthreads();
@@ -116,9 +139,9 @@ __global__ void __launch_bounds__(kApThreads, 1)
       if (!mbar_wait(&empty[s], ((i / kApStages) & 1) ^ 1, abort_sm)) break;
       uint8_t* st = sm + s * kApStage;
       mbar_expect_tx(&full[s], kApStage);
-      tma_load_2d_hint(st, &tmW, &full[s], kb * 64, colC0 + ch0, pol);
-      tma_load_2d_hint(st + kApA / 2, &tmW, &full[s], kb * 64, colZ0 + ch0, pol);
-      tma_load_2d(st + kApA, &tmH, &full[s], kb * 64, 0);
+      tma_load_2d_hint(st, tmW, &full[s], kb * 64, rowA0, pol);
+      tma_load_2d_hint(st + kApA / 2, tmW, &full[s], kb * 64, rowB0, pol);
+      tma_load_2d(st + kApA, tmH, &full[s], xoff + kb * 64, 0);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------- MMA --
@@ -156,7 +179,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
   // --------------------------- sum of the slices and the state update --
   // CTA `split` takes channels [c_lo, c_hi) of the block, all tokens
-  if (!*abort_sm) {
+  if (kMode == 0 && !*abort_sm) {
     const int per = (64 + a.nsplit - 1) / a.nsplit;
     const int c_lo = split * per;
     const int c_hi = c_lo + per < nvalid ? c_lo + per : nvalid;
@@ -196,6 +219,28 @@ __global__ void __launch_bounds__(kApThreads, 1)
                           Z + a.bias[rr * L.nb + colB0 + gch], fresh);
     }
   }
+  // ------------------------------ sum of the slices and the plain store --
+  // CTA `split` takes rows [r_lo, r_hi) of the tile, all tokens
+  if (kMode == 1 && !*abort_sm) {
+    const int per = (128 + a.nsplit - 1) / a.nsplit;
+    const int r_lo = split * per;
+    const int r_hi = r_lo + per < nvalid ? r_lo + per : nvalid;
+    const int nitems = r_hi > r_lo ? (r_hi - r_lo) * a.nb : 0;
+    const uint32_t dbase = smem_u32(dtile);
+    for (int it = threadIdx.x; it < nitems; it += kApThreads) {
+      const int row = r_lo + it / a.nb, b = it % a.nb;
+      float vs[kApMaxSplit];
+#pragma unroll
+      for (int r = 0; r < kApMaxSplit; ++r)
+        vs[r] = r < a.nsplit
+                    ? ld_dsmem_f32(mapa_shared(dbase, (uint32_t)r) + (uint32_t)((row * kApN + b) * 4))
+                    : 0.f;
+      float v = 0.f;
+#pragma unroll
+      for (int r = 0; r < kApMaxSplit; ++r) v += vs[r];
+      a.out[(size_t)b * a.ld_out + tile * 128 + row] = __float2bfloat16_rn(v);
+    }
+  }
   cluster_sync_all();  // no CTA leaves while its tile may still be read
   if (*abort_sm) {
     if (threadIdx.x == 0) atomicOr(a.err, CSA_DEV_TIMEOUT);
@@ -203,6 +248,18 @@ __global__ void __launch_bounds__(kApThreads, 1)
     while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
   }
   if (warp == 1) tmem_dealloc(tbase, 32);
+}
+
+__global__ void __launch_bounds__(kApThreads, 1)
+    append_project_tc(const __grid_constant__ CUtensorMap tmW,
+                      const __grid_constant__ CUtensorMap tmH, ApArgs a) {
+  skinny_body<0>(&tmW, &tmH, a);
+}
+
+__global__ void __launch_bounds__(kApThreads, 1)
+    out_proj_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                ApArgs a) {
+  skinny_body<1>(&tmW, &tmX, a);
 }
 
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
@@ -213,13 +270,14 @@ bool append_tc_supported(const csa_params& p, int nb) {
   return p.act == CSA_BF16 && nb >= 1 && nb <= kApN && tma_available();
 }
 
-static int ap_max_active_clusters(int csize) {
-  static int cache[64][kApMaxSplit + 1];
-  static bool have[64][kApMaxSplit + 1];
+// kern 0: append_project_tc, 1: out_proj_tc (same resources)
+static int ap_max_active_clusters(int csize, int kern = 0) {
+  static int cache[64][2][kApMaxSplit + 1];
+  static bool have[64][2][kApMaxSplit + 1];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || csize < 1 || csize > kApMaxSplit) return 0;
-  if (!have[dev][csize]) {
+  if (!have[dev][kern][csize]) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(csize * 148);
     cfg.blockDim = dim3(kApThreads);
@@ -232,14 +290,49 @@ static int ap_max_active_clusters(int csize) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, append_project_tc, &cfg) != cudaSuccess) {
+    const cudaError_t e = kern == 0 ? cudaOccupancyMaxActiveClusters(&n, append_project_tc, &cfg)
+                                    : cudaOccupancyMaxActiveClusters(&n, out_proj_tc, &cfg);
+    if (e != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
-    cache[dev][csize] = n;
-    have[dev][csize] = true;
+    cache[dev][kern][csize] = n;
+    have[dev][kern][csize] = true;
   }
-  return cache[dev][csize];
+  return cache[dev][kern][csize];
+}
+
+// slices of d for `tiles` output tiles and KB k-blocks: at most one CTA per
+// SM, at most a cluster of 8, no empty slice; sets a.kbs and a.nsplit
+static void plan_slices(ApArgs& a, int tiles, int kern) {
+  const int sms = sm_count();
+  int ns = sms / tiles;
+  if (ns > kApMaxSplit) ns = kApMaxSplit;
+  if (ns > a.KB) ns = a.KB;
+  if (ns < 1) ns = 1;
+  while (ns > 1 && ap_max_active_clusters(ns, kern) < 1) --ns;
+  a.kbs = (a.KB + ns - 1) / ns;
+  a.nsplit = (a.KB + a.kbs - 1) / a.kbs;
+}
+
+template <typename Kern>
+static csa_status launch_skinny(Kern kern, int tiles, const CUtensorMap& tmW,
+                                const CUtensorMap& tmX, const ApArgs& a, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tiles * a.nsplit);
+  cfg.blockDim = dim3(kApThreads);
+  cfg.dynamicSmemBytes = (size_t)kApSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = (unsigned)a.nsplit;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = kPdlAppend ? 1 : 0;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, a) == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
 csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, int nb, int d,
@@ -266,16 +359,8 @@ csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, in
   const int nbc = (p.c + 63) / 64, nbi = (a.cI + 63) / 64;
   const int tiles = p.overlap ? 2 * nbc + 2 * nbi : nbc;
   a.KB = (d + 63) / 64;
-  // slices of d: at most one CTA per SM (a second CTA on a few SMs would
-  // make them the last to finish), at most a cluster of 8, no empty slice
-  const int sms = sm_count();
-  int ns = sms / tiles;
-  if (ns > kApMaxSplit) ns = kApMaxSplit;
-  if (ns > a.KB) ns = a.KB;
-  if (ns < 1) ns = 1;
-  while (ns > 1 && ap_max_active_clusters(ns) < 1) --ns;
-  a.kbs = (a.KB + ns - 1) / ns;
-  a.nsplit = (a.KB + a.kbs - 1) / a.kbs;
+  // (a second CTA on a few SMs would make them the last to finish)
+  plan_slices(a, tiles, 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * a.nsplit);
   cfg.blockDim = dim3(kApThreads);
@@ -292,6 +377,110 @@ csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, in
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
   CSA_LAUNCH(KK_GEMM, st, cudaLaunchKernelEx(&cfg, append_project_tc, tmW, tmH, a));
+  return last_launch_status();
+}
+
+// ------------------------------------------- grouped output projection --
+// Packed weights: W^G transposed to K-major rows ([g d_g][c n_h / g]: row
+// i d_g + j is column j of W^G_i), then, 256-byte aligned, W^O transposed
+// ([d][g d_g]).
+
+static size_t op_wo_offset(int n_h, int c, int g, int d_g) {
+  return align_up((size_t)g * d_g * (size_t)(c * (n_h / g)) * 2, 256);
+}
+
+size_t out_proj_packed_bytes(int n_h, int c, int g, int d_g, int d) {
+  return op_wo_offset(n_h, c, g, d_g) + align_up((size_t)d * g * d_g * 2, 256);
+}
+
+size_t out_proj_ws_bytes(int R, int g, int d_g) {
+  return align_up((size_t)R * g * d_g * 2, 256);
+}
+
+// dst[(row0 + j) * K + k] = src[k * width + j] for k < K, j < width (a
+// 32 x 32-tiled transpose of one row-major [K][width] matrix)
+__global__ void transpose_bf16(const __nv_bfloat16* __restrict__ src, int K, int width,
+                               __nv_bfloat16* __restrict__ dst, size_t row0) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int k0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int k = k0 + r, j = j0 + threadIdx.x;
+    if (k < K && j < width) tile[r][threadIdx.x] = src[(size_t)k * width + j];
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int j = j0 + r, k = k0 + threadIdx.x;
+    if (k < K && j < width) dst[(row0 + j) * (size_t)K + k] = tile[threadIdx.x][r];
+  }
+}
+
+csa_status launch_out_proj_pack(int n_h, int c, int g, int d_g, int d, const void* WG,
+                                const void* WO, void* packed, cudaStream_t st) {
+  const int Kg = c * (n_h / g);
+  __nv_bfloat16* dst = (__nv_bfloat16*)packed;
+  const __nv_bfloat16* wg = (const __nv_bfloat16*)WG;
+  for (int i = 0; i < g; ++i) {
+    const dim3 grid((d_g + 31) / 32, (Kg + 31) / 32);
+    CSA_LAUNCH(KK_GEMM, st, transpose_bf16<<<grid, dim3(32, 8), 0, st>>>(
+        wg + (size_t)i * Kg * d_g, Kg, d_g, dst, (size_t)i * d_g));
+  }
+  __nv_bfloat16* wo = (__nv_bfloat16*)((char*)packed + op_wo_offset(n_h, c, g, d_g));
+  const dim3 grid((d + 31) / 32, (g * d_g + 31) / 32);
+  CSA_LAUNCH(KK_GEMM, st, transpose_bf16<<<grid, dim3(32, 8), 0, st>>>(
+      (const __nv_bfloat16*)WO, g * d_g, d, wo, 0));
+  return last_launch_status();
+}
+
+// Y = group products of O (bf16), out = Y W^O, 16 tokens a pair of launches
+csa_status launch_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void* O,
+                           const void* packed, void* out, void* ws, cudaStream_t st) {
+  if (!tma_available()) return CSA_ERR_UNSUPPORTED;
+  if (!set_kernel_smem((const void*)out_proj_tc, kApSmem)) return CSA_ERR_CUDA;
+  unsigned* err = device_error_word();
+  if (err == nullptr) return CSA_ERR_CUDA;
+  const int Kg = c * (n_h / g), GD = g * d_g;
+  const __nv_bfloat16* o = (const __nv_bfloat16*)O;
+  const __nv_bfloat16* wg = (const __nv_bfloat16*)packed;
+  const __nv_bfloat16* wo =
+      (const __nv_bfloat16*)((const char*)packed + op_wo_offset(n_h, c, g, d_g));
+  __nv_bfloat16* y = (__nv_bfloat16*)ws;
+  __nv_bfloat16* res = (__nv_bfloat16*)out;
+  for (int b0 = 0; b0 < R; b0 += kApN) {
+    const int nb = R - b0 < kApN ? R - b0 : kApN;
+    ApArgs a = {};
+    a.err = err;
+    a.nb = nb;
+    // group products: features i d_g + j read the tokens' columns i Kg..
+    CUtensorMap tmW, tmX;
+    if (!make_tmap_bf16(&tmW, wg, (uint64_t)GD, (uint64_t)Kg, 64)) return CSA_ERR_CUDA;
+    if (!make_tmap_bf16(&tmX, o + (size_t)b0 * n_h * c, (uint64_t)nb, (uint64_t)n_h * c, kApN))
+      return CSA_ERR_CUDA;
+    a.out = y + (size_t)b0 * GD;
+    a.ld_out = GD;
+    a.nfeat = GD;
+    a.rows_per_group = d_g;
+    a.x_per_group = Kg;
+    a.KB = Kg / 64;
+    const int tiles1 = GD / 128;
+    plan_slices(a, tiles1, 1);
+    csa_status s;
+    CSA_LAUNCH(KK_GEMM, st, s = launch_skinny(out_proj_tc, tiles1, tmW, tmX, a, st));
+    if (s != CSA_OK) return s;
+    // the output projection of the (bf16) group outputs
+    if (!make_tmap_bf16(&tmW, wo, (uint64_t)d, (uint64_t)GD, 64)) return CSA_ERR_CUDA;
+    if (!make_tmap_bf16(&tmX, y + (size_t)b0 * GD, (uint64_t)nb, (uint64_t)GD, kApN))
+      return CSA_ERR_CUDA;
+    a.out = res + (size_t)b0 * d;
+    a.ld_out = d;
+    a.nfeat = d;
+    a.rows_per_group = 1 << 30;  // one group
+    a.x_per_group = 0;
+    a.KB = (GD + 63) / 64;
+    const int tiles2 = (d + 127) / 128;
+    plan_slices(a, tiles2, 1);
+    CSA_LAUNCH(KK_GEMM, st, s = launch_skinny(out_proj_tc, tiles2, tmW, tmX, a, st));
+    if (s != CSA_OK) return s;
+  }
   return last_launch_status();
 }
 

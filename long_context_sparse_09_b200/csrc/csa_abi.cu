@@ -244,6 +244,46 @@ csa_status csa_pack_weights(const csa_params* p, int d, const void* Wkv_a,
   return launch_pack(*p, d, W, Bs, packed, S(stream));
 }
 
+// ------------------------------------------- grouped output projection --
+static csa_status check_out_proj(int n_h, int c, int g, int d_g, int d) {
+  if (n_h <= 0 || c <= 0 || g <= 0 || d_g <= 0 || d <= 0) return CSA_ERR_SHAPE;
+  if (n_h % g != 0) return CSA_ERR_SHAPE;
+  if ((c * (n_h / g)) % 64 != 0 || d_g % 128 != 0) return CSA_ERR_SHAPE;
+  return CSA_OK;
+}
+
+size_t csa_out_proj_packed_bytes(int n_h, int c, int g, int d_g, int d) {
+  if (check_out_proj(n_h, c, g, d_g, d) != CSA_OK) return 0;
+  return out_proj_packed_bytes(n_h, c, g, d_g, d);
+}
+
+csa_status csa_out_proj_pack(int n_h, int c, int g, int d_g, int d, const void* WG,
+                             const void* WO, void* packed, csa_stream_t stream) {
+  csa_status st = check_out_proj(n_h, c, g, d_g, d);
+  if (st != CSA_OK) return st;
+  if (!WG || !WO || !packed) return CSA_ERR_ARG;
+  if (!aligned16(packed)) return CSA_ERR_ALIGN;
+  return launch_out_proj_pack(n_h, c, g, d_g, d, WG, WO, packed, S(stream));
+}
+
+size_t csa_out_proj_workspace_bytes(int R, int n_h, int c, int g, int d_g, int d) {
+  if (R <= 0 || check_out_proj(n_h, c, g, d_g, d) != CSA_OK) return 0;
+  return out_proj_ws_bytes(R, g, d_g);
+}
+
+csa_status csa_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void* O,
+                        const void* packed, void* out, void* workspace, size_t ws_bytes,
+                        csa_stream_t stream) {
+  csa_status st = check_out_proj(n_h, c, g, d_g, d);
+  if (st != CSA_OK) return st;
+  if (R <= 0) return CSA_ERR_SHAPE;
+  if (!O || !packed || !out) return CSA_ERR_ARG;
+  if (!aligned16(O) || !aligned16(packed) || !aligned16(out)) return CSA_ERR_ALIGN;
+  if (workspace == nullptr || ws_bytes < out_proj_ws_bytes(R, g, d_g)) return CSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return CSA_ERR_ALIGN;
+  return launch_out_proj(R, n_h, c, g, d_g, d, O, packed, out, workspace, S(stream));
+}
+
 // -------------------------------------------------------------- compress --
 size_t csa_compress_workspace_bytes(const csa_params* p, int B, int T, int d) {
   if (check_params(p, p && p->overlap == 1) != CSA_OK || B <= 0 || T <= 0 || d <= 0) return 0;

@@ -32,6 +32,13 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
                            float* win_scale, void* ws, cudaStream_t st);
 
 size_t decode_tail_bytes(const csa_params& p, int B, int d);
+// grouped output projection (bf16; tensor cores, 16 tokens a pair of launches)
+size_t out_proj_packed_bytes(int n_h, int c, int g, int d_g, int d);
+size_t out_proj_ws_bytes(int R, int g, int d_g);
+csa_status launch_out_proj_pack(int n_h, int c, int g, int d_g, int d, const void* WG,
+                                const void* WO, void* packed, cudaStream_t st);
+csa_status launch_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void* O,
+                           const void* packed, void* out, void* ws, cudaStream_t st);
 // decode append, tensor-core projection (bf16, at most 16 tokens a launch)
 bool append_tc_supported(const csa_params& p, int nb);
 csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, int nb, int d,

@@ -129,6 +129,28 @@ def test_decode_append_argument_errors(lib):
     assert st == 1
 
 
+def test_out_proj_sizes_and_argument_errors(lib):
+    # V4-Pro: c = 512, n_h = 128, g = 16, d_g = 1024, d = 7168
+    assert lib.csa_out_proj_packed_bytes(128, 512, 16, 1024, 7168) == \
+        16 * 1024 * 4096 * 2 + 7168 * 16384 * 2
+    assert lib.csa_out_proj_workspace_bytes(4, 128, 512, 16, 1024, 7168) == 4 * 16384 * 2
+    # unsupported shapes: heads not divisible into groups, c n_h / g not a
+    # multiple of 64, d_g not a multiple of 128
+    assert lib.csa_out_proj_packed_bytes(128, 512, 12, 1024, 7168) == 0
+    assert lib.csa_out_proj_packed_bytes(8, 4, 2, 128, 64) == 0
+    assert lib.csa_out_proj_packed_bytes(8, 64, 2, 100, 64) == 0
+    fake = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    ws = 1 << 30
+    assert lib.csa_out_proj(4, 128, 512, 12, 1024, 7168, fake, fake, fake, fake, ws, None) == 2
+    assert lib.csa_out_proj(0, 128, 512, 16, 1024, 7168, fake, fake, fake, fake, ws, None) == 2
+    assert lib.csa_out_proj(4, 128, 512, 16, 1024, 7168, None, fake, fake, fake, ws, None) == 1
+    assert lib.csa_out_proj(4, 128, 512, 16, 1024, 7168, C.c_void_p((1 << 20) + 8), fake, fake,
+                            fake, ws, None) == 3
+    assert lib.csa_out_proj(4, 128, 512, 16, 1024, 7168, fake, fake, fake, None, 0, None) == 8
+    assert lib.csa_out_proj(4, 128, 512, 16, 1024, 7168, fake, fake, fake, fake, 16, None) == 8
+    assert lib.csa_out_proj_pack(128, 512, 16, 1024, 7168, None, fake, fake, None) == 1
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(bd, "_lib", None)
     monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "libcsa.so"))
