@@ -254,8 +254,8 @@ class DecodeStep:
     def time_out_proj(self, steps, stream):
         """Device time of csa_out_proj on the step's attention output (the
         grouped output projection of the workload's g and d_g; graph replays,
-        4 calls per graph; the weights, larger than twice the L2, stream from
-        HBM every call).  Returns (ms per call, packed weight bytes)."""
+        4 calls per graph; weights larger than the L2, streamed from HBM
+        each call).  Returns (ms per call, packed weight bytes)."""
         wl, dev = self.wl, self.out.device
         g, d_g, d = wl.g_out, wl.d_g, wl.d
         Kg = wl.c * wl.n_h // g
