@@ -13,7 +13,7 @@ import numpy as np
 import torch
 
 from . import (attend, compress, fp8mix_decode, fp8mix_encode, index_scores,
-               matmul, norm_rope_rows, nvis, round_bf16, topk, _f64)
+               matmul, norm_rope_rows, nvis, rmsnorm, rope, round_bf16, topk, _f64)
 
 
 def store(x: np.ndarray, fmt: str, rope_dims: int) -> np.ndarray:
@@ -81,3 +81,28 @@ def select(wl, t0s, qI, w, kI):
 def attend_wl(wl, t0s, q, idx, kv, win, win_pos0, sink, rope_shift=0.0):
     return attend(t0s, q, idx, wl.m, kv, wl.n_win, win, win_pos0, sink,
                   wl.rope_dims, wl.rope_base, wl.softmax_scale, rope_shift)
+
+
+def query_proj(H, pos, WDQ, WUQ, WIUQ, Ww, n_h: int, c: int, n_hI: int, c_I: int,
+               rope_dims: int, base: float, eps: float):
+    """The query side of the layer for tokens H [T][d] at positions pos [T]
+    (the reading notes eq. 13-15 and 18; 2.5.1, 2.5.2):
+        c^Q = h W^{DQ}                          (eq. 13, d -> d_c)
+        q^I = c^Q W^{IUQ}, one c_I row per head (eq. 14)
+        w   = h W^{w}                           (eq. 15)
+        q   = c^Q W^{UQ}, one c row per head    (eq. 18)
+    then every head of q is RMS-normalised (unit gain, 2.5.1) and rotated on
+    its last rope_dims at its token's position (2.5.2).  Readings: no norm on
+    c^Q and none and no rotation on q^I (the pages give neither; the
+    indexer keys have neither either).  Returns (c^Q, q, q^I, w)."""
+    H = _f64(H)
+    T = H.shape[0]
+    cQ = matmul(H, WDQ)
+    qI = matmul(cQ, WIUQ).reshape(T, n_hI, c_I)
+    w = matmul(H, Ww)
+    q = matmul(cQ, WUQ).reshape(T, n_h, c)
+    for t in range(T):
+        for h in range(n_h):
+            q[t, h] = rope(rmsnorm(q[t, h], eps), rope_dims, base, float(pos[t]))
+    return cQ, q, qI, w
+

@@ -535,3 +535,63 @@ def test_group_out_proj_parameter_counts_of_the_pages():
     O = np.zeros((1, 4, 2))
     with pytest.raises(ValueError):
         oracle.group_out_proj(O, np.zeros((2, 3, 5)), np.zeros((10, 3)))  # c n_h / g = 4
+
+
+# ------------------------------------------------------ query projections ---
+# "DeepSeekV4技术报告阅读笔记" eq. 13-15, 18 and 2.5.1-2.5.2.
+
+def _qp_inputs(T=5, d=24, d_c=12, n_h=3, c=16, n_hI=2, c_I=8, seed=53):
+    r = rng(seed)
+    return dict(H=r.standard_normal((T, d)), WDQ=r.standard_normal((d, d_c)) / d ** 0.5,
+                WUQ=r.standard_normal((d_c, n_h * c)) / d_c ** 0.5,
+                WIUQ=r.standard_normal((d_c, n_hI * c_I)) / d_c ** 0.5,
+                Ww=r.standard_normal((d, n_hI)) / d ** 0.5,
+                n_h=n_h, c=c, n_hI=n_hI, c_I=c_I)
+
+
+def _qp(x, pos, rope_dims=8, eps=1e-6, **over):
+    a = dict(x)
+    a.update(over)
+    return P.query_proj(a["H"], pos, a["WDQ"], a["WUQ"], a["WIUQ"], a["Ww"], a["n_h"], a["c"],
+                        a["n_hI"], a["c_I"], rope_dims, 10000.0, eps)
+
+
+def test_query_proj_low_rank_chain_is_two_matmuls():
+    x = _qp_inputs()
+    pos = np.arange(5)
+    cQ, q, qI, w = _qp(x, pos)
+    np.testing.assert_allclose(cQ, x["H"] @ x["WDQ"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(qI.reshape(5, -1), (x["H"] @ x["WDQ"]) @ x["WIUQ"],
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(w, x["H"] @ x["Ww"], rtol=1e-12, atol=1e-12)
+
+
+def test_query_heads_are_unit_rms_and_scale_free():
+    """Each q head has mean square 1 after the norm (the rotation keeps it),
+    and scaling h leaves q unchanged while q^I and w scale with it: the norm
+    applies to q only."""
+    x = _qp_inputs()
+    pos = np.array([0, 3, 17, 250, 4095])
+    _, q, qI, w = _qp(x, pos, eps=0.0)
+    np.testing.assert_allclose((q ** 2).mean(axis=2), 1.0, rtol=1e-12)
+    _, q2, qI2, w2 = _qp(x, pos, eps=0.0, H=3.0 * x["H"])
+    np.testing.assert_allclose(q2, q, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(qI2, 3.0 * qI, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(w2, 3.0 * w, rtol=1e-12, atol=1e-12)
+
+
+def test_query_rotation_uses_the_token_position():
+    """q(t) . R_s k depends on t - s only (2.5.2): shifting the query's and
+    the key's positions together leaves the score; position 0 is unrotated."""
+    x = _qp_inputs(T=1)
+    k = rng(7).standard_normal(16)
+    _, q0, _, _ = _qp(x, np.array([0]))
+    _, qn, _, _ = _qp(x, np.array([0]), rope_dims=0)
+    np.testing.assert_allclose(q0, qn, rtol=1e-12, atol=1e-12)
+    for t, s, shift in [(9, 4, 100), (1000, 3, 77)]:
+        _, qa, _, _ = _qp(x, np.array([t]))
+        _, qb, _, _ = _qp(x, np.array([t + shift]))
+        ka, kb = oracle.rope(k, 8, 10000.0, s), oracle.rope(k, 8, 10000.0, s + shift)
+        np.testing.assert_allclose(qa[0] @ ka, qb[0] @ kb, rtol=1e-9, atol=1e-9)
+        _, qc, _, _ = _qp(x, np.array([t + 1]))
+        assert not np.allclose(qc[0] @ ka, qa[0] @ ka)
