@@ -11,11 +11,11 @@
  *   [N]  "DeepSeekV4技术报告阅读笔记" (zouxinn.github.io), 2.3.1 eq. 9-12,
  *        2.3.2 eq. 13-17, 2.3.3 eq. 18-19, 2.4.1 eq. 20-23, 2.4.2 eq. 26,
  *        2.5.1 RMSNorm, 2.5.2 partial RoPE and R_{-t}, 2.5.3 window,
- *        2.5.4 eq. 27 attention sink.
+ *        2.5.4 eq. 27 attention sink; 2.3.3 grouped output projection.
  *   [P]  "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" (PaperTrace), 2.1 (m = 4,
  *        the 2m-slot per-channel softmax), 2.3 (HCA m' = 128, no overlap),
  *        2.4 (RMSNorm, last-64 RoPE, window of n_win, sink), 2.5 (RoPE dims in
- *        BF16, other dims in FP8).
+ *        BF16, other dims in FP8), 2.2 (output-projection groups, d_g).
  * Readings where the pages leave a step open are listed with each routine.
  */
 #include "csa_oracle.h"
