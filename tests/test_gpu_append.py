@@ -28,6 +28,12 @@ APPEND_CASES = [
     ("csa_b18", "csa", "bf16", "bf16", 18, 13, 64, 128, 32, 32, 4),
     # the heavy compression rate: entries span 128 tokens
     ("hca_m128", "hca", "bf16", "bf16", 1, 300, 64, 128, 32, 0, 128),
+    # the bench's launch configurations: the 1M decode (4 sequences, d = 7168,
+    # FP8-mixed; 20 tiles x 7 slices), the 64K decode (32 sequences: two
+    # launches) and the HCA decode (16 sequences, m' = 128)
+    ("pro_decode_shape", "csa", "bf16", "fp8mix", 4, 8, 7168, 512, 64, 128, 4),
+    ("flash_decode_shape", "csa", "bf16", "bf16", 32, 8, 4096, 512, 64, 128, 4),
+    ("hca_decode_shape", "hca", "bf16", "bf16", 16, 128, 4096, 512, 64, 0, 128),
 ]
 
 

@@ -20,6 +20,9 @@ CASES = [
     ("one_group", 5, 4, 64, 1, 128, 136),
     ("flash", 2, 64, 512, 8, 1024, 4096),
     ("pro", 1, 128, 512, 16, 1024, 7168),
+    # the bench's launch configurations: 4 tokens of V4-Pro, 32 of V4-Flash
+    ("pro_decode_shape", 4, 128, 512, 16, 1024, 7168),
+    ("flash_decode_shape", 32, 64, 512, 8, 1024, 4096),
 ]
 
 
