@@ -68,6 +68,10 @@ def _load():
                                 C.c_int, C.c_int, _dp, C.c_int, C.c_int, C.c_int,
                                 C.c_void_p, _dp, C.c_double, _dp, C.c_void_p]
     lib.ocsa_round_bf16.argtypes = [C.c_int, _dp, _dp]
+    lib.ocsa_e2m1_decode.restype = C.c_double
+    lib.ocsa_e2m1_decode.argtypes = [C.c_uint8]
+    lib.ocsa_mxfp4_encode.argtypes = [C.c_int, _dp, _up, _ip]
+    lib.ocsa_mxfp4_decode.argtypes = [C.c_int, _up, _ip, _dp]
     lib.ocsa_group_out_proj.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                         _dp, _dp, _dp, C.c_int, _dp, _dp]
     lib.ocsa_e4m3_decode.restype = C.c_double
@@ -220,6 +224,39 @@ def group_out_proj(O, WG, WO, round_mid: bool = True):
     out = np.empty((Q, d))
     _load().ocsa_group_out_proj(Q, n_h, c, g, d_g, d, O, WG, WO, 1 if round_mid else 0, Y, out)
     return Y, out
+
+
+def e2m1_decode(code: int) -> float:
+    return _load().ocsa_e2m1_decode(int(code))
+
+
+def mxfp4_encode(x):
+    """(codes uint8 [n], scale exponents int32 [ceil(n/32)]) of a vector."""
+    x = np.ascontiguousarray(_f64(x).reshape(-1))
+    codes = np.empty(x.size, dtype=np.uint8)
+    exps = np.empty((x.size + 31) // 32, dtype=np.int32)
+    _load().ocsa_mxfp4_encode(x.size, x, codes, exps)
+    return codes, exps
+
+
+def mxfp4_decode(codes, exps) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    exps = np.ascontiguousarray(exps, dtype=np.int32)
+    y = np.empty(codes.size)
+    _load().ocsa_mxfp4_decode(codes.size, codes, exps, y)
+    return y
+
+
+def mxfp4_round(x, block_axis_len: int | None = None) -> np.ndarray:
+    """The values x takes in MXFP4, blocks of 32 along each row of length
+    block_axis_len (default: the last axis)."""
+    x = _f64(x)
+    n = x.shape[-1] if block_axis_len is None else block_axis_len
+    rows = x.reshape(-1, n)
+    out = np.empty_like(rows)
+    for r in range(rows.shape[0]):
+        out[r] = mxfp4_decode(*mxfp4_encode(rows[r]))
+    return out.reshape(x.shape)
 
 
 def round_bf16(x) -> np.ndarray:

@@ -446,3 +446,54 @@ void ocsa_group_out_proj(int Q, int n_h, int c, int g, int d_g, int d, const dou
     }
   }
 }
+
+/* PaperTrace 3.3 ("FP4 (MXFP4) quantization-aware training ... the CSA
+ * indexer's QK path"): MXFP4 as the OCP Microscaling (MX) formats define it:
+ * blocks of 32 elements share one power-of-two scale (E8M0: 2^e, e in
+ * [-127, 127]); each element is FP4 E2M1 (1 sign, 2 exponent bits with bias
+ * 1, 1 mantissa bit; no infinities or NaN): magnitudes 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6.  Code = sign << 3 | magnitude index.  The block scale is
+ * 2^(floor(log2 max|x|) - 2) (2 = the exponent of E2M1's largest normal);
+ * elements are x / scale rounded to the nearest E2M1 value, ties to an even
+ * mantissa, saturating at 6. */
+double ocsa_e2m1_decode(uint8_t code) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  const double v = mag[code & 7];
+  return (code & 8) ? -v : v;
+}
+
+static uint8_t e2m1_encode(double v) {
+  const double a = fabs(v);
+  /* grid spacing of the binade: 0.5 below 2, 1 in [2, 4), 2 from 4 on */
+  const double step = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);
+  double q = nearbyint(a / step) * step; /* ties to even multiples: even mantissa */
+  if (q > 6.0) q = 6.0;
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  uint8_t m = 0;
+  for (uint8_t i = 0; i < 8; ++i)
+    if (mag[i] == q) m = i;
+  return (uint8_t)((v < 0.0 && q > 0.0 ? 8 : 0) | m);
+}
+
+void ocsa_mxfp4_encode(int n, const double* x, uint8_t* codes, int* scale_exp) {
+  for (int b0 = 0; b0 < n; b0 += 32) {
+    const int nb = n - b0 < 32 ? n - b0 : 32;
+    double amax = 0.0;
+    for (int i = 0; i < nb; ++i) amax = fmax(amax, fabs(x[b0 + i]));
+    int e = -127;
+    if (amax > 0.0) {
+      int ex;
+      frexp(amax, &ex); /* amax = f 2^ex, f in [0.5, 1) */
+      e = (ex - 1) - 2;
+      if (e < -127) e = -127;
+      if (e > 127) e = 127;
+    }
+    scale_exp[b0 / 32] = e;
+    for (int i = 0; i < nb; ++i) codes[b0 + i] = e2m1_encode(ldexp(x[b0 + i], -e));
+  }
+}
+
+void ocsa_mxfp4_decode(int n, const uint8_t* codes, const int* scale_exp, double* y) {
+  for (int i = 0; i < n; ++i) y[i] = ldexp(ocsa_e2m1_decode(codes[i]), scale_exp[i / 32]);
+}
+

@@ -127,6 +127,15 @@ void ocsa_group_out_proj(int Q, int n_h, int c, int g, int d_g, int d, const dou
                          const double* WG, const double* WO, int round_mid, double* Y,
                          double* out);
 
+/* MXFP4 (OCP Microscaling): blocks of 32 sharing a power-of-two scale
+ * 2^scale_exp[block] = 2^(floor(log2 max|x|) - 2); elements E2M1 (codes
+ * sign << 3 | index into 0, 0.5, 1, 1.5, 2, 3, 4, 6), rounded to nearest,
+ * ties to an even mantissa, saturating at 6.  PaperTrace 3.3 (the indexer's
+ * QK path in MXFP4). */
+double ocsa_e2m1_decode(uint8_t code);
+void ocsa_mxfp4_encode(int n, const double* x, uint8_t* codes, int* scale_exp);
+void ocsa_mxfp4_decode(int n, const uint8_t* codes, const int* scale_exp, double* y);
+
 #ifdef __cplusplus
 }
 #endif

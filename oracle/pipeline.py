@@ -13,7 +13,8 @@ import numpy as np
 import torch
 
 from . import (attend, compress, fp8mix_decode, fp8mix_encode, index_scores,
-               matmul, norm_rope_rows, nvis, rmsnorm, rope, round_bf16, topk, _f64)
+               matmul, mxfp4_round, norm_rope_rows, nvis, rmsnorm, rope, round_bf16, topk,
+               _f64)
 
 
 def store(x: np.ndarray, fmt: str, rope_dims: int) -> np.ndarray:
@@ -105,4 +106,27 @@ def query_proj(H, pos, WDQ, WUQ, WIUQ, Ww, n_h: int, c: int, n_hI: int, c_I: int
         for h in range(n_h):
             q[t, h] = rope(rmsnorm(q[t, h], eps), rope_dims, base, float(pos[t]))
     return cQ, q, qI, w
+
+
+def index_scores_fp4(wl, t0s, qI, w, kI):
+    """Index scores of eq. 16 with the QK path in MXFP4 and bf16 scores
+    (PaperTrace 3.3): every head of q^I and every row of K^I is rounded to
+    MXFP4 along c_I (blocks of 32); the products, ReLU and the w-weighted
+    head sum are then exact, and the score is rounded to bf16 (-inf where
+    the entry is not visible).  Readings: w stays fp32; the rounding to bf16
+    is the score's only rounding after the inputs'."""
+    s = index_scores(t0s, wl.m, mxfp4_round(qI), w, mxfp4_round(kI))
+    return np.where(np.isfinite(s), round_bf16(np.where(np.isfinite(s), s, 0.0)), s)
+
+
+def topk_recall(idx_a, idx_b) -> np.ndarray:
+    """Per query, the fraction of idx_b's selected entries (-1 padding
+    ignored) that idx_a also selects: the KV recall of a selection."""
+    idx_a, idx_b = np.asarray(idx_a), np.asarray(idx_b)
+    out = np.empty(idx_a.shape[0])
+    for q in range(idx_a.shape[0]):
+        b = set(int(i) for i in idx_b[q] if i >= 0)
+        a = set(int(i) for i in idx_a[q] if i >= 0)
+        out[q] = len(a & b) / len(b) if b else 1.0
+    return out
 

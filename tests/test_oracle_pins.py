@@ -595,3 +595,89 @@ def test_query_rotation_uses_the_token_position():
         np.testing.assert_allclose(qa[0] @ ka, qb[0] @ kb, rtol=1e-9, atol=1e-9)
         _, qc, _, _ = _qp(x, np.array([t + 1]))
         assert not np.allclose(qc[0] @ ka, qa[0] @ ka)
+
+
+# ------------------------------------------------------------------ MXFP4 ---
+# The indexer's QK path in MXFP4 ("02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文"
+# 3.3); the format is the OCP Microscaling one (tests/golden/e2m1_values.txt).
+
+def _golden_e2m1():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "e2m1_values.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    return {int(r[0]): float(r[-1]) for r in rows}
+
+
+def test_e2m1_decode_matches_the_spec_table():
+    for code, v in _golden_e2m1().items():
+        got = oracle.e2m1_decode(code)
+        assert got == v and math.copysign(1.0, got) == math.copysign(1.0, v), code
+
+
+def _nearest_e2m1(v):
+    """Brute force: the E2M1 magnitude nearest to |v| (ties to the even
+    mantissa, i.e. the even code), saturating at 6."""
+    grid = [(abs(val), code) for code, val in _golden_e2m1().items() if code < 8]
+    a = min(abs(v), 6.0)
+    best = min(grid, key=lambda g: (abs(g[0] - a), g[1] & 1))
+    return math.copysign(best[0], v) if best[0] else 0.0
+
+
+def test_mxfp4_elements_are_the_nearest_e2m1_values():
+    r = rng(61)
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 7.9]
+    for trial in range(50):
+        x = r.uniform(-8, 8, 32)
+        x[0] = 7.5 if trial % 2 else -7.5  # block maximum in [4, 8): scale 2^0
+        x[1:1 + len(mids)] = mids
+        codes, exps = oracle.mxfp4_encode(x)
+        assert exps.tolist() == [0]
+        got = oracle.mxfp4_decode(codes, exps)
+        want = np.array([_nearest_e2m1(v) for v in x])
+        np.testing.assert_array_equal(np.abs(got), np.abs(want))
+
+
+def test_mxfp4_block_scale_and_error_bound():
+    r = rng(62)
+    for _ in range(40):
+        x = r.standard_normal(96) * 10.0 ** r.uniform(-3, 3)
+        codes, exps = oracle.mxfp4_encode(x)
+        y = oracle.mxfp4_decode(codes, exps)
+        for b in range(3):
+            blk, e = x[32 * b:32 * b + 32], int(exps[b])
+            amax = np.abs(blk).max()
+            assert 4.0 * 2.0 ** e <= amax < 8.0 * 2.0 ** e   # the top binade holds the max
+            err = np.abs(y[32 * b:32 * b + 32] - blk)
+            # half a grid step (at most 1 scale unit) below 6, saturation above
+            assert np.all(err <= np.maximum(2.0 ** e, np.abs(blk) - 6.0 * 2.0 ** e) + 1e-300)
+
+
+def test_mxfp4_power_of_two_equivariance():
+    x = rng(63).standard_normal(64)
+    c0, e0 = oracle.mxfp4_encode(x)
+    c1, e1 = oracle.mxfp4_encode(x * 2.0 ** 5)
+    np.testing.assert_array_equal(c0, c1)
+    np.testing.assert_array_equal(e1, e0 + 5)
+
+
+def test_fp4_index_scores_on_representable_inputs():
+    """Inputs already in MXFP4 pass unchanged: the FP4 scores are the exact
+    scores rounded to bf16; a top-k on them keeps full recall of itself."""
+    wl = WORKLOADS["tiny_csa_prefill_f32"]
+    r = rng(64)
+    n_hI, c_I, N = wl.n_hI, wl.c_I, 40
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    kI = r.choice(grid, (N, c_I)) * r.choice([-1, 1], (N, c_I)) * 2.0 ** -3
+    kI[:, ::32] = 6.0 * 2.0 ** -3  # every block holds its top value
+    qI = r.choice(grid, (2, n_hI, c_I)) * 2.0 ** -2
+    qI[:, :, ::32] = 4.0 * 2.0 ** -2
+    w = r.standard_normal((2, n_hI))
+    t0s = np.array([N * wl.m - 1, 17])
+    np.testing.assert_array_equal(oracle.mxfp4_round(kI), kI)
+    s4 = P.index_scores_fp4(wl, t0s, qI, w, kI)
+    ref = oracle.index_scores(t0s, wl.m, qI, w, kI)
+    fin = np.isfinite(ref)
+    np.testing.assert_array_equal(np.isfinite(s4), fin)
+    np.testing.assert_array_equal(s4[fin], oracle.round_bf16(ref[fin]))
+    idx, _ = oracle.topk(s4, np.array([oracle.nvis(int(t), wl.m, N) for t in t0s]), 8)
+    assert P.topk_recall(idx, idx).tolist() == [1.0, 1.0]
