@@ -4,19 +4,24 @@
  * The operations are those of DeepSeek-V4's Compressed Sparse Attention and
  * Heavily Compressed Attention as described in "DeepSeekV4技术报告阅读笔记"
  * (zouxinn.github.io; cited below as [N] with its section / equation numbers)
- * and "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" (PaperTrace; cited as [P]).
+ * and "02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" (PaperTrace; cited as [P]):
+ * compression (prefill, and one token at a time for decode), indexer scores
+ * and top-k, the shared-KV attention with window and sink, and the grouped
+ * output projection that follows it.
  *
  * Conventions for every call
  *   - All tensor arguments are DEVICE pointers to caller-owned memory, laid
  *     out row-major with the last dimension contiguous, as stated per
- *     argument.  The library allocates nothing and keeps no state besides one
- *     device error word per GPU.
+ *     argument.  The library allocates nothing and keeps no device state
+ *     besides one error word per GPU (and the fixed scratch array of
+ *     csa_index_topk_noalloc).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and runs asynchronously; outputs are valid once the stream has
  *     reached the call.
  *   - Argument errors are reported synchronously by the return value before
  *     anything is launched.  Errors found on the device (an index or window
- *     row out of range) set bits in the device error word, which
+ *     row out of range, a bounded wait that ran out) set bits in the device
+ *     error word, which
  *     csa_device_status() reads; the offending element is skipped, never
  *     dereferenced.
  *   - Queries are numbered r = b*Q + j for sequence b < B and query j < Q.
