@@ -110,6 +110,15 @@ def _p(t):
     return C.c_void_p(t.data_ptr())
 
 
+def _want(t, dtype, what, min_bytes=0):
+    """Argument check of the binding: a tensor of the dtype the call reads,
+    holding at least min_bytes (the C ABI sees only the pointer)."""
+    if t.dtype != dtype:
+        raise ValueError(f"{what}: {dtype} expected, got {t.dtype}")
+    if t.numel() * t.element_size() < min_bytes:
+        raise ValueError(f"{what}: at least {min_bytes} bytes expected")
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return C.c_void_p(s.cuda_stream)
@@ -230,6 +239,10 @@ def out_proj_pack(WG, WO, stream=None) -> torch.Tensor:
     packing takes n_h = g, c = c n_h / g."""
     g, Kg, d_g = WG.shape
     d = WO.shape[1]
+    _want(WG, torch.bfloat16, "WG")
+    _want(WO, torch.bfloat16, "WO")
+    if WO.shape[0] != g * d_g:
+        raise ValueError("WO: [g d_g][d] expected")
     nbytes = lib().csa_out_proj_packed_bytes(g, Kg, g, d_g, d)
     if nbytes == 0:
         raise CsaError("csa_out_proj_packed_bytes", 2, "unsupported shapes")
@@ -247,6 +260,9 @@ def csa_out_proj(O, packed, g, d_g, out, workspace=None, stream=None):
     """O [R][n_h][c] bf16 -> out [R][d] bf16 (grouped output projection)."""
     R, n_h, c = O.shape
     d = out.shape[1]
+    _want(O, torch.bfloat16, "O")
+    _want(out, torch.bfloat16, "out", R * d * 2)
+    _want(packed, torch.uint8, "packed", lib().csa_out_proj_packed_bytes(n_h, c, g, d_g, d))
     ws, wsb = _ws(out_proj_workspace_bytes(R, n_h, c, g, d_g, d), O.device, workspace)
     st = lib().csa_out_proj(R, n_h, c, g, d_g, d, _p(O), _p(packed), _p(out), _p(ws), wsb,
                             _stream(stream))

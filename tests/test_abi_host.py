@@ -156,3 +156,16 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(bd, "LIB_PATH", str(tmp_path / "libcsa.so"))
     with pytest.raises(RuntimeError):
         bd.lib()
+
+
+def test_binding_checks_dtypes_and_sizes_before_the_call(lib):
+    import torch
+    O = torch.zeros(2, 8, 64)  # fp32: the call reads bf16
+    out = torch.zeros(2, 200, dtype=torch.bfloat16)
+    packed = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="O"):
+        bd.csa_out_proj(O, packed, 2, 128, out)
+    with pytest.raises(ValueError, match="packed"):  # smaller than the packed weights
+        bd.csa_out_proj(O.to(torch.bfloat16), packed, 2, 128, out)
+    with pytest.raises(ValueError, match="WG"):
+        bd.out_proj_pack(torch.zeros(2, 256, 128), torch.zeros(256, 200, dtype=torch.bfloat16))
