@@ -207,11 +207,23 @@ def decode_tail_bytes(p: CsaParams, B, d) -> int:
     return lib().csa_decode_tail_bytes(C.byref(p), B, d)
 
 
+def _append_args(p: CsaParams, H, t, tail, win, win_pos0):
+    """The decode append reads H in the activation dtype, B int32 positions
+    and a tail of decode_tail_bytes; check them (the C ABI sees pointers)."""
+    B, d = H.shape
+    _want(H, torch.float32 if p.act == CSA_F32 else torch.bfloat16, "H")
+    _want(t, torch.int32, "t", B * 4)
+    _want(tail, torch.float32, "tail", decode_tail_bytes(p, B, d))
+    if win is not None:
+        _want(win_pos0, torch.int32, "win_pos0", B * 4)
+
+
 def csa_decode_append(p: CsaParams, H, t, packed, tail, ckv, ckv_scale, kI, win, win_scale,
                       win_pos0, stream=None):
     """H [B][d] new tokens at positions t [B]; tail from decode_tail_bytes;
     ckv [B][N][row] (ckv_scale [B][N]), kI [B][N][c_I], win [B][W][row]
     (win_scale [B][W]), win_pos0 [B]."""
+    _append_args(p, H, t, tail, win, win_pos0)
     B, d = H.shape
     N = ckv.shape[1]
     W = win.shape[1] if win is not None else 0
@@ -223,6 +235,7 @@ def csa_decode_append(p: CsaParams, H, t, packed, tail, ckv, ckv_scale, kI, win,
 
 def hca_decode_append(p: CsaParams, H, t, packed, tail, ckv, ckv_scale, win, win_scale,
                       win_pos0, stream=None):
+    _append_args(p, H, t, tail, win, win_pos0)
     B, d = H.shape
     N = ckv.shape[1]
     W = win.shape[1] if win is not None else 0

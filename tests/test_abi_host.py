@@ -169,3 +169,22 @@ def test_binding_checks_dtypes_and_sizes_before_the_call(lib):
         bd.csa_out_proj(O.to(torch.bfloat16), packed, 2, 128, out)
     with pytest.raises(ValueError, match="WG"):
         bd.out_proj_pack(torch.zeros(2, 256, 128), torch.zeros(256, 200, dtype=torch.bfloat16))
+
+
+def test_binding_checks_decode_append_inputs(lib):
+    import torch
+    wl = WORKLOADS["pro_csa_decode_1m"]
+    p = bd.params_for(wl)
+    B, d = 2, wl.d
+    H = torch.zeros(B, d)  # fp32 for a bf16 configuration
+    t = torch.zeros(B, dtype=torch.int32)
+    tail = torch.zeros(bd.decode_tail_bytes(p, B, d) // 4)
+    with pytest.raises(ValueError, match="H"):
+        bd.csa_decode_append(p, H, t, None, tail, None, None, None, None, None, None)
+    with pytest.raises(ValueError, match="tail"):
+        bd.csa_decode_append(p, H.to(torch.bfloat16), t, None, tail[:10], None, None, None,
+                             None, None, None)
+    with pytest.raises(ValueError, match="t"):
+        bd.hca_decode_append(bd.params_for(WORKLOADS["hca_decode_1m"]),
+                             torch.zeros(B, 4096, dtype=torch.bfloat16), t.long(), None, tail,
+                             None, None, None, None, None)
