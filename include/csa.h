@@ -238,10 +238,14 @@ csa_status csa_index_topk(const csa_params* p, int B, int Q,
  * synchronise the device.  The pages have no counterpart: this is a library
  * convenience, not part of the method.
  *   Same arguments and results as csa_index_topk, without the workspace.
- *   The scratch is one fixed 16 MiB device array inside the library (enough
- *   for B*Q*N <= 4,194,304 scores); it occupies that memory on every GPU
- *   that loads the library until the process exits.  A request that needs
- *   more returns CSA_ERR_WORKSPACE before anything is launched.
+ *   The scratch is one fixed 16 MiB device array inside the library; it
+ *   occupies that memory on every GPU that loads the library until the
+ *   process exits.  A request fits when csa_index_topk_workspace_bytes(p, B,
+ *   Q, N) -- the workspace csa_index_topk would take: 4 B*Q*N bytes of fp32
+ *   scores, the tile plan and, for a few long queries, the multi-CTA top-k
+ *   lists -- is at most 16 MiB (16,777,216 bytes); the 1M-context decode of
+ *   4 sequences needs about 6.6 MiB.  A request that needs more returns
+ *   CSA_ERR_WORKSPACE before anything is launched.
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
  *   Every call on a device shares the same array: calls whose kernels can

@@ -119,6 +119,46 @@ def _want(t, dtype, what, min_bytes=0):
         raise ValueError(f"{what}: at least {min_bytes} bytes expected")
 
 
+def _act(p: CsaParams):
+    return torch.float32 if p.act == CSA_F32 else torch.bfloat16
+
+
+def _esize(p: CsaParams) -> int:
+    return 4 if p.act == CSA_F32 else 2
+
+
+def kv_row_bytes(p: CsaParams) -> int:
+    """Bytes of one cache row in the KV format of p."""
+    if p.kv == CSA_F32:
+        return 4 * p.c
+    if p.kv == CSA_BF16:
+        return 2 * p.c
+    return (p.c - p.rope_dims) + 2 * p.rope_dims
+
+
+def _want_kv(p: CsaParams, rec, scale, rows: int, what: str):
+    """A cache of `rows` rows in the KV format of p (and its scale plane)."""
+    if rec is None:
+        return
+    if p.kv == CSA_KV_FP8MIX:
+        _want(rec, torch.uint8, what, rows * kv_row_bytes(p))
+        if scale is None:
+            raise ValueError(f"{what}_scale: the FP8-mixed format needs its scale plane")
+        _want(scale, torch.float32, what + "_scale", rows * 4)
+    else:
+        _want(rec, torch.float32 if p.kv == CSA_F32 else torch.bfloat16, what,
+              rows * kv_row_bytes(p))
+        if scale is not None:
+            raise ValueError(f"{what}_scale: only the FP8-mixed format has a scale plane")
+
+
+def _per_seq(n: int, B: int, what: str) -> int:
+    if B <= 0 or n % B != 0:
+        raise ValueError(f"{what}: {n} rows are not a whole number of rows per sequence "
+                         f"for {B} sequences")
+    return n // B
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return C.c_void_p(s.cuda_stream)
@@ -184,8 +224,22 @@ def compress_workspace_bytes(p: CsaParams, B, T, d) -> int:
     return lib().csa_compress_workspace_bytes(C.byref(p), B, T, d)
 
 
+def _compress_args(p: CsaParams, H, packed, ckv, ckv_scale, kI, win, win_scale):
+    """csa_compress / hca_compress read H in the activation dtype and write
+    T/m entries (and indexer keys) and T window rows per sequence."""
+    B, T, d = H.shape
+    _want(H, _act(p), "H")
+    _want(packed, torch.uint8, "packed", lib().csa_packed_weight_bytes(C.byref(p), d))
+    nE = T // p.m
+    _want_kv(p, ckv, ckv_scale, B * nE, "ckv")
+    if kI is not None:
+        _want(kI, _act(p), "kI", B * nE * p.c_I * _esize(p))
+    _want_kv(p, win, win_scale, B * T, "win")
+
+
 def csa_compress(p: CsaParams, H, packed, ckv, ckv_scale, kI, win, win_scale,
                  workspace=None, stream=None):
+    _compress_args(p, H, packed, ckv, ckv_scale, kI, win, win_scale)
     B, T, d = H.shape
     ws, wsb = _ws(compress_workspace_bytes(p, B, T, d), H.device, workspace)
     st = lib().csa_compress(C.byref(p), B, T, d, _p(H), _p(packed), _p(ckv), _p(ckv_scale),
@@ -195,6 +249,7 @@ def csa_compress(p: CsaParams, H, packed, ckv, ckv_scale, kI, win, win_scale,
 
 def hca_compress(p: CsaParams, H, packed, ckv, ckv_scale, win, win_scale,
                  workspace=None, stream=None):
+    _compress_args(p, H, packed, ckv, ckv_scale, None, win, win_scale)
     B, T, d = H.shape
     ws, wsb = _ws(compress_workspace_bytes(p, B, T, d), H.device, workspace)
     st = lib().hca_compress(C.byref(p), B, T, d, _p(H), _p(packed), _p(ckv), _p(ckv_scale),
@@ -287,12 +342,28 @@ def index_topk_workspace_bytes(p: CsaParams, B, Q, N) -> int:
     return lib().csa_index_topk_workspace_bytes(C.byref(p), B, Q, N)
 
 
+def _index_args(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out):
+    """Shapes of csa_index_topk's tensors, checked against what the call
+    reads and writes; returns (B, Q, N)."""
+    B, N = kI.shape[0], kI.shape[1]
+    R = qI.shape[0]
+    Q = _per_seq(R, B, "qI")
+    es = _esize(p)
+    _want(qI, _act(p), "qI", R * p.n_hI * p.c_I * es)
+    _want(kI, _act(p), "kI", B * N * p.c_I * es)
+    _want(w, torch.float32, "w", R * p.n_hI * 4)
+    _want(q_pos, torch.int32, "q_pos", R * 4)
+    _want(idx_out, torch.int32, "idx_out", R * p.topk * 4)
+    if score_out is not None:
+        _want(score_out, torch.float32, "score_out", R * p.topk * 4)
+    return B, Q, N
+
+
 def csa_index_topk(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out=None,
                    workspace=None, stream=None):
     """q_pos [B*Q], qI [B*Q][n_hI][c_I], w [B*Q][n_hI], kI [B][N][c_I] ->
     idx_out [B*Q][topk] (and score_out [B*Q][topk])."""
-    B, N = kI.shape[0], kI.shape[1]
-    Q = qI.shape[0] // B
+    B, Q, N = _index_args(p, q_pos, qI, w, kI, idx_out, score_out)
     ws, wsb = _ws(index_topk_workspace_bytes(p, B, Q, N), qI.device, workspace)
     st = lib().csa_index_topk(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI), N,
                               _p(idx_out), _p(score_out), _p(ws), wsb, _stream(stream))
@@ -303,8 +374,7 @@ def csa_index_topk_noalloc(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out=No
                            stream=None):
     """csa_index_topk with the library's fixed scratch instead of a
     workspace (for callers that cannot allocate device memory)."""
-    B, N = kI.shape[0], kI.shape[1]
-    Q = qI.shape[0] // B
+    B, Q, N = _index_args(p, q_pos, qI, w, kI, idx_out, score_out)
     st = lib().csa_index_topk_noalloc(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI), N,
                                       _p(idx_out), _p(score_out), _stream(stream))
     _check("csa_index_topk_noalloc", st)
@@ -315,13 +385,38 @@ def attend_workspace_bytes(p: CsaParams, B, Q, N) -> int:
     return lib().csa_attend_workspace_bytes(C.byref(p), B, Q, N)
 
 
+def _attend_args(p: CsaParams, q_pos, q, idx, ckv, ckv_scale, win, win_scale, win_pos0,
+                 sink, out):
+    """Shapes of csa_attend / hca_attend's tensors, checked against what the
+    call reads and writes; returns (B, Q, N, W)."""
+    B, N = ckv.shape[0], ckv.shape[1]
+    R = q.shape[0]
+    Q = _per_seq(R, B, "q")
+    W = win.shape[1] if win is not None else 0
+    es = _esize(p)
+    _want(q, _act(p), "q", R * p.n_h * p.c * es)
+    _want(out, _act(p), "out", R * p.n_h * p.c * es)
+    _want(q_pos, torch.int32, "q_pos", R * 4)
+    _want(sink, torch.float32, "sink", p.n_h * 4)
+    if idx is not None:
+        _want(idx, torch.int32, "idx", R * p.topk * 4)
+    _want_kv(p, ckv, ckv_scale, B * N, "ckv")
+    if win is not None:
+        if win.shape[0] != B:
+            raise ValueError("win: one window per sequence expected")
+        _want_kv(p, win, win_scale, B * W, "win")
+        _want(win_pos0, torch.int32, "win_pos0", B * 4)
+    return B, Q, N, W
+
+
 def csa_attend(p: CsaParams, q_pos, q, idx, ckv, ckv_scale, win, win_scale, win_pos0,
                sink, out, workspace=None, stream=None):
     """q [B*Q][n_h][c], idx [B*Q][topk], ckv [B][N][row], win [B][W][row] ->
     out [B*Q][n_h][c]."""
-    B, N = ckv.shape[0], ckv.shape[1]
-    Q = q.shape[0] // B
-    W = win.shape[1] if win is not None else 0
+    if idx is None:
+        raise ValueError("idx: csa_attend attends selected entries")
+    B, Q, N, W = _attend_args(p, q_pos, q, idx, ckv, ckv_scale, win, win_scale, win_pos0,
+                              sink, out)
     ws, wsb = _ws(attend_workspace_bytes(p, B, Q, N), q.device, workspace)
     st = lib().csa_attend(C.byref(p), B, Q, _p(q_pos), _p(q), _p(idx), _p(ckv), _p(ckv_scale),
                           N, _p(win), _p(win_scale), W, _p(win_pos0), _p(sink), _p(out),
@@ -331,9 +426,8 @@ def csa_attend(p: CsaParams, q_pos, q, idx, ckv, ckv_scale, win, win_scale, win_
 
 def hca_attend(p: CsaParams, q_pos, q, ckv, ckv_scale, win, win_scale, win_pos0, sink,
                out, workspace=None, stream=None):
-    B, N = ckv.shape[0], ckv.shape[1]
-    Q = q.shape[0] // B
-    W = win.shape[1] if win is not None else 0
+    B, Q, N, W = _attend_args(p, q_pos, q, None, ckv, ckv_scale, win, win_scale, win_pos0,
+                              sink, out)
     ws, wsb = _ws(attend_workspace_bytes(p, B, Q, N), q.device, workspace)
     st = lib().hca_attend(C.byref(p), B, Q, _p(q_pos), _p(q), _p(ckv), _p(ckv_scale), N,
                           _p(win), _p(win_scale), W, _p(win_pos0), _p(sink), _p(out),

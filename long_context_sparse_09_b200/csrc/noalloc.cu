@@ -9,6 +9,7 @@
 // indexer) from a fixed array compiled into the library instead of a
 // caller-provided workspace.  The array lives in device memory on every GPU
 // that loads the library, from the first call until the process exits.
+#include <atomic>
 #include <cstdint>
 
 #include "common.cuh"
@@ -16,24 +17,29 @@
 
 namespace csa {
 
-// 16 MiB: room for B*Q*N = 4,194,304 fp32 scores (the 1M-context decode of 4
-// sequences needs 1,048,576).
+// 16 MiB.  A request fits when csa_index_topk_workspace_bytes(p, B, Q, N),
+// the workspace the allocating entry point would take, is at most this: the
+// fp32 scores (4 B*Q*N bytes) plus the tile plan and, for a few long
+// queries, the multi-CTA top-k lists.  The 1M-context decode of 4 sequences
+// needs about 6.6 MiB.
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device
 // memory: its device address is looked up once per device, with that device
-// current, and cached here.
+// current, and cached here.  Host threads may make their first calls on a
+// device at the same time: each slot is an atomic, and a thread that finds
+// it empty looks the address up itself (the lookups agree).
 static void* noalloc_scratch_ptr() {
-  static void* addr[64] = {nullptr};
+  static std::atomic<void*> addr[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
+  void* p = addr[dev].load(std::memory_order_relaxed);
+  if (p == nullptr) {
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
+    addr[dev].store(p, std::memory_order_relaxed);
   }
-  return addr[dev];
+  return p;
 }
 
 }  // namespace csa

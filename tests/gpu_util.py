@@ -108,3 +108,79 @@ def check_topk(idx_gpu, score_gpu, scores_ref, nv, k, tol, what=""):
                 assert gap <= lim, (
                     f"{what} q{q}: index {s} differs, |I(s)-I(kth)| = {gap:.3g} "
                     f"> 1e-6 relative ({lim:.3g})")
+
+
+# ------------------------------------------------------ FP8-mixed records --
+# Relative deviation allowed between the GPU's fp32 row (the value it
+# quantises) and the oracle's fp64 row, as a fraction of the row's largest
+# FP8-dim magnitude.  Both sides compute the same row from the same stored
+# inputs; they differ only by fp32 rounding in the GPU's sums (bf16 products
+# accumulated in fp32 over d terms, the 2m-slot softmax, RMSNorm, RoPE), a few
+# parts in 10^7 of max|x| on these inputs; 2^-16 = 1.5e-5 leaves a 30x margin.
+FP8_SLACK = 2.0 ** -16
+
+_E4M3 = None
+
+
+def _e4m3_values() -> np.ndarray:
+    global _E4M3
+    if _E4M3 is None:
+        _E4M3 = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    return _E4M3
+
+
+def check_fp8_records(rec, scale, x_ref, wl, what, slack=FP8_SLACK):
+    """Pin of the FP8-mixed storage rule on the GPU's records ("02 ·
+    DeepSeek-V4: 压缩注意力撑起 1M 上下文" 2.5: RoPE dims in BF16, the others in
+    FP8; the reading: per row scale = max|x| / 448 over the FP8 dims in
+    fp32, E4M3 code = round-to-nearest-even, saturating, of x / scale).
+
+    rec [.., rows, (c - rope) + 2 rope] uint8 and scale [.., rows] fp32 are
+    the GPU's; x_ref [rows][c] is the oracle's unquantised fp64 row.
+    * scale: equal to oracle.fp8mix_encode's scale within `slack` relative
+      (a rule such as max|x| / 240 is off by 87%);
+    * codes: the GPU quantises its own fp32 row, which lies within
+      slack * max|x| of the oracle's, so its scaled value lies within
+      y +- slack * (448 + |y|) of the oracle's y = x / scale.  Rounding to
+      nearest is monotone, so the GPU's code must decode to a value between
+      the oracle encoder's codes of those two extremes: the oracle's own code
+      wherever the band holds no rounding boundary (nearly every element),
+      its neighbour only where it does.  Truncation, a wrong scale or a
+      wrong rounding mode fail on most elements;
+    * RoPE dims: the GPU's bf16 value lies between the bf16 roundings of the
+      two extremes x +- slack * max|x|."""
+    r2 = rec.detach().cpu().contiguous().reshape(-1, rec.shape[-1]).numpy()
+    sg = scale.detach().cpu().reshape(-1).numpy().astype(np.float64)
+    x = np.asarray(x_ref, dtype=np.float64).reshape(-1, wl.c)
+    assert r2.shape[0] == x.shape[0], (what, r2.shape, x.shape)
+    nf = wl.c - wl.rope_dims
+    codes_o, _, s_o = oracle.fp8mix_encode(x, wl.rope_dims)
+    s_o = s_o.astype(np.float64)
+    rel = np.abs(sg / s_o - 1.0)
+    assert rel.max() <= slack, (
+        f"{what}: scale differs from max|x|/448 by {rel.max():.3g} relative (> {slack:.3g}) "
+        f"at row {int(rel.argmax())}")
+    y = (x[:, :nf].astype(np.float32) / s_o[:, None].astype(np.float32)).astype(np.float64)
+    band = slack * (448.0 + np.abs(y))
+    enc = np.vectorize(oracle.e4m3_encode, otypes=[np.uint8])
+    tab = _e4m3_values()
+    v_lo = tab[enc(np.clip(y - band, -448.0, 448.0))]
+    v_hi = tab[enc(np.clip(y + band, -448.0, 448.0))]
+    cg = r2[:, :nf]
+    v_g = tab[cg]
+    bad = (v_g < v_lo) | (v_g > v_hi)
+    n_diff = int(np.count_nonzero(cg != codes_o))
+    assert not bad.any(), (
+        f"{what}: {int(bad.sum())} E4M3 codes outside the rounding band "
+        f"(first at {np.argwhere(bad)[0].tolist()}: gpu {int(cg[bad][0]):#x}, oracle "
+        f"{int(codes_o[bad][0]):#x}); {n_diff} codes differ in all")
+    # RoPE dims: little-endian bf16 bit patterns after the codes
+    bits = r2[:, nf:].copy().view(np.uint16).astype(np.uint32) << 16
+    got_r = bits.view(np.float32).astype(np.float64)
+    amax = (s_o * 448.0)[:, None]
+    xr = x[:, nf:]
+    r_lo = oracle.round_bf16(xr - slack * amax)
+    r_hi = oracle.round_bf16(xr + slack * amax)
+    bad_r = (got_r < r_lo) | (got_r > r_hi)
+    assert not bad_r.any(), f"{what}: {int(bad_r.sum())} bf16 RoPE dims outside the rounding band"
+    return n_diff
