@@ -300,6 +300,20 @@ csa_status hca_attend(const csa_params* p, int B, int Q, const int32_t* q_pos,
  * this process (all GPUs), a counter for benchmarks.
  * ------------------------------------------------------------------------- */
 csa_status csa_device_status(csa_stream_t stream, uint32_t* flags);
+
+/* csa_diag_bounded_wait: runs, on purpose, the failure path of the bounded
+ * device-side wait that every kernel of the library uses (no page
+ * counterpart: a diagnostic of the library).  One CTA holds a TMEM
+ * allocation and waits on an mbarrier with a limit of limit_ns
+ * (0 < limit_ns <= 2e9, the kernels' own limit); with arrive = 0 nothing
+ * arrives, the wait gives up, CSA_DEV_TIMEOUT is set in the device error
+ * word and the CTA winds down like the library's kernels (TMEM freed, kernel
+ * returns); with arrive = 1 a second warp arrives after limit_ns / 10 and
+ * the wait completes.  waited_ns (device pointer, nullable) receives the
+ * time spent waiting.  CSA_ERR_ARG for a limit out of range or arrive not
+ * 0/1. */
+csa_status csa_diag_bounded_wait(uint64_t limit_ns, int arrive, uint64_t* waited_ns,
+                                 csa_stream_t stream);
 const char* csa_status_string(csa_status s);
 uint64_t csa_kernel_launches(void);
 int csa_abi_version(void);

@@ -72,6 +72,7 @@ _SIGS = {
     "csa_index_topk_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_noalloc": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
+    "csa_diag_bounded_wait": (C.c_int, [C.c_uint64, _i, _vp, _vp]),
     "csa_attend_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_attend": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp,
                              _vp, _vp, _sz, _vp]),
@@ -185,6 +186,17 @@ def device_status(stream=None) -> int:
     flags = C.c_uint32(0)
     _check("csa_device_status", lib().csa_device_status(_stream(stream), C.byref(flags)))
     return flags.value
+
+
+def diag_bounded_wait(limit_ns: int, arrive: bool, waited=None, stream=None):
+    """Run the bounded device wait's failure path (arrive False) or its
+    completing path (arrive True); waited: optional int64 device tensor of
+    one element receiving the ns spent waiting."""
+    if waited is not None:
+        _want(waited, torch.int64, "waited", 8)
+    _check("csa_diag_bounded_wait",
+           lib().csa_diag_bounded_wait(int(limit_ns), 1 if arrive else 0, _p(waited),
+                                       _stream(stream)))
 
 
 def profile_enable(on: bool = True):

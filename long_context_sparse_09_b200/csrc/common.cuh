@@ -17,7 +17,7 @@ void count_launch(int n = 1);
 // Kernel kinds for the profiler (csa_profile_*).
 enum KernelKind {
   KK_PACK = 0, KK_GEMM, KK_FOLD, KK_WINDOW, KK_SCORES, KK_TOPK, KK_ATTN,
-  KK_COMBINE, KK_PLAN, KK_TOPK_HIST, KK_TOPK_SELECT, KK_TOPK_FINAL, KK_COUNT
+  KK_COMBINE, KK_PLAN, KK_TOPK_HIST, KK_TOPK_SELECT, KK_TOPK_FINAL, KK_DIAG, KK_COUNT
 };
 // Bracket one launch: begin() before it, end() after it, same stream.
 int prof_begin(int kind, cudaStream_t st);

@@ -61,7 +61,7 @@ void prof_end(int slot, cudaStream_t st) {
 static const char* kKindNames[KK_COUNT] = {
     "pack_weights", "compress_gemm", "compress_fold", "compress_window", "index_scores",
     "topk_radix", "attend", "attend_combine", "index_plan", "topk_hist", "topk_select",
-    "topk_final"};
+    "topk_final", "diag_bounded_wait"};
 
 unsigned int* device_error_word() {
   // cudaGetSymbolAddress is per device; cache one address per device index.
