@@ -85,7 +85,7 @@ def attend_wl(wl, t0s, q, idx, kv, win, win_pos0, sink, rope_shift=0.0):
 
 
 def query_proj(H, pos, WDQ, WUQ, WIUQ, Ww, n_h: int, c: int, n_hI: int, c_I: int,
-               rope_dims: int, base: float, eps: float):
+               rope_dims: int, base: float, eps: float, round_mid: bool = False):
     """The query side of the layer for tokens H [T][d] at positions pos [T]
     (the reading notes eq. 13-15 and 18; 2.5.1, 2.5.2):
         c^Q = h W^{DQ}                          (eq. 13, d -> d_c)
@@ -95,10 +95,16 @@ def query_proj(H, pos, WDQ, WUQ, WIUQ, Ww, n_h: int, c: int, n_hI: int, c_I: int
     then every head of q is RMS-normalised (unit gain, 2.5.1) and rotated on
     its last rope_dims at its token's position (2.5.2).  Readings: no norm on
     c^Q and none and no rotation on q^I (the pages give neither; the
-    indexer keys have neither either).  Returns (c^Q, q, q^I, w)."""
+    indexer keys have neither either).  With round_mid, c^Q is rounded to
+    bf16 (the activation dtype) before the two up-projections, as a
+    stored low-rank latent is (reading: the latent between the products is
+    stored in the activation dtype, like the group outputs of the output
+    projection).  Returns (c^Q, q, q^I, w)."""
     H = _f64(H)
     T = H.shape[0]
     cQ = matmul(H, WDQ)
+    if round_mid:
+        cQ = round_bf16(cQ)
     qI = matmul(cQ, WIUQ).reshape(T, n_hI, c_I)
     w = matmul(H, Ww)
     q = matmul(cQ, WUQ).reshape(T, n_h, c)

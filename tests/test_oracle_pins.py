@@ -597,6 +597,31 @@ def test_query_rotation_uses_the_token_position():
         assert not np.allclose(qc[0] @ ka, qa[0] @ ka)
 
 
+def test_query_latent_rounding_is_the_only_change():
+    """round_mid rounds c^Q to bf16 before the up-projections and nothing
+    else: with W^DQ the identity and bf16-representable h, c^Q is already a
+    bf16 value and all four outputs are bit-identical; with h off the bf16
+    grid they differ, and equal the chain run on bf16(h W^DQ) by matmuls."""
+    x = _qp_inputs(d=12, d_c=12)
+    x["WDQ"] = np.eye(12)
+    pos = np.array([1, 5, 9, 70, 300])
+    x["H"] = oracle.round_bf16(x["H"])
+    a = _qp(x, pos)
+    b = P.query_proj(x["H"], pos, x["WDQ"], x["WUQ"], x["WIUQ"], x["Ww"], 3, 16, 2, 8, 8,
+                     10000.0, 1e-6, round_mid=True)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+    x2 = _qp_inputs()
+    c = P.query_proj(x2["H"], pos, x2["WDQ"], x2["WUQ"], x2["WIUQ"], x2["Ww"], 3, 16, 2, 8, 8,
+                     10000.0, 1e-6, round_mid=True)
+    d = _qp(x2, pos)
+    assert not np.array_equal(c[2], d[2])
+    cq = oracle.round_bf16(x2["H"] @ x2["WDQ"])
+    np.testing.assert_array_equal(c[0], cq)
+    np.testing.assert_allclose(c[2].reshape(5, -1), cq @ x2["WIUQ"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(c[3], d[3], rtol=0, atol=0)  # w does not see the latent
+
+
 # ------------------------------------------------------------------ MXFP4 ---
 # The indexer's QK path in MXFP4 ("02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文"
 # 3.3); the format is the OCP Microscaling one (tests/golden/e2m1_values.txt).
