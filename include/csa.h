@@ -212,6 +212,42 @@ csa_status csa_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void
                         csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_query_proj: the query side of the layer for R tokens ([N] eq. 13-15
+ * and 18, 2.5.1-2.5.2), the projections that feed csa_index_topk and
+ * csa_attend:
+ *   c^Q = h W^{DQ}                 (eq. 13, d -> d_c; the low-rank latent,
+ *                                   stored bf16 and read back as bf16)
+ *   w   = h W^w                    (eq. 15, n_hI fp32 head weights)
+ *   q^I = c^Q W^{IUQ}              (eq. 14, n_hI heads of c_I; no norm, no
+ *                                   RoPE, like the indexer keys)
+ *   q   = RoPE_t(RMSNorm(c^Q W^{UQ})) per head (eq. 18; unit-gain RMSNorm
+ *                                   over each head's c values, RoPE at the
+ *                                   token's position t on the last
+ *                                   rope_dims, interleaved pairs)
+ * bf16 only (tensor cores; CSA_ERR_UNSUPPORTED otherwise); 16 tokens a
+ * triple of launches (weights streamed once per 16 tokens: the decode form).
+ *   WDQ [d][d_c], Ww [d][n_hI], WUQ [d_c][n_h c], WIUQ [d_c][n_hI c_I] bf16
+ *       (row-major, x W form) -> packed, csa_query_proj_packed_bytes() bytes
+ *       from csa_query_proj_pack (K-major rows, zero-padded)
+ *   H   [R][d] bf16, pos [R] int32 token positions
+ *   cQ  [R][d_c] bf16, q [R][n_h][c] bf16, qI [R][n_hI][c_I] bf16,
+ *   w   [R][n_hI] fp32            outputs (caller-owned)
+ *   workspace  csa_query_proj_workspace_bytes() bytes (q before its norm,
+ *              fp32)
+ * Shapes: d % 64 == 0, d_c % 64 == 0, c % 4 == 0; pointers 16-byte
+ * aligned.  Argument errors as for every call.
+ * ------------------------------------------------------------------------- */
+size_t csa_query_proj_packed_bytes(const csa_params* p, int d, int d_c);
+csa_status csa_query_proj_pack(const csa_params* p, int d, int d_c, const void* WDQ,
+                               const void* Ww, const void* WUQ, const void* WIUQ,
+                               void* packed, csa_stream_t stream);
+size_t csa_query_proj_workspace_bytes(const csa_params* p, int R, int d, int d_c);
+csa_status csa_query_proj(const csa_params* p, int R, int d, int d_c, const void* H,
+                          const int32_t* pos, const void* packed, void* cQ, void* q,
+                          void* qI, float* w, void* workspace, size_t ws_bytes,
+                          csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * csa_index_topk: Lightning-Indexer scores and top-k selection ([N] eq. 16-17,
  * [P] 2.2):  I[r][s] = sum_h w[r][h] * ReLU(qI[r][h] . kI[b][s])  for every
  * visible s, then the topk largest.  Ties are broken towards the lower index.

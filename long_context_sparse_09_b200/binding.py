@@ -69,6 +69,11 @@ _SIGS = {
     "csa_out_proj_pack": (C.c_int, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "csa_out_proj_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "csa_out_proj": (C.c_int, [_i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "csa_query_proj_packed_bytes": (_sz, [_P, _i, _i]),
+    "csa_query_proj_pack": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "csa_query_proj_workspace_bytes": (_sz, [_P, _i, _i, _i]),
+    "csa_query_proj": (C.c_int, [_P, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                 _vp]),
     "csa_index_topk_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_noalloc": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
@@ -347,6 +352,48 @@ def csa_out_proj(O, packed, g, d_g, out, workspace=None, stream=None):
     st = lib().csa_out_proj(R, n_h, c, g, d_g, d, _p(O), _p(packed), _p(out), _p(ws), wsb,
                             _stream(stream))
     _check("csa_out_proj", st)
+
+
+# ------------------------------------------------ query-side projections --
+def query_proj_pack(p: CsaParams, WDQ, Ww, WUQ, WIUQ, stream=None) -> torch.Tensor:
+    """WDQ [d][d_c], Ww [d][n_hI], WUQ [d_c][n_h c], WIUQ [d_c][n_hI c_I]
+    (bf16, device) -> the packed buffer for csa_query_proj."""
+    d, d_c = WDQ.shape
+    for t, nm, shp in ((WDQ, "WDQ", (d, d_c)), (Ww, "Ww", (d, p.n_hI)),
+                       (WUQ, "WUQ", (d_c, p.n_h * p.c)), (WIUQ, "WIUQ", (d_c, p.n_hI * p.c_I))):
+        _want(t, torch.bfloat16, nm)
+        if tuple(t.shape) != shp:
+            raise ValueError(f"{nm}: shape {shp} expected, got {tuple(t.shape)}")
+    nbytes = lib().csa_query_proj_packed_bytes(C.byref(p), d, d_c)
+    if nbytes == 0:
+        raise CsaError("csa_query_proj_packed_bytes", 2, "unsupported shapes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=WDQ.device)
+    st = lib().csa_query_proj_pack(C.byref(p), d, d_c, _p(WDQ), _p(Ww), _p(WUQ), _p(WIUQ),
+                                   _p(packed), _stream(stream))
+    _check("csa_query_proj_pack", st)
+    return packed
+
+
+def query_proj_workspace_bytes(p: CsaParams, R, d, d_c) -> int:
+    return lib().csa_query_proj_workspace_bytes(C.byref(p), R, d, d_c)
+
+
+def csa_query_proj(p: CsaParams, H, pos, packed, d_c, cQ, q, qI, w, workspace=None,
+                   stream=None):
+    """H [R][d] bf16 at positions pos [R] -> cQ [R][d_c], q [R][n_h][c],
+    qI [R][n_hI][c_I] (bf16) and w [R][n_hI] (fp32)."""
+    R, d = H.shape
+    _want(H, torch.bfloat16, "H")
+    _want(pos, torch.int32, "pos", R * 4)
+    _want(packed, torch.uint8, "packed", lib().csa_query_proj_packed_bytes(C.byref(p), d, d_c))
+    _want(cQ, torch.bfloat16, "cQ", R * d_c * 2)
+    _want(q, torch.bfloat16, "q", R * p.n_h * p.c * 2)
+    _want(qI, torch.bfloat16, "qI", R * p.n_hI * p.c_I * 2)
+    _want(w, torch.float32, "w", R * p.n_hI * 4)
+    ws, wsb = _ws(query_proj_workspace_bytes(p, R, d, d_c), H.device, workspace)
+    st = lib().csa_query_proj(C.byref(p), R, d, d_c, _p(H), _p(pos), _p(packed), _p(cQ), _p(q),
+                              _p(qI), _p(w), _p(ws), wsb, _stream(stream))
+    _check("csa_query_proj", st)
 
 
 # --------------------------------------------------------- index / top-k --

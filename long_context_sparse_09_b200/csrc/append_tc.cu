@@ -43,12 +43,22 @@ struct ApArgs {
   unsigned* err;
   size_t per_seq;
   int nb, KB, kbs, nsplit, m, overlap, c, cI;
-  // plain-store form: out[b * ld_out + f] for features f < nfeat; the tile
-  // of features f0.. reads the tokens' columns from (f0 / rows_per_group) *
-  // x_per_group on
-  __nv_bfloat16* out;
-  int ld_out, nfeat, rows_per_group, x_per_group;
+  // plain-store form: features f < fsplit go to out[b * ld_out + f],
+  // features fsplit <= f < nfeat to out2[b * ld_out2 + f - fsplit], each as
+  // bf16 or, with out_f32 / out2_f32 set, as fp32; the tile of features
+  // f0.. reads the tokens' columns from (f0 / rows_per_group) * x_per_group on
+  void* out;
+  void* out2;
+  int ld_out, ld_out2, fsplit, out_f32, out2_f32;
+  int nfeat, rows_per_group, x_per_group;
 };
+
+__device__ __forceinline__ void store_feature(void* base, int f32, size_t i, float v) {
+  if (f32)
+    reinterpret_cast<float*>(base)[i] = v;
+  else
+    reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(v);
+}
 
 // kMode 0: the compressor projection and state update; 1: a plain store.
 template <int kMode>
@@ -238,7 +248,11 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
       float v = 0.f;
 #pragma unroll
       for (int r = 0; r < kApMaxSplit; ++r) v += vs[r];
-      a.out[(size_t)b * a.ld_out + tile * 128 + row] = __float2bfloat16_rn(v);
+      const int f = tile * 128 + row;
+      if (f < a.fsplit)
+        store_feature(a.out, a.out_f32, (size_t)b * a.ld_out + f, v);
+      else
+        store_feature(a.out2, a.out2_f32, (size_t)b * a.ld_out2 + (f - a.fsplit), v);
     }
   }
   cluster_sync_all();  // no CTA leaves while its tile may still be read
@@ -458,6 +472,7 @@ csa_status launch_out_proj(int R, int n_h, int c, int g, int d_g, int d, const v
     a.out = y + (size_t)b0 * GD;
     a.ld_out = GD;
     a.nfeat = GD;
+    a.fsplit = GD;
     a.rows_per_group = d_g;
     a.x_per_group = Kg;
     a.KB = Kg / 64;
@@ -473,6 +488,7 @@ csa_status launch_out_proj(int R, int n_h, int c, int g, int d_g, int d, const v
     a.out = res + (size_t)b0 * d;
     a.ld_out = d;
     a.nfeat = d;
+    a.fsplit = d;
     a.rows_per_group = 1 << 30;  // one group
     a.x_per_group = 0;
     a.KB = (GD + 63) / 64;
@@ -480,6 +496,167 @@ csa_status launch_out_proj(int R, int n_h, int c, int g, int d_g, int d, const v
     plan_slices(a, tiles2, 1);
     CSA_LAUNCH(KK_GEMM, st, s = launch_skinny(out_proj_tc, tiles2, tmW, tmX, a, st));
     if (s != CSA_OK) return s;
+  }
+  return last_launch_status();
+}
+
+// ------------------------------------------------ query-side projections --
+// "DeepSeekV4技术报告阅读笔记" eq. 13-15 and 18, 2.5.1-2.5.2.  Packed weights:
+// stage 1 K-major rows [d_c + n_hI][d] (W^{DQ} transposed, then W^w
+// transposed), then, 256-byte aligned, stage 2 K-major rows
+// [n_h c + n_hI c_I][d_c] (W^{UQ} transposed, then W^{IUQ} transposed).
+// Each stage's rows are padded with zero rows to a multiple of 128, so that
+// every 64-row weight box lies inside its tensor map.
+
+struct QpLayout {
+  size_t off2 = 0, total = 0;
+  int n1 = 0, n2 = 0;    // features of the two stages
+  int n1p = 0, n2p = 0;  // rows after padding
+};
+
+static QpLayout qp_layout(const csa_params& p, int d, int d_c) {
+  QpLayout L;
+  L.n1 = d_c + p.n_hI;
+  L.n2 = p.n_h * p.c + p.n_hI * p.c_I;
+  L.n1p = (int)align_up((size_t)L.n1, 128);
+  L.n2p = (int)align_up((size_t)L.n2, 128);
+  L.off2 = align_up((size_t)L.n1p * d * 2, 256);
+  L.total = L.off2 + align_up((size_t)L.n2p * d_c * 2, 256);
+  return L;
+}
+
+size_t query_proj_packed_bytes(const csa_params& p, int d, int d_c) {
+  return qp_layout(p, d, d_c).total;
+}
+
+size_t query_proj_ws_bytes(const csa_params& p, int R) {
+  return align_up((size_t)R * p.n_h * p.c * 4, 256);
+}
+
+csa_status launch_query_proj_pack(const csa_params& p, int d, int d_c, const void* WDQ,
+                                  const void* Ww, const void* WUQ, const void* WIUQ,
+                                  void* packed, cudaStream_t st) {
+  const QpLayout L = qp_layout(p, d, d_c);
+  __nv_bfloat16* s1 = (__nv_bfloat16*)packed;
+  __nv_bfloat16* s2 = (__nv_bfloat16*)((char*)packed + L.off2);
+  auto tr = [&](const void* src, int K, int width, __nv_bfloat16* dst, size_t row0) {
+    const dim3 grid((width + 31) / 32, (K + 31) / 32);
+    CSA_LAUNCH(KK_GEMM, st, transpose_bf16<<<grid, dim3(32, 8), 0, st>>>(
+        (const __nv_bfloat16*)src, K, width, dst, row0));
+  };
+  if (cudaMemsetAsync(packed, 0, L.total, st) != cudaSuccess) return CSA_ERR_CUDA;  // pad rows
+  tr(WDQ, d, d_c, s1, 0);
+  tr(Ww, d, p.n_hI, s1, (size_t)d_c);
+  tr(WUQ, d_c, p.n_h * p.c, s2, 0);
+  tr(WIUQ, d_c, p.n_hI * p.c_I, s2, (size_t)p.n_h * p.c);
+  return last_launch_status();
+}
+
+// Per (token, head) of q: RMSNorm over the c values (unit gain, 2.5.1) and
+// RoPE at the token's position on the last rope_dims (interleaved pairs,
+// 2.5.2), stored as bf16.  One warp per (token, head).
+__global__ void __launch_bounds__(256) query_finish(const float* __restrict__ qraw,
+                                                    const int32_t* __restrict__ pos, int R,
+                                                    int n_h, int c, int rope_dims, float eps,
+                                                    double base,
+                                                    __nv_bfloat16* __restrict__ q) {
+  pdl_wait();
+  const int warp = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp >= R * n_h) return;
+  const int r = warp / n_h;
+  const float* x = qraw + (size_t)warp * c;
+  float ss = 0.f;
+  for (int j = lane * 4; j < c; j += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(x + j);
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+  }
+  ss = warp_sum(ss);
+  const float inv = rsqrtf(ss / (float)c + eps);
+  const int r0 = c - rope_dims;
+  const double t = (double)pos[r];
+  __nv_bfloat16* out = q + (size_t)warp * c;
+  for (int j = lane * 2; j < c; j += 64) {
+    float a = x[j] * inv, b = x[j + 1] * inv;
+    if (j >= r0) {
+      float cs, sn;
+      rope_cs(t, (j - r0) >> 1, rope_dims, base, &cs, &sn);
+      const float a2 = a * cs - b * sn, b2 = a * sn + b * cs;
+      a = a2;
+      b = b2;
+    }
+    *reinterpret_cast<__nv_bfloat162*>(out + j) = __floats2bfloat162_rn(a, b);
+  }
+}
+
+// c^Q, w (stage 1) and q, q^I (stage 2 and the finish), 16 tokens a triple
+// of launches
+csa_status launch_query_proj(const csa_params& p, int R, int d, int d_c, const void* H,
+                             const int32_t* pos, const void* packed, void* cQ, void* q,
+                             void* qI, float* w, void* ws, cudaStream_t st) {
+  if (!tma_available()) return CSA_ERR_UNSUPPORTED;
+  if (!set_kernel_smem((const void*)out_proj_tc, kApSmem)) return CSA_ERR_CUDA;
+  unsigned* err = device_error_word();
+  if (err == nullptr) return CSA_ERR_CUDA;
+  const QpLayout L = qp_layout(p, d, d_c);
+  const __nv_bfloat16* w1 = (const __nv_bfloat16*)packed;
+  const __nv_bfloat16* w2 = (const __nv_bfloat16*)((const char*)packed + L.off2);
+  const __nv_bfloat16* h = (const __nv_bfloat16*)H;
+  __nv_bfloat16* cq = (__nv_bfloat16*)cQ;
+  float* qraw = (float*)ws;
+  const int nq = p.n_h * p.c;
+  for (int b0 = 0; b0 < R; b0 += kApN) {
+    const int nb = R - b0 < kApN ? R - b0 : kApN;
+    ApArgs a = {};
+    a.err = err;
+    a.nb = nb;
+    a.rows_per_group = 1 << 30;  // one group: every tile reads the tokens from column 0
+    CUtensorMap tmW, tmX;
+    // stage 1: [c^Q | w] = h [W^{DQ} | W^w]
+    if (!make_tmap_bf16(&tmW, w1, (uint64_t)L.n1p, (uint64_t)d, 64)) return CSA_ERR_CUDA;
+    if (!make_tmap_bf16(&tmX, h + (size_t)b0 * d, (uint64_t)nb, (uint64_t)d, kApN))
+      return CSA_ERR_CUDA;
+    a.out = cq + (size_t)b0 * d_c;
+    a.ld_out = d_c;
+    a.out_f32 = 0;
+    a.out2 = w + (size_t)b0 * p.n_hI;
+    a.ld_out2 = p.n_hI;
+    a.out2_f32 = 1;
+    a.fsplit = d_c;
+    a.nfeat = L.n1;
+    a.KB = d / 64;
+    const int tiles1 = (L.n1 + 127) / 128;
+    plan_slices(a, tiles1, 1);
+    csa_status s;
+    CSA_LAUNCH(KK_GEMM, st, s = launch_skinny(out_proj_tc, tiles1, tmW, tmX, a, st));
+    if (s != CSA_OK) return s;
+    // stage 2: [q (fp32, before the norm) | q^I] = c^Q [W^{UQ} | W^{IUQ}]
+    if (!make_tmap_bf16(&tmW, w2, (uint64_t)L.n2p, (uint64_t)d_c, 64)) return CSA_ERR_CUDA;
+    if (!make_tmap_bf16(&tmX, cq + (size_t)b0 * d_c, (uint64_t)nb, (uint64_t)d_c, kApN))
+      return CSA_ERR_CUDA;
+    a.out = qraw + (size_t)b0 * nq;
+    a.ld_out = nq;
+    a.out_f32 = 1;
+    a.out2 = (__nv_bfloat16*)qI + (size_t)b0 * p.n_hI * p.c_I;
+    a.ld_out2 = p.n_hI * p.c_I;
+    a.out2_f32 = 0;
+    a.fsplit = nq;
+    a.nfeat = L.n2;
+    a.KB = d_c / 64;
+    const int tiles2 = (L.n2 + 127) / 128;
+    plan_slices(a, tiles2, 1);
+    CSA_LAUNCH(KK_GEMM, st, s = launch_skinny(out_proj_tc, tiles2, tmW, tmX, a, st));
+    if (s != CSA_OK) return s;
+    // per-head RMSNorm and RoPE of q
+    const int warps = nb * p.n_h;
+    cudaError_t e = cudaSuccess;
+    CSA_LAUNCH(KK_FOLD, st,
+               e = launch_maybe_pdl(kPdlAppend, query_finish, dim3((warps + 7) / 8), dim3(256),
+                                    (size_t)0, st, (const float*)(qraw + (size_t)b0 * nq),
+                                    pos + b0, nb, p.n_h, p.c, p.rope_dims, p.rms_eps,
+                                    (double)p.rope_base,
+                                    (__nv_bfloat16*)q + (size_t)b0 * nq));
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
   return last_launch_status();
 }

@@ -284,6 +284,51 @@ csa_status csa_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void
   return launch_out_proj(R, n_h, c, g, d_g, d, O, packed, out, workspace, S(stream));
 }
 
+// ------------------------------------------------- query-side projections --
+static csa_status check_query_proj(const csa_params* p, int d, int d_c) {
+  csa_status st = check_params(p, true);
+  if (st != CSA_OK) return st;
+  if (d <= 0 || d_c <= 0) return CSA_ERR_SHAPE;
+  if (p->act != CSA_BF16) return CSA_ERR_UNSUPPORTED;
+  if (d % 64 != 0 || d_c % 64 != 0 || p->c % 4 != 0) return CSA_ERR_SHAPE;
+  return CSA_OK;
+}
+
+size_t csa_query_proj_packed_bytes(const csa_params* p, int d, int d_c) {
+  if (check_query_proj(p, d, d_c) != CSA_OK) return 0;
+  return query_proj_packed_bytes(*p, d, d_c);
+}
+
+csa_status csa_query_proj_pack(const csa_params* p, int d, int d_c, const void* WDQ,
+                               const void* Ww, const void* WUQ, const void* WIUQ, void* packed,
+                               csa_stream_t stream) {
+  csa_status st = check_query_proj(p, d, d_c);
+  if (st != CSA_OK) return st;
+  if (!WDQ || !Ww || !WUQ || !WIUQ || !packed) return CSA_ERR_ARG;
+  if (!aligned16(packed)) return CSA_ERR_ALIGN;
+  return launch_query_proj_pack(*p, d, d_c, WDQ, Ww, WUQ, WIUQ, packed, S(stream));
+}
+
+size_t csa_query_proj_workspace_bytes(const csa_params* p, int R, int d, int d_c) {
+  if (R <= 0 || check_query_proj(p, d, d_c) != CSA_OK) return 0;
+  return query_proj_ws_bytes(*p, R);
+}
+
+csa_status csa_query_proj(const csa_params* p, int R, int d, int d_c, const void* H,
+                          const int32_t* pos, const void* packed, void* cQ, void* q, void* qI,
+                          float* w, void* workspace, size_t ws_bytes, csa_stream_t stream) {
+  csa_status st = check_query_proj(p, d, d_c);
+  if (st != CSA_OK) return st;
+  if (R <= 0) return CSA_ERR_SHAPE;
+  if (!H || !pos || !packed || !cQ || !q || !qI || !w) return CSA_ERR_ARG;
+  if (!aligned16(H) || !aligned16(packed) || !aligned16(cQ) || !aligned16(q) ||
+      !aligned16(qI) || !aligned16(w))
+    return CSA_ERR_ALIGN;
+  if (workspace == nullptr || ws_bytes < query_proj_ws_bytes(*p, R)) return CSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return CSA_ERR_ALIGN;
+  return launch_query_proj(*p, R, d, d_c, H, pos, packed, cQ, q, qI, w, workspace, S(stream));
+}
+
 // -------------------------------------------------------------- compress --
 size_t csa_compress_workspace_bytes(const csa_params* p, int B, int T, int d) {
   if (check_params(p, p && p->overlap == 1) != CSA_OK || B <= 0 || T <= 0 || d <= 0) return 0;

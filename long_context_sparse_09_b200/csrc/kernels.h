@@ -39,6 +39,15 @@ csa_status launch_out_proj_pack(int n_h, int c, int g, int d_g, int d, const voi
                                 const void* WO, void* packed, cudaStream_t st);
 csa_status launch_out_proj(int R, int n_h, int c, int g, int d_g, int d, const void* O,
                            const void* packed, void* out, void* ws, cudaStream_t st);
+// query-side projections (bf16; tensor cores, 16 tokens a triple of launches)
+size_t query_proj_packed_bytes(const csa_params& p, int d, int d_c);
+size_t query_proj_ws_bytes(const csa_params& p, int R);
+csa_status launch_query_proj_pack(const csa_params& p, int d, int d_c, const void* WDQ,
+                                  const void* Ww, const void* WUQ, const void* WIUQ,
+                                  void* packed, cudaStream_t st);
+csa_status launch_query_proj(const csa_params& p, int R, int d, int d_c, const void* H,
+                             const int32_t* pos, const void* packed, void* cQ, void* q,
+                             void* qI, float* w, void* ws, cudaStream_t st);
 // decode append, tensor-core projection (bf16, at most 16 tokens a launch)
 bool append_tc_supported(const csa_params& p, int nb);
 csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, int nb, int d,

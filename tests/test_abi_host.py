@@ -340,3 +340,56 @@ def test_noalloc_scratch_bound_is_the_workspace_size(lib):
     st_hi = lib.csa_index_topk_noalloc(C.byref(p), 4, 1, None, fake, fake, fake, hi, fake,
                                        None, None)
     assert st_lo in (1, 5) and st_hi == 8, (lo, hi, st_lo, st_hi)
+
+
+def test_query_proj_sizes_and_argument_errors(lib):
+    wl = WORKLOADS["pro_csa_decode_1m"]
+    p = bd.params_for(wl)
+    d, d_c = wl.d, wl.d_c
+    n1 = -(-(d_c + wl.n_hI) // 128) * 128
+    n2 = -(-(wl.n_h * wl.c + wl.n_hI * wl.c_I) // 128) * 128
+    assert lib.csa_query_proj_packed_bytes(C.byref(p), d, d_c) == n1 * d * 2 + n2 * d_c * 2
+    assert lib.csa_query_proj_workspace_bytes(C.byref(p), 4, d, d_c) == 4 * wl.n_h * wl.c * 4
+    assert lib.csa_query_proj_packed_bytes(C.byref(p), d + 32, d_c) == 0  # d % 64
+    pf = bd.params_for(WORKLOADS["tiny_csa_prefill_f32"])
+    assert lib.csa_query_proj_packed_bytes(C.byref(pf), 512, 128) == 0  # fp32: unsupported
+    fake = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    ws = 1 << 30
+    assert lib.csa_query_proj(C.byref(p), 4, d, d_c, fake, None, fake, fake, fake, fake, fake,
+                              fake, ws, None) == 1
+    assert lib.csa_query_proj(C.byref(p), 0, d, d_c, fake, fake, fake, fake, fake, fake, fake,
+                              fake, ws, None) == 2
+    assert lib.csa_query_proj(C.byref(p), 4, d, d_c, fake, fake, fake, fake,
+                              C.c_void_p((1 << 20) + 4), fake, fake, fake, ws, None) == 3
+    assert lib.csa_query_proj(C.byref(p), 4, d, d_c, fake, fake, fake, fake, fake, fake, fake,
+                              fake, 16, None) == 8
+    assert lib.csa_query_proj(C.byref(pf), 4, 512, 128, fake, fake, fake, fake, fake, fake,
+                              fake, fake, ws, None) == 7
+
+
+def test_binding_checks_query_proj_tensors(lib):
+    import torch
+    wl = WORKLOADS["flash_csa_decode_64k"].with_(d=256, d_c=128, n_h=4, c=128, rope_dims=32,
+                                                 n_hI=4, c_I=64)
+    p = bd.params_for(wl)
+    R = 3
+    H = torch.zeros(R, 256, dtype=torch.bfloat16)
+    pos = torch.zeros(R, dtype=torch.int32)
+    packed = torch.zeros(lib.csa_query_proj_packed_bytes(C.byref(p), 256, 128), dtype=torch.uint8)
+    cQ = torch.zeros(R, 128, dtype=torch.bfloat16)
+    q = torch.zeros(R, 4, 128, dtype=torch.bfloat16)
+    qI = torch.zeros(R, 4, 64, dtype=torch.bfloat16)
+    w = torch.zeros(R, 4)
+    with pytest.raises(ValueError, match=r"^H:"):
+        bd.csa_query_proj(p, H.float(), pos, packed, 128, cQ, q, qI, w)
+    with pytest.raises(ValueError, match=r"^q:"):
+        bd.csa_query_proj(p, H, pos, packed, 128, cQ, q[:2], qI, w)
+    with pytest.raises(ValueError, match=r"^w:"):
+        bd.csa_query_proj(p, H, pos, packed, 128, cQ, q, qI, w.to(torch.bfloat16))
+    with pytest.raises(ValueError, match=r"^packed:"):
+        bd.csa_query_proj(p, H, pos, packed[:64], 128, cQ, q, qI, w)
+    with pytest.raises(ValueError, match=r"^WUQ:"):
+        bd.query_proj_pack(p, torch.zeros(256, 128, dtype=torch.bfloat16),
+                           torch.zeros(256, 4, dtype=torch.bfloat16),
+                           torch.zeros(128, 100, dtype=torch.bfloat16),
+                           torch.zeros(128, 256, dtype=torch.bfloat16))
