@@ -290,6 +290,20 @@ class DecodeStep:
         del gr, packed
         return e0.elapsed_time(e1) / (reps * per_graph), nbytes
 
+    def step_work(self):
+        """("hbm", algorithmic bytes of one step): every cache byte the step
+        must read once (indexer keys, the selected entries, the window rows;
+        all visible entries for HCA) plus the queries and the outputs."""
+        wl, B, N = self.wl, self.wl.B, self.N
+        row = synth.kv_record_bytes(wl) + (4 if wl.kv == "fp8mix" else 0)
+        qo = 2 * wl.n_h * wl.c * 2 + 4
+        if wl.variant == "csa":
+            per_q = (N * wl.c_I * 2 + wl.n_hI * (wl.c_I * 2 + 4) + wl.topk * row
+                     + wl.n_win * row + qo)
+        else:
+            per_q = (N + wl.n_win) * row + qo
+        return "hbm", B * per_q
+
     def dominant(self):
         """(kernel kind, algorithmic bytes per launch, source file)."""
         wl, B, N = self.wl, self.wl.B, self.N
@@ -411,7 +425,8 @@ class PrefillStep:
         H = i["H"][0, :n_tok].cpu()
         t0 = time.perf_counter()
         P.compress_seq(wl, W, H)
-        t_comp = (time.perf_counter() - t0) / n_tok
+        s_comp = time.perf_counter() - t0
+        t_comp = s_comp / n_tok
         st = synth._Streams(wl.seed + 99, "cpu")
         kv = P.cache_values(*synth.cache_rows(wl, st, "bkv", (), nE), wl.kv, wl.c, wl.rope_dims)
         win = P.cache_values(*synth.cache_rows(wl, st, "bwin", (), T), wl.kv, wl.c, wl.rope_dims)
@@ -425,10 +440,15 @@ class PrefillStep:
         t0 = time.perf_counter()
         idx, _, _, _ = P.select(wl, t0s, qI, w, kI)
         P.attend_wl(wl, t0s, q, idx, kv, win, 0, sink)
-        t_query = (time.perf_counter() - t0) / n_q
-        secs = t_comp + t_query  # per token
-        return 1, secs, (f"compression of {n_tok} tokens and index/top-k/attention of {n_q} "
-                         f"queries spread over {T}; tokens/s extrapolated from the time per token")
+        s_query = time.perf_counter() - t0
+        t_query = s_query / n_q
+        per_token = t_comp + t_query
+        measured = s_comp + s_query
+        # (tokens' worth of work measured, seconds measured): their ratio is
+        # the extrapolated rate 1 / (t_comp + t_query)
+        return measured / per_token, measured, (
+            f"compression of {n_tok} tokens and index/top-k/attention of {n_q} queries spread "
+            f"over {T}; tokens/s extrapolated from the time per token of the two parts")
 
     def units(self):
         return self.wl.B * self.wl.T  # tokens per step
@@ -444,9 +464,159 @@ class PrefillStep:
         attn = 4.0 * keys * wl.n_h * wl.c
         return comp, index, attn
 
+    def step_work(self):
+        """("tensor", algorithmic FLOPs of one step)."""
+        return "tensor", sum(self.flops())
+
     def dominant(self):
         comp, index, attn = self.flops()
         return "attend", attn, "attend_tc.cu", "tensor"
+
+
+# --------------------------------------------------------------- measure --
+# workloads measured after the default one, as sub-objects of its line
+OTHER_WORKLOADS = ("flash_csa_prefill_32k", "hca_decode_1m", "flash_csa_decode_64k")
+
+
+def time_step(step, steps, warmup, world, stream):
+    """Device time of one step.  The timed step is a CUDA-graph replay of
+    the library calls (launch overhead out of the way); `steps` replays sit
+    between CUDA events on the launching stream, barriers and a synchronize
+    on both sides, max over ranks.  A second graph of the same step carries
+    the per-kernel event pairs of the library's profiler; it is replayed as
+    many times right after the timed region and gives the kernel times (its
+    event nodes would otherwise add to the step time)."""
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    assert bd.device_status() == 0, "device error word set during warm-up"
+    l0 = bd.kernel_launches()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step.run()
+    launches_per_step = bd.kernel_launches() - l0
+    bd.profile_enable(True)
+    step.run()
+    torch.cuda.synchronize()
+    bd.profile_collect()  # warms the event pool so capture creates no events
+    graph_prof = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_prof):
+        step.run()
+    bd.profile_enable(False)
+    for _ in range(warmup):
+        graph.replay()
+        graph_prof.replay()
+    torch.cuda.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    ms = e0.elapsed_time(e1) / steps
+    e0.record(stream)
+    for _ in range(steps):
+        graph_prof.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof_ms = e0.elapsed_time(e1) / steps
+    prof = bd.profile_collect()  # per-kernel device time of the last replay
+    assert bd.device_status() == 0, "device error word set during the timed steps"
+    del graph, graph_prof
+    return {"ms": _max_over_ranks(ms, world), "prof_ms": prof_ms, "prof": prof,
+            "launches_per_step": launches_per_step}
+
+
+def rooflines(step, prof, ms):
+    """(dominant-kernel roofline, per-kernel split, whole-step roofline)."""
+    wl = step.wl
+    kind, nbytes, src, bound = step.dominant()
+    kms, kcnt = prof.get(kind, (0.0, 0))  # one replay: kcnt launches of the kernel
+    hbm, tfl, peak_src = _peaks()
+    roof = None
+    if kcnt and bound == "hbm":
+        per_launch_ms = kms / kcnt
+        achieved = nbytes / (per_launch_ms / 1e3) / 1e9
+        tr = NCU_TRAFFIC.get((kind, wl.name))
+        traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
+        roof = {"bound": bound, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": kind,
+                "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
+                "peak_source": peak_src}
+    elif kcnt:
+        per_launch_ms = kms / kcnt
+        achieved = nbytes / (per_launch_ms / 1e3) / 1e12
+        tr = NCU_TRAFFIC.get((kind, wl.name))
+        traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tfl, "unit": "TFLOP/s",
+                "frac": round(achieved / tfl, 4), "traffic": traffic, "kernel": kind,
+                "algorithmic_flops_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
+                "peak_source": peak_src}
+    kernels = {k: {"ms_per_step": round(v[0], 5), "launches": v[1],
+                   "share": round(v[0] / max(sum(x[0] for x in prof.values()), 1e-12), 4)}
+               for k, v in prof.items() if v[1]}
+    sbound, work = step.step_work()
+    if sbound == "hbm":
+        t_roof = work / (hbm * 1e9) * 1e3
+        step_roof = {"bound": "hbm", "algorithmic_bytes_per_step": work, "peak": hbm,
+                     "unit": "GB/s", "achieved": round(work / (ms / 1e3) / 1e9, 1)}
+    else:
+        t_roof = work / (tfl * 1e12) * 1e3
+        step_roof = {"bound": "tensor", "algorithmic_flops_per_step": work, "peak": tfl,
+                     "unit": "TFLOP/s", "achieved": round(work / (ms / 1e3) / 1e12, 1)}
+    step_roof.update({"roofline_ms": round(t_roof, 5), "frac": round(t_roof / ms, 4),
+                      "peak_source": peak_src})
+    return roof, kernels, step_roof
+
+
+def cpu_baseline(step, target_s):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    step (decode: the step's queries, repeated until about target_s of
+    oracle time; prefill: the sample PrefillStep.cpu_baseline describes)."""
+    import oracle
+    wl = step.wl
+    unit = "query-tok/s" if wl.mode == "decode" else "tok/s"
+    if wl.mode == "decode":
+        nq, secs, sample, passes = 0, 0.0, "", 0
+        while secs < target_s and passes < 64:
+            n1, s1, sample = step.cpu_baseline()
+            nq, secs, passes = nq + n1, secs + s1, passes + 1
+        sample = f"{sample}, {passes} passes"
+    else:
+        nq, secs, sample = step.cpu_baseline()
+    return {"value": round(nq / secs, 4), "unit": unit, "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": sample, "seconds": round(secs, 4)}
+
+
+def measure_other(wl, args, world, rank, dev, stream):
+    """One more workload of the metric, timed like the default one (graph
+    replays between CUDA events, per-kernel split, rooflines, clocks, the
+    oracle on a bounded sample); returns its sub-object."""
+    step = (DecodeStep if wl.mode == "decode" else PrefillStep)(wl, dev, seed_offset=rank)
+    steps = args.steps if wl.mode == "decode" else max(3, min(args.steps, 20))
+    clocks = ClockSampler(dev)
+    time.sleep(0.15)
+    t = time_step(step, steps, max(3, args.warmup), world, stream)
+    clk = clocks.stop()
+    roof, kernels, step_roof = rooflines(step, t["prof"], t["ms"])
+    unit = "query-tok/s" if wl.mode == "decode" else "tok/s"
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(step, 5.0)
+    out = {"value": round(step.units() * world / (t["ms"] / 1e3), 2), "unit": unit,
+           "ms_per_step": round(t["ms"], 5), "steps": steps,
+           "config": {"batch_per_gpu": wl.B, "context": wl.T, "m": wl.m, "topk": wl.topk,
+                      "n_h": wl.n_h, "c": wl.c, "kv_format": wl.kv, "n_win": wl.n_win,
+                      "d": wl.d, "dtype": wl.act},
+           "gpu_launches": t["launches_per_step"] * steps,
+           "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
+           "ms_per_step_with_events": round(t["prof_ms"], 5),
+           "cpu_baseline": cpu, "clocks": clk}
+    del step
+    return out
 
 
 # -------------------------------------------------------------------- main --
@@ -464,57 +634,14 @@ def run_ours(args, world, rank, local):
     torch.manual_seed(0)
     step = (DecodeStep if wl.mode == "decode" else PrefillStep)(wl, dev, seed_offset=rank)
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-    assert bd.device_status() == 0, "device error word set during warm-up"
-    # The timed step is a CUDA-graph replay of the library calls (launch
-    # overhead out of the way).  A second graph of the same step carries the
-    # per-kernel event pairs of the library's profiler; it is replayed as
-    # many times right after the timed region and gives the kernel times
-    # (its event nodes would otherwise add to the step time).
-    l0 = bd.kernel_launches()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step.run()
-    launches_per_step = bd.kernel_launches() - l0
-    bd.profile_enable(True)
-    step.run()
-    torch.cuda.synchronize()
-    bd.profile_collect()  # warms the event pool so capture creates no events
-    graph_prof = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_prof):
-        step.run()
-    bd.profile_enable(False)
-    for _ in range(args.warmup):
-        graph.replay()
-        graph_prof.replay()
-    torch.cuda.synchronize()
     clocks = ClockSampler(dev)
     time.sleep(0.15)
-    _barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    _barrier(world)
-    ms = e0.elapsed_time(e1) / args.steps
-    e0.record(stream)
-    for _ in range(args.steps):
-        graph_prof.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    prof_ms = e0.elapsed_time(e1) / args.steps
-    prof = bd.profile_collect()  # per-kernel device time of the last replay
+    t = time_step(step, args.steps, args.warmup, world, stream)
     clk = clocks.stop()
-    launches = launches_per_step * args.steps
-    ms = _max_over_ranks(ms, world)
+    ms, prof_ms, prof = t["ms"], t["prof_ms"], t["prof"]
+    launches = t["launches_per_step"] * args.steps
     units = step.units() * world
     value = units / (ms / 1e3)
-    assert bd.device_status() == 0, "device error word set during the timed steps"
 
     # end to end through the public API: every step copies its inputs from
     # pinned host memory to the device, runs the library calls eagerly and
@@ -580,6 +707,7 @@ def run_ours(args, world, rank, local):
         e2e_step(k)
     torch.cuda.synchronize()
     _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     arm()  # the first copies start inside the timed region
     for k in range(args.steps):
@@ -609,47 +737,23 @@ def run_ours(args, world, rank, local):
                     "weight_bytes": o_bytes,
                     "hbm_frac": round(o_bytes / (o_ms / 1e3) / 1e9 / hbm0, 4)}
 
-    kind, nbytes, src, bound = step.dominant()
-    kms, kcnt = prof.get(kind, (0.0, 0))  # one replay: kcnt launches of the kernel
-    hbm, tfl, peak_src = _peaks()
-    roof = None
-    if kcnt and bound == "hbm":
-        per_launch_ms = kms / kcnt
-        achieved = nbytes / (per_launch_ms / 1e3) / 1e9
-        tr = NCU_TRAFFIC.get((kind, wl.name))
-        traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
-        roof = {"bound": bound, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": traffic, "kernel": kind,
-                "algorithmic_bytes_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
-                "peak_source": peak_src}
-    elif kcnt:
-        per_launch_ms = kms / kcnt
-        achieved = nbytes / (per_launch_ms / 1e3) / 1e12
-        tr = NCU_TRAFFIC.get((kind, wl.name))
-        traffic = tr[0] if tr and tr[1] == _src_hash(src) else None
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tfl, "unit": "TFLOP/s",
-                "frac": round(achieved / tfl, 4), "traffic": traffic, "kernel": kind,
-                "algorithmic_flops_per_launch": nbytes, "launch_ms": round(per_launch_ms, 5),
-                "peak_source": peak_src}
-    kernels = {k: {"ms_per_step": round(v[0], 5), "launches": v[1],
-                   "share": round(v[0] / max(sum(x[0] for x in prof.values()), 1e-12), 4)}
-               for k, v in prof.items() if v[1]}
-
+    roof, kernels, step_roof = rooflines(step, prof, ms)
+    entries = getattr(step, "N", getattr(step, "nE", 0))
     unit = "query-tok/s" if wl.mode == "decode" else "tok/s"
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(step, "cpu_baseline"):
-        import oracle
-        if wl.mode == "decode":
-            # the step's queries, repeated until about 10 s of oracle time
-            nq, secs, sample, passes = 0, 0.0, "", 0
-            while secs < 10.0 and passes < 64:
-                n1, s1, sample = step.cpu_baseline()
-                nq, secs, passes = nq + n1, secs + s1, passes + 1
-            sample = f"{sample}, {passes} passes"
-        else:
-            nq, secs, sample = step.cpu_baseline()
-        cpu = {"value": round(nq / secs, 4), "unit": unit, "cores": oracle.num_threads(),
-               "kind": "oracle", "sample": sample, "seconds": round(secs, 4)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(step, 10.0)
+
+    # the other workloads of the metric (prefill tokens/s, the HCA and the
+    # V4-Flash decode), each timed the same way, as sub-objects of the line
+    others = {}
+    if args.workload == DEFAULT_BENCH and not args.batch and not args.context and \
+            not args.no_others:
+        del step, dev_flat, dev_in, dev_out
+        torch.cuda.empty_cache()
+        for name in OTHER_WORKLOADS:
+            others[name] = measure_other(WORKLOADS[name], args, world, rank, dev, stream)
+            torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
@@ -658,11 +762,11 @@ def run_ours(args, world, rank, local):
             "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.T,
-                       "entries_per_seq": getattr(step, "N", getattr(step, "nE", 0)),
+                       "entries_per_seq": entries,
                        "m": wl.m, "topk": wl.topk,
                        "n_h": wl.n_h, "c": wl.c, "kv_format": wl.kv, "n_win": wl.n_win,
                        "l2": "inputs larger than L2 (cache streamed every step)"},
-            "e2e": {"value": round(step.units() * world / (e2e_ms / 1e3), 2),
+            "e2e": {"value": round(units / (e2e_ms / 1e3), 2),
                     "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 5)},
             "gpu_launches": launches,
@@ -671,10 +775,12 @@ def run_ours(args, world, rank, local):
             "ms_per_step_with_events": round(prof_ms, 5),
             "roofline": roof,
             "kernels": kernels,
+            "step_roofline": step_roof,
             "decode_append": append,
             "out_proj": out_proj,
             "cpu_baseline": cpu,
             "clocks": clk,
+            "workloads": others,
         }
         print(json.dumps(line), flush=True)
 
@@ -771,6 +877,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_BENCH, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-others", action="store_true",
+                    help="time the named workload only (no prefill / HCA / Flash sub-objects)")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (profiling)")
     ap.add_argument("--context", type=int, default=0, help="override context length (profiling)")
     args = ap.parse_args()
