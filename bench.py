@@ -134,16 +134,22 @@ def _max_over_ranks(x, world):
 
 # --------------------------------------------------------------- workloads --
 class DecodeStep:
-    """Resident cache + one query per sequence; a step = index/top-k + attend."""
+    """Resident cache + one query per sequence; a step = index/top-k + attend.
+    With fp4, the indexer keys are held in MXFP4 (quantised once from the
+    same bf16 keys; the cache is resident state) and the step scores them
+    with csa_index_topk_mxfp4."""
 
-    def __init__(self, wl, device, seed_offset=0):
+    def __init__(self, wl, device, seed_offset=0, fp4=False):
         self.wl = wl
+        self.fp4 = fp4
         self.p = bd.params_for(wl)
         inp = synth.decode_inputs(wl.with_(seed=wl.seed + D.seed_offset(seed_offset)),
                                   device=device)
         self.inp = inp
         B, N = wl.B, inp["N"]
         self.N = N
+        if fp4:
+            self.kcodes, self.kscales = bd.mxfp4_quantize(inp["kI"])
         self.out = torch.empty(B, wl.n_h, wl.c, dtype=torch.bfloat16, device=device)
         if wl.variant == "csa":
             self.idx = torch.empty(B, wl.topk, dtype=torch.int32, device=device)
@@ -158,9 +164,14 @@ class DecodeStep:
         out = self.out if out is None else out
         q_pos = i["q_pos"] if q_pos is None else q_pos
         if wl.variant == "csa":
-            bd.csa_index_topk(self.p, q_pos, i["qI"] if qI is None else qI,
-                              i["w"] if w is None else w, i["kI"], self.idx,
-                              workspace=self.ws_i)
+            if self.fp4:
+                bd.csa_index_topk_mxfp4(self.p, q_pos, i["qI"] if qI is None else qI,
+                                        i["w"] if w is None else w, self.kcodes, self.kscales,
+                                        self.idx, workspace=self.ws_i)
+            else:
+                bd.csa_index_topk(self.p, q_pos, i["qI"] if qI is None else qI,
+                                  i["w"] if w is None else w, i["kI"], self.idx,
+                                  workspace=self.ws_i)
             bd.csa_attend(self.p, q_pos, q, self.idx, i["ckv"], i["ckv_scale"], i["win"],
                           i["win_scale"], i["win_pos0"], i["sink"], out,
                           workspace=self.ws_a)
@@ -251,6 +262,69 @@ class DecodeStep:
         del g, gp, packs
         return ms, wbytes, split
 
+    def recall_vs_bf16(self):
+        """Per query, the fraction of the bf16 indexer's selection that this
+        step's MXFP4 selection also makes (KV recall, plain set arithmetic)."""
+        i, wl = self.inp, self.wl
+        self.run()
+        got = self.idx.cpu().numpy()
+        ref = torch.empty_like(self.idx)
+        bd.csa_index_topk(self.p, i["q_pos"], i["qI"], i["w"], i["kI"], ref, workspace=self.ws_i)
+        ref = ref.cpu().numpy()
+        out = []
+        for a, b in zip(got, ref):
+            sb = set(int(x) for x in b if x >= 0)
+            out.append(len(sb & set(int(x) for x in a if x >= 0)) / max(len(sb), 1))
+        return out
+
+    def time_query_proj(self, steps, stream):
+        """Device time of csa_query_proj for the step's tokens at the
+        workload's d, d_c and head shapes (random bf16 weights N(0, 1/fan_in);
+        graph replays of one call per copy of the packed weights, the copies
+        together at least twice the L2, so every call streams its weights from
+        HBM).  Returns (ms per call, packed weight bytes)."""
+        wl, dev = self.wl, self.out.device
+        B, d, d_c = wl.B, wl.d, wl.d_c
+        gen = torch.Generator(device=dev).manual_seed(wl.seed + 13)
+        rnd = lambda *sh: (torch.randn(*sh, device=dev, generator=gen) / sh[0] ** 0.5).to(
+            torch.bfloat16)
+        packed0 = bd.query_proj_pack(self.p, rnd(d, d_c), rnd(d, wl.n_hI),
+                                     rnd(d_c, wl.n_h * wl.c), rnd(d_c, wl.n_hI * wl.c_I))
+        nbytes = packed0.numel()
+        ncopy = max(2, min(16, -(-2 * L2_BYTES // nbytes)))
+        packs = [packed0] + [packed0.clone() for _ in range(ncopy - 1)]
+        H = torch.randn(B, d, device=dev, generator=gen).to(torch.bfloat16)
+        pos = self.inp["q_pos"]
+        cQ = torch.empty(B, d_c, dtype=torch.bfloat16, device=dev)
+        q = torch.empty(B, wl.n_h, wl.c, dtype=torch.bfloat16, device=dev)
+        qI = torch.empty(B, wl.n_hI, wl.c_I, dtype=torch.bfloat16, device=dev)
+        w = torch.empty(B, wl.n_hI, device=dev)
+        ws = torch.empty(bd.query_proj_workspace_bytes(self.p, B, d, d_c), dtype=torch.uint8,
+                         device=dev)
+
+        def call(pk):
+            bd.csa_query_proj(self.p, H, pos, pk, d_c, cQ, q, qI, w, workspace=ws)
+
+        for pk in packs:
+            call(pk)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for pk in packs:
+                call(pk)
+        for _ in range(3):
+            g.replay()
+        reps = max(1, steps // ncopy)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert bd.device_status() == 0, "device error word set by the query projection"
+        del g, packs
+        return e0.elapsed_time(e1) / (reps * ncopy), nbytes
+
     def time_out_proj(self, steps, stream):
         """Device time of csa_out_proj on the step's attention output (the
         grouped output projection of the workload's g and d_g; graph replays,
@@ -297,8 +371,9 @@ class DecodeStep:
         wl, B, N = self.wl, self.wl.B, self.N
         row = synth.kv_record_bytes(wl) + (4 if wl.kv == "fp8mix" else 0)
         qo = 2 * wl.n_h * wl.c * 2 + 4
+        key_row = (wl.c_I // 2 + wl.c_I // 32) if self.fp4 else wl.c_I * 2
         if wl.variant == "csa":
-            per_q = (N * wl.c_I * 2 + wl.n_hI * (wl.c_I * 2 + 4) + wl.topk * row
+            per_q = (N * key_row + wl.n_hI * (wl.c_I * 2 + 4) + wl.topk * row
                      + wl.n_win * row + qo)
         else:
             per_q = (N + wl.n_win) * row + qo
@@ -308,8 +383,9 @@ class DecodeStep:
         """(kernel kind, algorithmic bytes per launch, source file)."""
         wl, B, N = self.wl, self.wl.B, self.N
         if wl.variant == "csa":
-            nbytes = B * N * wl.c_I * 2 + B * wl.n_hI * (wl.c_I * 2 + 4) + B * 4
-            return "index_scores", nbytes, "index_tc.cu", "hbm"
+            key_row = (wl.c_I // 2 + wl.c_I // 32) if self.fp4 else wl.c_I * 2
+            nbytes = B * N * key_row + B * wl.n_hI * (wl.c_I * 2 + 4) + B * 4
+            return "index_scores", nbytes, "index_fp4.cu" if self.fp4 else "index_tc.cu", "hbm"
         rb = synth.kv_record_bytes(wl)
         nbytes = B * (N + wl.n_win) * rb + 2 * B * wl.n_h * wl.c * 2
         return "attend", nbytes, "attend_tc.cu", "hbm"
@@ -475,7 +551,8 @@ class PrefillStep:
 
 # --------------------------------------------------------------- measure --
 # workloads measured after the default one, as sub-objects of its line
-OTHER_WORKLOADS = ("flash_csa_prefill_32k", "hca_decode_1m", "flash_csa_decode_64k")
+OTHER_WORKLOADS = ("flash_csa_prefill_32k", "hca_decode_1m", "flash_csa_decode_64k",
+                   "pro_csa_decode_1m+mxfp4")
 
 
 def time_step(step, steps, warmup, world, stream):
@@ -591,11 +668,16 @@ def cpu_baseline(step, target_s):
             "kind": "oracle", "sample": sample, "seconds": round(secs, 4)}
 
 
-def measure_other(wl, args, world, rank, dev, stream):
+def measure_other(wl, args, world, rank, dev, stream, fp4=False):
     """One more workload of the metric, timed like the default one (graph
     replays between CUDA events, per-kernel split, rooflines, clocks, the
-    oracle on a bounded sample); returns its sub-object."""
-    step = (DecodeStep if wl.mode == "decode" else PrefillStep)(wl, dev, seed_offset=rank)
+    oracle on a bounded sample); returns its sub-object.  fp4: the decode
+    step with MXFP4 indexer keys, plus its selection's recall of the bf16
+    indexer's selection."""
+    if wl.mode == "decode":
+        step = DecodeStep(wl, dev, seed_offset=rank, fp4=fp4)
+    else:
+        step = PrefillStep(wl, dev, seed_offset=rank)
     steps = args.steps if wl.mode == "decode" else max(3, min(args.steps, 20))
     clocks = ClockSampler(dev)
     time.sleep(0.15)
@@ -604,7 +686,7 @@ def measure_other(wl, args, world, rank, dev, stream):
     roof, kernels, step_roof = rooflines(step, t["prof"], t["ms"])
     unit = "query-tok/s" if wl.mode == "decode" else "tok/s"
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fp4:
         cpu = cpu_baseline(step, 5.0)
     out = {"value": round(step.units() * world / (t["ms"] / 1e3), 2), "unit": unit,
            "ms_per_step": round(t["ms"], 5), "steps": steps,
@@ -615,6 +697,9 @@ def measure_other(wl, args, world, rank, dev, stream):
            "roofline": roof, "step_roofline": step_roof, "kernels": kernels,
            "ms_per_step_with_events": round(t["prof_ms"], 5),
            "cpu_baseline": cpu, "clocks": clk}
+    if fp4:
+        out["indexer_keys"] = "MXFP4 (E2M1 codes + E8M0 block scales, 68 B per entry)"
+        out["recall_vs_bf16_topk"] = [round(r, 4) for r in step.recall_vs_bf16()]
     del step
     return out
 
@@ -737,6 +822,15 @@ def run_ours(args, world, rank, local):
                     "weight_bytes": o_bytes,
                     "hbm_frac": round(o_bytes / (o_ms / 1e3) / 1e9 / hbm0, 4)}
 
+    query_proj = None
+    if wl.mode == "decode" and wl.variant == "csa" and wl.act == "bf16":
+        # the query-side projections before the step (timed on their own)
+        qp_ms, qp_bytes = step.time_query_proj(min(args.steps, 200), stream)
+        hbm0, _, _ = _peaks()
+        query_proj = {"ms_per_call": round(qp_ms, 5), "tokens": wl.B, "d_c": wl.d_c,
+                      "weight_bytes": qp_bytes,
+                      "hbm_frac": round(qp_bytes / (qp_ms / 1e3) / 1e9 / hbm0, 4)}
+
     roof, kernels, step_roof = rooflines(step, prof, ms)
     entries = getattr(step, "N", getattr(step, "nE", 0))
     unit = "query-tok/s" if wl.mode == "decode" else "tok/s"
@@ -752,7 +846,9 @@ def run_ours(args, world, rank, local):
         del step, dev_flat, dev_in, dev_out
         torch.cuda.empty_cache()
         for name in OTHER_WORKLOADS:
-            others[name] = measure_other(WORKLOADS[name], args, world, rank, dev, stream)
+            base, _, variant = name.partition("+")
+            others[name] = measure_other(WORKLOADS[base], args, world, rank, dev, stream,
+                                         fp4=variant == "mxfp4")
             torch.cuda.empty_cache()
 
     if rank == 0:
@@ -778,6 +874,7 @@ def run_ours(args, world, rank, local):
             "step_roofline": step_roof,
             "decode_append": append,
             "out_proj": out_proj,
+            "query_proj": query_proj,
             "cpu_baseline": cpu,
             "clocks": clk,
             "workloads": others,

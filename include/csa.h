@@ -65,6 +65,9 @@ typedef enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_KV_FP8MIX = 2 } csa_dtype;
 #define CSA_DEV_BAD_INDEX 0x1u  /* a top-k index >= the visible entries */
 #define CSA_DEV_BAD_WINDOW 0x2u /* a window token outside the window rows */
 #define CSA_DEV_TIMEOUT 0x4u    /* a bounded wait gave up */
+#define CSA_DEV_RANGE 0x8u      /* an MXFP4 block exponent outside [-23, 13] (the
+                                   MXFP4 indexer's exact range); that block was
+                                   scored with its exponent clamped */
 
 typedef struct {
   int m;          /* tokens per compressed entry (CSA m, HCA m') */
@@ -294,6 +297,39 @@ csa_status csa_index_topk_noalloc(const csa_params* p, int B, int Q,
                                   const float* w, const void* kI, int N,
                                   int32_t* idx_out, float* score_out,
                                   csa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * MXFP4 indexer ("02 · DeepSeek-V4: 压缩注意力撑起 1M 上下文" 3.3: the
+ * indexer's QK path in FP4 with bf16 scores).  Format (OCP Microscaling
+ * MXFP4): a row of `width` values is cut into blocks of 32 consecutive
+ * values; a block's scale is 2^e with e = floor(log2 max|x|) - 2 (-127 for
+ * an all-zero block), stored as one E8M0 byte e + 127; each value is
+ * x / 2^e rounded to the nearest E2M1 value (0, 0.5, 1, 1.5, 2, 3, 4, 6;
+ * ties to the even mantissa; saturating at 6), stored as a 4-bit code (bit
+ * 3 the sign), value 2j in the low nibble of byte j.
+ *
+ * csa_mxfp4_quantize: x [rows][width] bf16 -> codes [rows][width/2] bytes,
+ *   scales [rows][width/32] bytes.  width % 32 == 0; x and codes 16-byte
+ *   aligned.
+ * csa_index_topk_mxfp4: csa_index_topk with the keys in MXFP4 (kI_codes
+ *   [B][N][c_I/2], kI_scales [B][N][c_I/32]) and q^I (bf16, as in
+ *   csa_index_topk) rounded to MXFP4 per head and block inside the call.
+ *   The score of an entry is sum_h w_h ReLU(q^I_h . K^I_s) of the rounded
+ *   values, accumulated in fp32 and rounded to bf16 (returned as fp32
+ *   values); ties are broken towards the lower index as in csa_index_topk.
+ *   Requires act = CSA_BF16, c_I = 128, n_hI a multiple of 16 up to 64
+ *   (else CSA_ERR_UNSUPPORTED).  Block exponents must lie in [-23, 13]
+ *   (block maxima in [2^-21, 2^16)) for exact products; a block outside
+ *   that range with a nonzero code raises CSA_DEV_RANGE.  Workspace:
+ *   csa_index_topk_workspace_bytes().
+ * ------------------------------------------------------------------------- */
+csa_status csa_mxfp4_quantize(int rows, int width, const void* x, void* codes, void* scales,
+                              csa_stream_t stream);
+csa_status csa_index_topk_mxfp4(const csa_params* p, int B, int Q, const int32_t* q_pos,
+                                const void* qI, const float* w, const void* kI_codes,
+                                const void* kI_scales, int N, int32_t* idx_out,
+                                float* score_out, void* workspace, size_t ws_bytes,
+                                csa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * csa_attend: shared-KV multi-query attention of each query over its

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 CSA_F32, CSA_BF16, CSA_KV_FP8MIX = 0, 1, 2
 _DT = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8mix": CSA_KV_FP8MIX}
-DEV_BAD_INDEX, DEV_BAD_WINDOW, DEV_TIMEOUT = 0x1, 0x2, 0x4
+DEV_BAD_INDEX, DEV_BAD_WINDOW, DEV_TIMEOUT, DEV_RANGE = 0x1, 0x2, 0x4, 0x8
 
 
 class CsaError(RuntimeError):
@@ -78,6 +78,9 @@ _SIGS = {
     "csa_index_topk": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "csa_index_topk_noalloc": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
     "csa_diag_bounded_wait": (C.c_int, [C.c_uint64, _i, _vp, _vp]),
+    "csa_mxfp4_quantize": (C.c_int, [_i, _i, _vp, _vp, _vp, _vp]),
+    "csa_index_topk_mxfp4": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp,
+                                       _sz, _vp]),
     "csa_attend_workspace_bytes": (_sz, [_P, _i, _i, _i]),
     "csa_attend": (C.c_int, [_P, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp,
                              _vp, _vp, _sz, _vp]),
@@ -437,6 +440,48 @@ def csa_index_topk_noalloc(p: CsaParams, q_pos, qI, w, kI, idx_out, score_out=No
     st = lib().csa_index_topk_noalloc(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI), N,
                                       _p(idx_out), _p(score_out), _stream(stream))
     _check("csa_index_topk_noalloc", st)
+
+
+# -------------------------------------------------------- MXFP4 indexer --
+def mxfp4_quantize(x, codes=None, scales=None, stream=None):
+    """x [..., width] bf16 (device) -> (codes [..., width/2] uint8, scales
+    [..., width/32] uint8) in the MXFP4 format of include/csa.h."""
+    _want(x, torch.bfloat16, "x")
+    width = x.shape[-1]
+    rows = x.numel() // max(width, 1)
+    lead = tuple(x.shape[:-1])
+    if codes is None:
+        codes = torch.empty(lead + (width // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (width // 32,), dtype=torch.uint8, device=x.device)
+    _want(codes, torch.uint8, "codes", rows * (width // 2))
+    _want(scales, torch.uint8, "scales", rows * (width // 32))
+    _check("csa_mxfp4_quantize", lib().csa_mxfp4_quantize(rows, width, _p(x), _p(codes),
+                                                          _p(scales), _stream(stream)))
+    return codes, scales
+
+
+def csa_index_topk_mxfp4(p: CsaParams, q_pos, qI, w, kI_codes, kI_scales, idx_out,
+                         score_out=None, workspace=None, stream=None):
+    """csa_index_topk with MXFP4 keys: kI_codes [B][N][c_I/2] and kI_scales
+    [B][N][c_I/32] (uint8); q^I is rounded to MXFP4 inside the call and the
+    scores are bf16 values."""
+    B, N = kI_codes.shape[0], kI_codes.shape[1]
+    R = qI.shape[0]
+    Q = _per_seq(R, B, "qI")
+    _want(qI, torch.bfloat16, "qI", R * p.n_hI * p.c_I * 2)
+    _want(w, torch.float32, "w", R * p.n_hI * 4)
+    _want(q_pos, torch.int32, "q_pos", R * 4)
+    _want(kI_codes, torch.uint8, "kI_codes", B * N * p.c_I // 2)
+    _want(kI_scales, torch.uint8, "kI_scales", B * N * p.c_I // 32)
+    _want(idx_out, torch.int32, "idx_out", R * p.topk * 4)
+    if score_out is not None:
+        _want(score_out, torch.float32, "score_out", R * p.topk * 4)
+    ws, wsb = _ws(index_topk_workspace_bytes(p, B, Q, N), qI.device, workspace)
+    st = lib().csa_index_topk_mxfp4(C.byref(p), B, Q, _p(q_pos), _p(qI), _p(w), _p(kI_codes),
+                                    _p(kI_scales), N, _p(idx_out), _p(score_out), _p(ws), wsb,
+                                    _stream(stream))
+    _check("csa_index_topk_mxfp4", st)
 
 
 # ---------------------------------------------------------------- attend --

@@ -888,6 +888,11 @@ static int max_active_clusters(bool fp8, int csize) {
   return cache[dev][fp8][csize];
 }
 
+// most key slices per (query, head block); a build may lower it
+#ifndef CSA_ATTN_MAX_SPLIT
+#define CSA_ATTN_MAX_SPLIT 256
+#endif
+
 void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, int* kps,
                     int* cluster) {
   const int hbn = (p.n_h + 63) / 64;
@@ -897,7 +902,7 @@ void attend_tc_plan(const csa_params& p, int R, int N, bool dense, int* nsplit, 
   const int ntiles = (nk_max + KT - 1) / KT;
   int s = base >= 148 ? 1 : 148 / base;
   if (s > ntiles) s = ntiles;
-  if (s > 256) s = 256;
+  if (s > CSA_ATTN_MAX_SPLIT) s = CSA_ATTN_MAX_SPLIT;
   if (s < 1) s = 1;
   int k = (nk_max + s - 1) / s;
   k = (k + KT - 1) / KT * KT;

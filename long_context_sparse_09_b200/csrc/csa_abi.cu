@@ -440,6 +440,36 @@ csa_status csa_index_topk(const csa_params* p, int B, int Q, const int32_t* q_po
                            S(stream));
 }
 
+// ------------------------------------------------------ MXFP4 indexer --
+csa_status csa_mxfp4_quantize(int rows, int width, const void* x, void* codes, void* scales,
+                              csa_stream_t stream) {
+  if (rows < 0 || width <= 0 || width % 32 != 0) return CSA_ERR_SHAPE;
+  if (rows == 0) return CSA_OK;
+  if (!x || !codes || !scales) return CSA_ERR_ARG;
+  if (!aligned16(x) || !aligned16(codes)) return CSA_ERR_ALIGN;
+  return launch_mxfp4_quantize(rows, width, x, codes, scales, S(stream));
+}
+
+csa_status csa_index_topk_mxfp4(const csa_params* p, int B, int Q, const int32_t* q_pos,
+                                const void* qI, const float* w, const void* kI_codes,
+                                const void* kI_scales, int N, int32_t* idx_out,
+                                float* score_out, void* workspace, size_t ws_bytes,
+                                csa_stream_t stream) {
+  csa_status st = check_params(p, true);
+  if (st != CSA_OK) return st;
+  if (B <= 0 || Q <= 0 || N < 0) return CSA_ERR_SHAPE;
+  if (!index_fp4_supported(*p)) return CSA_ERR_UNSUPPORTED;
+  if (!q_pos || !qI || !w || !idx_out || (N > 0 && (!kI_codes || !kI_scales))) return CSA_ERR_ARG;
+  if (!aligned16(qI) || !aligned16(w) || (kI_codes && !aligned16(kI_codes)) ||
+      (kI_scales && ((uintptr_t)kI_scales & 3u)))
+    return CSA_ERR_ALIGN;
+  const size_t need = index_topk_ws_bytes(*p, B, Q, N);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return CSA_ERR_WORKSPACE;
+  const Mxfp4Keys keys{kI_codes, kI_scales};
+  return launch_index_topk(*p, B, Q, q_pos, qI, w, nullptr, N, idx_out, score_out, workspace,
+                           S(stream), &keys);
+}
+
 // ---------------------------------------------------------------- attend --
 size_t csa_attend_workspace_bytes(const csa_params* p, int B, int Q, int N) {
   if (check_params(p, false) != CSA_OK || B <= 0 || Q <= 0 || N < 0) return 0;

@@ -24,6 +24,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "index_common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -43,10 +44,6 @@ struct IdxTcArgs {
   int stream_keys;    // every key tile is read by one group only: read it evict-first
 };
 
-constexpr int kHistBins = 4096;  // top 12 bits of the order-preserving score key
-
-constexpr int kTileM = 128;
-constexpr int kInlineGroups = 64;  // groups whose tile prefix a CTA computes itself
 constexpr int kMaxAcc = 8;  // TMEM accumulator ring depth (bounded by 512 columns)
 constexpr int kKBlockBytes = kTileM * 128;  // 128 rows x 64 bf16
 
@@ -84,31 +81,6 @@ __global__ void __launch_bounds__(1024) index_plan(const int32_t* __restrict__ q
   }
   if (threadIdx.x == 0) prefix[ngroups] = (int)running;
 }
-
-// Walk of a CTA over its slice of the flat (group, tile) list.
-struct TileCursor {
-  int g, t, left;
-  __device__ void init(const int* prefix, int ngroups, int start, int count) {
-    int lo = 0, hi = ngroups;
-    while (lo < hi) {  // last g with prefix[g] <= start
-      int mid = (lo + hi + 1) >> 1;
-      if (prefix[mid] <= start) lo = mid; else hi = mid - 1;
-    }
-    g = lo;
-    t = start - prefix[g];
-    left = count;
-  }
-  __device__ int tiles(const int* prefix) const { return prefix[g + 1] - prefix[g]; }
-  __device__ bool first(int pos_in_cta) const { return t == 0 || pos_in_cta == 0; }
-  __device__ bool last(const int* prefix) const { return left == 1 || t + 1 == tiles(prefix); }
-  __device__ void next(const int* prefix, int ngroups) {
-    --left;
-    if (++t >= tiles(prefix)) {
-      t = 0;
-      do { ++g; } while (g < ngroups && prefix[g + 1] == prefix[g]);
-    }
-  }
-};
 
 template <int G, int KB, int S, int NE, int NQ>
 __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
@@ -546,6 +518,32 @@ static bool encode_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D byte tensor [rows][cols] (cols contiguous, a multiple of 16), boxes
+// of box_cols x box_rows, without swizzle or (box_cols = 64) in the 64-byte
+// swizzle.
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_cols, uint32_t box_rows, bool swizzle64) {
+  const TmapKey k{base, rows, cols, box_rows, swizzle64 ? 65u : 1u};
+  TmapEntry& e = tmap_slot(k);
+  if (e.valid && e.key == k) {
+    *m = e.map;
+    return true;
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  if (fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE,
+         swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  e = TmapEntry{k, *m, true};
+  return true;
 }
 
 bool tma_available() { return encode_fn() != nullptr; }

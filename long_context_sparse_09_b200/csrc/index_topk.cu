@@ -615,6 +615,12 @@ csa_status launch_index_scores_tc(const csa_params& p, int B, int Q, const int32
 __global__ void index_plan(const int32_t* q_pos, int G, int ngroups, int m, int N, int* prefix,
                            unsigned* zero_words, size_t nzero);
 
+bool index_fp4_supported(const csa_params& p);
+csa_status launch_index_scores_fp4(const csa_params& p, int B, int Q, const int32_t* q_pos,
+                                   const void* qI, const float* w, const void* kcodes,
+                                   const void* kscales, int N, float* scores, int* plan,
+                                   unsigned* ghist, cudaStream_t st);
+
 static bool use_multi_topk(int R, int N, int k) {
   return R <= 64 && N >= 4096 && k <= kAboveCap && (N + kChunk - 1) / kChunk <= kMaxChunks;
 }
@@ -680,7 +686,7 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
                              const int32_t* q_pos, const void* qI,
                              const float* w, const void* kI, int N,
                              int32_t* idx_out, float* score_out, void* ws,
-                             cudaStream_t st) {
+                             cudaStream_t st, const Mxfp4Keys* fp4) {
   const IdxWsLayout L = idx_ws_layout(p, B, Q, N);
   const int R = B * Q;
   char* base = (char*)ws;
@@ -695,7 +701,14 @@ csa_status launch_index_topk(const csa_params& p, int B, int Q,
     nzero = (L.ccnt - L.ghist) / 4;  // ghist and done
   }
   bool hist_done = false;
-  if (index_tc_supported(p)) {
+  if (fp4 != nullptr) {
+    if (!index_fp4_supported(p)) return CSA_ERR_UNSUPPORTED;
+    if (multi && cudaMemsetAsync(mw.ghist, 0, nzero * 4, st) != cudaSuccess) return CSA_ERR_CUDA;
+    csa_status s = launch_index_scores_fp4(p, B, Q, q_pos, qI, w, fp4->codes, fp4->scales, N,
+                                           scores, plan, multi ? mw.ghist : nullptr, st);
+    if (s != CSA_OK) return s;
+    hist_done = multi && N > 0;
+  } else if (index_tc_supported(p)) {
     csa_status s = launch_index_scores_tc(p, B, Q, q_pos, qI, w, kI, N, scores, plan, mw.ghist,
                                           nzero, multi ? mw.ghist : nullptr, &hist_done, st);
     if (s != CSA_OK) return s;

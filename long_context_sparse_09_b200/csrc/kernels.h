@@ -60,11 +60,20 @@ csa_status launch_decode_append(const csa_params& p, int B, int d, const void* H
                                 int32_t* win_pos0, int W, cudaStream_t st);
 
 size_t index_topk_ws_bytes(const csa_params& p, int B, int Q, int N);
+// indexer keys in MXFP4: E2M1 codes [B*N][c_I/2] and E8M0 scales [B*N][c_I/32]
+struct Mxfp4Keys {
+  const void* codes;
+  const void* scales;
+};
+// scores from bf16 keys (kI), or from MXFP4 keys (fp4 != null, kI unused)
 csa_status launch_index_topk(const csa_params& p, int B, int Q,
                              const int32_t* q_pos, const void* qI,
                              const float* w, const void* kI, int N,
                              int32_t* idx_out, float* score_out, void* ws,
-                             cudaStream_t st);
+                             cudaStream_t st, const Mxfp4Keys* fp4 = nullptr);
+bool index_fp4_supported(const csa_params& p);
+csa_status launch_mxfp4_quantize(long long rows, int width, const void* x, void* codes,
+                                 void* scales, cudaStream_t st);
 
 size_t attend_ws_bytes(const csa_params& p, int B, int Q, int N, bool dense);
 csa_status launch_attend(const csa_params& p, bool dense, int B, int Q,
