@@ -260,6 +260,27 @@ __global__ void __launch_bounds__(256) fold_entries(
                                                   nb, L.b_BIa, L.b_BIb, ch));
 }
 
+// The entries folded by the GEMM's epilogue (F [B*nE][c + cI] fp32, main
+// channels then indexer channels): RMSNorm + RoPE at m*i and the store of
+// the entry; the indexer key rounded to the activation dtype.
+template <typename TA, int kKV>
+__global__ void __launch_bounds__(256) finish_entries(
+    const float* __restrict__ F, int nE, int c, int cI, int m, int rd, float eps,
+    double base, void* __restrict__ ckv, float* __restrict__ ckv_scale, TA* __restrict__ kI) {
+  extern __shared__ float xs[];  // c floats
+  __shared__ float red[32];
+  const size_t e = blockIdx.x;
+  const int i = (int)(e % nE);
+  const float* src = F + e * (size_t)(c + cI);
+  for (int ch = threadIdx.x; ch < c; ch += blockDim.x) xs[ch] = src[ch];
+  __syncthreads();
+  norm_rope_shared(xs, c, rd, eps, (double)m * i, base, red);
+  const size_t rowb = kv_row_bytes(kKV, c, rd);
+  store_kv_row<kKV>(xs, c, rd, (char*)ckv + e * rowb, ckv_scale ? ckv_scale + e : nullptr, red);
+  if (kI != nullptr)
+    for (int ch = threadIdx.x; ch < cI; ch += blockDim.x) kI[e * cI + ch] = from_f32<TA>(src[c + ch]);
+}
+
 template <int kKV>
 __global__ void __launch_bounds__(256) window_rows(const float* __restrict__ P,
                                                   int ncols, int colC, int T, int c,
@@ -281,10 +302,32 @@ __global__ void __launch_bounds__(256) window_rows(const float* __restrict__ P,
 bool gemm_tc_supported(int M, int N, int K);
 csa_status launch_gemm_tc(const void* A, const void* B, float* C, int M, int N, int K,
                           cudaStream_t st);
+bool gemm_fold_supported(const csa_params& p, int d);
+size_t gemm_fold_ws_bytes(const csa_params& p, int B, int T);
+csa_status launch_gemm_fold(const csa_params& p, const PackLayout& L, int B, int T, int d,
+                            const void* H, const void* packed, const float* bias, float* F,
+                            float* Ca, cudaStream_t st);
 
+// bf16 projections whose shapes the fold epilogue covers skip the fp32
+// product: the workspace holds the folded entries and the C^a rows
 size_t compress_ws_bytes(const csa_params& p, int B, int T, int d) {
+  if (gemm_fold_supported(p, d)) return gemm_fold_ws_bytes(p, B, T);
   PackLayout L = pack_layout(p, d);
   return align_up((size_t)B * T * L.ncols * sizeof(float), 256);
+}
+
+template <typename TA, int kKV>
+static void launch_finish(const csa_params& p, const float* F, const float* Ca, int B, int T,
+                          int nE, void* ckv, float* ckv_scale, void* kI, void* win,
+                          float* win_scale, cudaStream_t st) {
+  size_t smem = (size_t)p.c * sizeof(float);
+  if (nE > 0)
+    CSA_LAUNCH(KK_FOLD, st, finish_entries<TA, kKV><<<B * nE, 256, smem, st>>>(
+        F, nE, p.c, p.overlap ? p.c_I : 0, p.m, p.rope_dims, p.rms_eps, (double)p.rope_base,
+        ckv, ckv_scale, (TA*)kI));
+  if (win != nullptr)
+    CSA_LAUNCH(KK_WINDOW, st, window_rows<kKV><<<B * T, 256, smem, st>>>(
+        Ca, p.c, 0, T, p.c, p.rope_dims, p.rms_eps, (double)p.rope_base, win, win_scale));
 }
 
 template <typename TA, int kKV>
@@ -313,6 +356,23 @@ csa_status launch_compress(const csa_params& p, int B, int T, int d,
   const int M = B * T;
   float* P = (float*)ws;
   dim3 grid((L.ncols + 63) / 64, (M + 63) / 64);
+  if (gemm_fold_supported(p, d)) {
+    // the projection with the softmax and fold in its epilogue, then the
+    // norm, RoPE and store of the entries and the window rows
+    const float* bias = (const float*)((const char*)packed + L.bias_off);
+    const int nE = T / p.m;
+    float* F = (float*)ws;
+    float* Ca = (float*)((char*)ws + align_up((size_t)B * nE * (p.c + (p.overlap ? p.c_I : 0)) * 4, 256));
+    csa_status s = launch_gemm_fold(p, L, B, T, d, H, packed, bias, F, Ca, st);
+    if (s != CSA_OK) return s;
+    if (p.kv == CSA_F32)
+      launch_finish<__nv_bfloat16, CSA_F32>(p, F, Ca, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    else if (p.kv == CSA_BF16)
+      launch_finish<__nv_bfloat16, CSA_BF16>(p, F, Ca, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    else
+      launch_finish<__nv_bfloat16, CSA_KV_FP8MIX>(p, F, Ca, B, T, nE, ckv, ckv_scale, kI, win, win_scale, st);
+    return last_launch_status();
+  }
   if (p.act == CSA_BF16 && gemm_tc_supported(M, L.ncols, d)) {
     csa_status s = launch_gemm_tc(H, packed, P, M, L.ncols, d, st);
     if (s != CSA_OK) return s;

@@ -225,6 +225,11 @@ COMP_CASES = [
     ("csa_fp8", "csa", "bf16", "fp8mix", 1, 64, 128, 512, 64, 64, 4),
     ("hca_bf16", "hca", "bf16", "bf16", 2, 100, 128, 128, 32, 0, 16),
     ("hca_f32", "hca", "f32", "f32", 1, 77, 64, 64, 16, 0, 8),
+    # the GEMM with the fold epilogue: overlapping row tiles across two
+    # sequences with ragged ends, m = 8 (15 entries a tile), HCA m' = 128
+    ("csa_fp8_two_seq", "csa", "bf16", "fp8mix", 2, 250, 192, 512, 64, 128, 4),
+    ("csa_m8_bf16", "csa", "bf16", "bf16", 1, 200, 128, 256, 64, 64, 8),
+    ("hca_m128_bf16", "hca", "bf16", "bf16", 2, 300, 128, 256, 64, 0, 128),
 ]
 
 
