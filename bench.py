@@ -45,9 +45,10 @@ L2_BYTES = 126 * 1000 * 1000  # B200 L2 capacity
 # ncu DRAM traffic per launch of the dominant kernel, with the hash of the
 # source file it was measured on (the value is dropped once the file changes).
 NCU_TRAFFIC = {
-    # ncu --set full, pro_csa_decode_1m with 2 sequences (134.29 MB read +
-    # 3.75 MB written), scaled by the units of a full launch (4 sequences)
-    ("index_scores", "pro_csa_decode_1m"): (276.08e6, "9bec71653865"),
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on
+    # pro_csa_decode_1m with 2 sequences (134.30 MB read + 3.48 MB written),
+    # scaled by the units of a full launch (4 sequences)
+    ("index_scores", "pro_csa_decode_1m"): (275.55e6, "c749cc826acd"),
 }
 
 

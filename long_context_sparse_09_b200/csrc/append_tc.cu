@@ -33,10 +33,12 @@ constexpr int kApB = kApN * 64 * 2;         // 2 KB: 16 token rows x 64 k
 constexpr int kApStage = kApA + kApB;       // a multiple of 1024
 constexpr int kApThreads = 192;             // warp 0 TMA, 1 MMA, 2-5 epilogue
 constexpr int kApMaxSplit = 8;              // portable cluster size
+constexpr int kApPrefetch = 16;             // k-blocks a CTA pulls into L2 up front
 constexpr int kApSmem = 1024 + kApStages * kApStage + 128 * kApN * 4 + 256;
 
 struct ApArgs {
   PackLayout L;
+  const uint8_t* dec = nullptr;  // tile-major weight blocks (compressor), or null
   const float* bias;
   const int32_t* tpos;
   float* state;
@@ -52,6 +54,35 @@ struct ApArgs {
   int ld_out, ld_out2, fsplit, out_f32, out2_f32;
   int nfeat, rows_per_group, x_per_group;
 };
+
+// The compressor tile `tile` (64 channels of one part: 0 a main, 1 b main,
+// 2 a indexer, 3 b indexer) -> its first C row and first Z row in the packed
+// [ncols][d] weights, the part, its first channel and its valid channels.
+struct ApTile {
+  int rowA0, rowB0, part, ch0, nvalid;
+};
+__host__ __device__ inline ApTile ap_tile(const PackLayout& L, int c, int cI, int tile) {
+  const int nbc = (c + 63) / 64, nbi = (cI + 63) / 64;
+  ApTile t;
+  int blk;
+  if (tile < nbc) {
+    t.part = 0; blk = tile;
+  } else if (tile < 2 * nbc) {
+    t.part = 1; blk = tile - nbc;
+  } else if (tile < 2 * nbc + nbi) {
+    t.part = 2; blk = tile - 2 * nbc;
+  } else {
+    t.part = 3; blk = tile - 2 * nbc - nbi;
+  }
+  const int colC0 = t.part == 0 ? L.col_Ca : t.part == 1 ? L.col_Cb : t.part == 2 ? L.col_CIa : L.col_CIb;
+  const int colZ0 = t.part == 0 ? L.col_Za : t.part == 1 ? L.col_Zb : t.part == 2 ? L.col_ZIa : L.col_ZIb;
+  const int nchan = t.part < 2 ? c : cI;
+  t.ch0 = blk * 64;
+  t.nvalid = nchan - t.ch0 < 64 ? nchan - t.ch0 : 64;
+  t.rowA0 = colC0 + t.ch0;
+  t.rowB0 = colZ0 + t.ch0;
+  return t;
+}
 
 __device__ __forceinline__ void store_feature(void* base, int f32, size_t i, float v) {
   if (f32)
@@ -85,27 +116,15 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
   bool partb = false;
   const PackLayout& L = a.L;
   if constexpr (kMode == 0) {
-    const int nbc = (a.c + 63) / 64, nbi = (a.cI + 63) / 64;
-    int blk;
-    if (tile < nbc) {
-      part = 0; blk = tile;
-    } else if (tile < 2 * nbc) {
-      part = 1; blk = tile - nbc;
-    } else if (tile < 2 * nbc + nbi) {
-      part = 2; blk = tile - 2 * nbc;
-    } else {
-      part = 3; blk = tile - 2 * nbc - nbi;
-    }
-    const int colC0 = part == 0 ? L.col_Ca : part == 1 ? L.col_Cb : part == 2 ? L.col_CIa : L.col_CIb;
-    const int colZ0 = part == 0 ? L.col_Za : part == 1 ? L.col_Zb : part == 2 ? L.col_ZIa : L.col_ZIb;
+    const ApTile tt = ap_tile(L, a.c, a.cI, tile);
+    part = tt.part;
     colB0 = part == 0 ? L.b_Ba : part == 1 ? L.b_Bb : part == 2 ? L.b_BIa : L.b_BIb;
-    const int nchan = part < 2 ? a.c : a.cI;
     sch0 = part < 2 ? 0 : a.c;  // state channel of the part's channel 0
     partb = part == 1 || part == 3;
-    ch0 = blk * 64;
-    nvalid = nchan - ch0 < 64 ? nchan - ch0 : 64;
-    rowA0 = colC0 + ch0;
-    rowB0 = colZ0 + ch0;
+    ch0 = tt.ch0;
+    nvalid = tt.nvalid;
+    rowA0 = tt.rowA0;
+    rowB0 = tt.rowB0;
   } else {
     const int f0 = tile * 128;
     rowA0 = f0;
@@ -134,12 +153,67 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const int kb0 = split * a.kbs;
+  const int kb1 = kb0 + a.kbs < a.KB ? kb0 + a.kbs : a.KB;
+  if (kMode == 0 && threadIdx.x == 0 && a.dec != nullptr) {
+    // The weights do not come from the previous kernel: the first k-blocks
+    // of this CTA's range are pulled into L2 while it finishes (a prefetch
+    // only fills L2, where later writes would land anyway).  The plain-store
+    // form streams more weights than L2 holds and does not prefetch.
+    const int npre = kb1 - kb0 < kApPrefetch ? kb1 - kb0 : kApPrefetch;
+    for (int i = 0; i < npre; ++i)
+      bulk_prefetch_l2(a.dec + ((size_t)tile * a.KB + kb0 + i) * kApA, kApA);
+  }
   // launched as a programmatic dependent: the set-up above overlaps the
   // previous kernel; h and the state are touched only after this
   pdl_wait();
   const uint32_t tbase = *tbase_sm;
-  const int kb0 = split * a.kbs;
-  const int kb1 = kb0 + a.kbs < a.KB ? kb0 + a.kbs : a.KB;
+
+  // Items of the state update: the (channel, token) pairs of this CTA's
+  // share of the block, handed out from thread 64 on so that the two
+  // issuing lanes take none while there are at most 128.  Each epilogue
+  // thread loads its first item's position, bias and state while the
+  // weights stream.
+  int c_lo = 0, nitems = 0;
+  if (kMode == 0) {
+    const int per = (64 + a.nsplit - 1) / a.nsplit;
+    c_lo = split * per;
+    const int c_hi = c_lo + per < nvalid ? c_lo + per : nvalid;
+    nitems = c_hi > c_lo ? (c_hi - c_lo) * a.nb : 0;
+  }
+  const int me = (threadIdx.x + 128) % kApThreads;
+  const int nch = a.c + a.cI;
+  const int S = a.overlap ? 2 : 1;
+  // state of item `it`: its slot triple, bias and whether it starts the entry
+  struct ApItem {
+    float* slot;  // running max; denominator at + nch, weighted sum at + 2 nch
+    float* src;   // C^a_t of the window row (part a main), else null
+    float mx, den, num, zb;
+    bool fresh;
+  };
+  auto item_state = [&](int it) {
+    ApItem q;
+    const int ch = c_lo + it / a.nb, b = it % a.nb;
+    const int t = a.tpos[b];
+    const int j = t / a.m, rr = t % a.m;
+    float* st = a.state + (size_t)b * a.per_seq;
+    const int gch = ch0 + ch;  // channel within the part
+    q.src = part == 0 ? st + gch : nullptr;
+    const int entry = partb ? j + 1 : j;
+    q.fresh = rr == 0 && (partb || !a.overlap || j == 0);
+    q.slot = st + a.c + (size_t)(entry % S) * 3 * nch + sch0 + gch;
+    q.zb = a.bias[rr * L.nb + colB0 + gch];
+    q.mx = q.den = q.num = 0.f;
+    if (!q.fresh) {
+      q.mx = q.slot[0];
+      q.den = q.slot[nch];
+      q.num = q.slot[2 * nch];
+    }
+    return q;
+  };
+  ApItem pre{};
+  const bool have_pre = kMode == 0 && warp >= 2 && me < nitems;
+  if (have_pre) pre = item_state(me);
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ loads --
@@ -149,8 +223,12 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
       if (!mbar_wait(&empty[s], ((i / kApStages) & 1) ^ 1, abort_sm)) break;
       uint8_t* st = sm + s * kApStage;
       mbar_expect_tx(&full[s], kApStage);
-      tma_load_2d_hint(st, tmW, &full[s], kb * 64, rowA0, pol);
-      tma_load_2d_hint(st + kApA / 2, tmW, &full[s], kb * 64, rowB0, pol);
+      if (kMode == 0 && a.dec != nullptr) {  // one contiguous pre-swizzled block
+        bulk_load_hint(st, a.dec + ((size_t)tile * a.KB + kb) * kApA, kApA, &full[s], pol);
+      } else {
+        tma_load_2d_hint(st, tmW, &full[s], kb * 64, rowA0, pol);
+        tma_load_2d_hint(st + kApA / 2, tmW, &full[s], kb * 64, rowB0, pol);
+      }
       tma_load_2d(st + kApA, tmH, &full[s], xoff + kb * 64, 0);
     }
   } else if (warp == 1 && lane == 0) {
@@ -190,14 +268,8 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
   // --------------------------- sum of the slices and the state update --
   // CTA `split` takes channels [c_lo, c_hi) of the block, all tokens
   if (kMode == 0 && !*abort_sm) {
-    const int per = (64 + a.nsplit - 1) / a.nsplit;
-    const int c_lo = split * per;
-    const int c_hi = c_lo + per < nvalid ? c_lo + per : nvalid;
-    const int nitems = c_hi > c_lo ? (c_hi - c_lo) * a.nb : 0;
-    const int nch = a.c + a.cI;
-    const int S = a.overlap ? 2 : 1;
     const uint32_t dbase = smem_u32(dtile);
-    for (int it = threadIdx.x; it < nitems; it += kApThreads) {
+    for (int it = me; it < nitems; it += kApThreads) {
       const int ch = c_lo + it / a.nb, b = it % a.nb;
       // every slice's pair is loaded first, then summed in slice order
       float cs[kApMaxSplit], zs[kApMaxSplit];
@@ -216,17 +288,13 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
         C += cs[r];
         Z += zs[r];
       }
-      const int t = a.tpos[b];
-      const int j = t / a.m, rr = t % a.m;
-      float* st = a.state + (size_t)b * a.per_seq;
-      const int gch = ch0 + ch;  // channel within the part
-      if (part == 0) st[gch] = C;  // C^a_t: the window row's source
-      const int entry = partb ? j + 1 : j;
-      const bool fresh = rr == 0 && (partb || !a.overlap || j == 0);
-      float* slot = st + a.c + (size_t)(entry % S) * 3 * nch;
-      const int sch = sch0 + gch;
-      running_softmax_add(slot + sch, slot + nch + sch, slot + 2 * nch + sch, C,
-                          Z + a.bias[rr * L.nb + colB0 + gch], fresh);
+      const ApItem q = (it == me && have_pre) ? pre : item_state(it);
+      if (q.src != nullptr) *q.src = C;  // C^a_t: the window row's source
+      float mx = q.mx, den = q.den, num = q.num;
+      running_softmax_step(mx, den, num, C, Z + q.zb, q.fresh);
+      q.slot[0] = mx;
+      q.slot[nch] = den;
+      q.slot[2 * nch] = num;
     }
   }
   // ------------------------------ sum of the slices and the plain store --
@@ -359,6 +427,7 @@ csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, in
   if (!set_kernel_smem((const void*)append_project_tc, kApSmem)) return CSA_ERR_CUDA;
   ApArgs a;
   a.L = L;
+  a.dec = nullptr;  // set below once the tile count is known
   a.bias = bias;
   a.tpos = t;
   a.state = state;
@@ -373,6 +442,8 @@ csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, in
   const int nbc = (p.c + 63) / 64, nbi = (a.cI + 63) / 64;
   const int tiles = p.overlap ? 2 * nbc + 2 * nbi : nbc;
   a.KB = (d + 63) / 64;
+  if (L.dec_tiles == tiles && L.dec_kb == a.KB)
+    a.dec = (const uint8_t*)packed + L.dec_off;
   // (a second CTA on a few SMs would make them the last to finish)
   plan_slices(a, tiles, 0);
   cudaLaunchConfig_t cfg = {};
@@ -391,6 +462,45 @@ csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, in
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
   CSA_LAUNCH(KK_GEMM, st, cudaLaunchKernelEx(&cfg, append_project_tc, tmW, tmH, a));
+  return last_launch_status();
+}
+
+// One 16 KB block per (tile, k-block), block index tile * KB + kb: the
+// tile's 64 C rows, then its 64 Z rows, columns 64 kb .. 64 kb + 63, laid out
+// as the 128-byte swizzle puts them in shared memory (row r's 16-byte chunk j
+// at 128 r + 16 (j ^ r % 8)), so that one bulk copy fills a stage.  Channels
+// past the part's end and columns past d are zero.
+__global__ void __launch_bounds__(256) pack_dec_tiles(const __nv_bfloat16* __restrict__ W,
+                                                      int d, int ncols, PackLayout L, int c,
+                                                      int cI, int KB, uint8_t* __restrict__ dst) {
+  const int tile = blockIdx.x / KB, kb = blockIdx.x % KB;
+  const ApTile tt = ap_tile(L, c, cI, tile);
+  uint8_t* blk = dst + (size_t)blockIdx.x * kDecBlockBytes;
+  const unsigned short* Wb = reinterpret_cast<const unsigned short*>(W);
+  for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
+    const int r = i >> 3, j = i & 7, rr = r & 63;
+    const int row = (r < 64 ? tt.rowA0 : tt.rowB0) + rr;
+    const int k0 = kb * 64 + j * 8;
+    uint32_t v[4] = {0u, 0u, 0u, 0u};
+    if (rr < tt.nvalid && row < ncols) {
+      const unsigned short* src = Wb + (size_t)row * d;
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (k0 + e < d) v[e >> 1] |= (uint32_t)src[k0 + e] << (16 * (e & 1));
+    }
+    *reinterpret_cast<uint4*>(blk + r * 128 + ((j ^ (r & 7)) << 4)) =
+        make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+csa_status launch_pack_dec_tiles(const csa_params& p, const PackLayout& L, int d, void* packed,
+                                 cudaStream_t st) {
+  if (p.act != CSA_BF16 || L.dec_tiles <= 0) return CSA_OK;
+  const int cI = p.overlap ? p.c_I : 0;
+  CSA_LAUNCH(KK_PACK, st,
+             pack_dec_tiles<<<L.dec_tiles * L.dec_kb, 256, 0, st>>>(
+                 (const __nv_bfloat16*)packed, d, L.ncols, L, p.c, cI, L.dec_kb,
+                 (uint8_t*)packed + L.dec_off));
   return last_launch_status();
 }
 

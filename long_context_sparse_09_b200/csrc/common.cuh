@@ -120,17 +120,23 @@ __device__ __forceinline__ void rope_cs(double pos, int p, int rope_dims,
 // Decode compressor: fold one (C, z) pair into an open entry's running
 // softmax (largest logit, denominator, weighted sum of C); `fresh` starts
 // the entry.
-__device__ __forceinline__ void running_softmax_add(float* mx, float* den, float* num, float C,
-                                                    float z, bool fresh) {
+__device__ __forceinline__ void running_softmax_step(float& mx, float& den, float& num, float C,
+                                                     float z, bool fresh) {
   if (fresh) {
-    *mx = z; *den = 1.f; *num = C;
+    mx = z; den = 1.f; num = C;
     return;
   }
-  const float m0 = *mx, m1 = fmaxf(m0, z);
+  const float m0 = mx, m1 = fmaxf(m0, z);
   const float s0 = expf(m0 - m1), s1 = expf(z - m1);
-  *mx = m1;
-  *den = fmaf(*den, s0, s1);
-  *num = fmaf(*num, s0, s1 * C);
+  mx = m1;
+  den = fmaf(den, s0, s1);
+  num = fmaf(num, s0, s1 * C);
+}
+__device__ __forceinline__ void running_softmax_add(float* mx, float* den, float* num, float C,
+                                                    float z, bool fresh) {
+  float m = fresh ? 0.f : *mx, d = fresh ? 0.f : *den, n = fresh ? 0.f : *num;
+  running_softmax_step(m, d, n, C, z, fresh);
+  *mx = m; *den = d; *num = n;
 }
 
 // ------------------------------------------------------------ reductions --

@@ -35,6 +35,12 @@ PackLayout pack_layout(const csa_params& p, int d) {
   }
   L.bias_off = align_up((size_t)L.ncols * d * esize(p.act), 256);
   L.total = L.bias_off + align_up((size_t)p.m * L.nb * 4, 256);
+  if (p.act == CSA_BF16) {  // tile-major copy for the decode projection
+    L.dec_tiles = (c + 63) / 64 + (p.overlap ? (c + 63) / 64 + 2 * ((ci + 63) / 64) : 0);
+    L.dec_kb = (d + 63) / 64;
+    L.dec_off = align_up(L.total, 1024);
+    L.total = L.dec_off + (size_t)L.dec_tiles * L.dec_kb * kDecBlockBytes;
+  }
   return L;
 }
 
@@ -93,6 +99,10 @@ csa_status launch_pack(const csa_params& p, int d, const void* const W[8],
     int n = p.m * bw[t];
     CSA_LAUNCH(KK_PACK, st, pack_bias<<<(n + 255) / 256, 256, 0, st>>>(
                                 Bias[t], p.m, bw[t], bias, L.nb, bcols[t]));
+  }
+  if (L.dec_tiles > 0) {
+    const csa_status s = launch_pack_dec_tiles(p, L, d, packed, st);
+    if (s != CSA_OK) return s;
   }
   return last_launch_status();
 }

@@ -10,7 +10,11 @@
 namespace csa {
 
 // Packed compressor weights: [ncols][d] act dtype (K-major rows, one per GEMM
-// output column), then fp32 biases [m][nb] at bias_off.
+// output column), then fp32 biases [m][nb] at bias_off, then (bf16 only) at
+// dec_off the same weights again as the decode projection streams them: per
+// (tile of 64 channels of one part, k-block of 64) one contiguous 16 KB block
+// of its 64 C rows and 64 Z rows, already in the 128-byte swizzle of shared
+// memory ([dec_tiles][dec_kb][16 KB]).
 struct PackLayout {
   int ncols = 0;
   int col_Ca = -1, col_Cb = -1, col_Za = -1, col_Zb = -1;
@@ -18,6 +22,8 @@ struct PackLayout {
   int nb = 0;
   int b_Ba = -1, b_Bb = -1, b_BIa = -1, b_BIb = -1;
   size_t bias_off = 0;
+  size_t dec_off = 0;
+  int dec_tiles = 0, dec_kb = 0;
   size_t total = 0;
 };
 PackLayout pack_layout(const csa_params& p, int d);
@@ -50,6 +56,9 @@ csa_status launch_query_proj(const csa_params& p, int R, int d, int d_c, const v
                              void* qI, float* w, void* ws, cudaStream_t st);
 // decode append, tensor-core projection (bf16, at most 16 tokens a launch)
 bool append_tc_supported(const csa_params& p, int nb);
+constexpr size_t kDecBlockBytes = 16384;  // one tile-major weight block
+csa_status launch_pack_dec_tiles(const csa_params& p, const PackLayout& L, int d, void* packed,
+                                 cudaStream_t st);
 csa_status launch_append_project_tc(const csa_params& p, const PackLayout& L, int nb, int d,
                                     const void* H, const void* packed, const float* bias,
                                     const int32_t* t, float* state, int cI, size_t per_seq,
