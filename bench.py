@@ -718,7 +718,10 @@ def run_ours(args, world, rank, local):
         wl = wl.with_(T=args.context)
     dev = torch.device(f"cuda:{local}")
     torch.manual_seed(0)
-    step = (DecodeStep if wl.mode == "decode" else PrefillStep)(wl, dev, seed_offset=rank)
+    if wl.mode == "decode":
+        step = DecodeStep(wl, dev, seed_offset=rank, fp4=args.fp4 and wl.variant == "csa")
+    else:
+        step = PrefillStep(wl, dev, seed_offset=rank)
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(dev)
     time.sleep(0.15)
@@ -862,6 +865,7 @@ def run_ours(args, world, rank, local):
                        "entries_per_seq": entries,
                        "m": wl.m, "topk": wl.topk,
                        "n_h": wl.n_h, "c": wl.c, "kv_format": wl.kv, "n_win": wl.n_win,
+                       "indexer_keys": "mxfp4" if getattr(step, "fp4", False) else "bf16",
                        "l2": "inputs larger than L2 (cache streamed every step)"},
             "e2e": {"value": round(units / (e2e_ms / 1e3), 2),
                     "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -979,6 +983,8 @@ def main():
                     help="time the named workload only (no prefill / HCA / Flash sub-objects)")
     ap.add_argument("--batch", type=int, default=0, help="override sequences per GPU (profiling)")
     ap.add_argument("--context", type=int, default=0, help="override context length (profiling)")
+    ap.add_argument("--fp4", action="store_true",
+                    help="decode step with the MXFP4 indexer as the named workload (profiling)")
     args = ap.parse_args()
     if args.impl == "reference":
         # rank 0 alone times the oracle on the host; no process group

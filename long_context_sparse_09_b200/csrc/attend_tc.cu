@@ -433,8 +433,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           // QK(i+1) early only if its tile and S buffer are already there;
           // P V(i) must not wait behind a late tile
           bool qk_next = false;
-          if (i + 1 < ntiles && mbar_try_wait(&kfull[(i + 1) % NS], ((i + 1) / NS) & 1) &&
-              mbar_try_wait(&sfree[(i + 1) & 1], (((i + 1) >> 1) & 1) ^ 1)) {
+          if (i + 1 < ntiles && mbar_test_wait(&kfull[(i + 1) % NS], ((i + 1) / NS) & 1) &&
+              mbar_test_wait(&sfree[(i + 1) & 1], (((i + 1) >> 1) & 1) ^ 1)) {
             if (!issue_qk(i + 1)) break;
             qk_next = true;
           }

@@ -141,6 +141,11 @@ ATTN_CASES = [
     ("csa_fp8_decode", "csa", "bf16", "fp8mix", 2, 1, 1500, 32, 512, 64, 4, 96, 128, "decode"),
     ("csa_f32_prefill", "csa", "f32", "f32", 1, 200, 64, 8, 128, 32, 4, 16, 16, "prefill"),
     ("csa_bf16_prefill_many", "csa", "bf16", "bf16", 1, 700, 300, 16, 512, 64, 4, 32, 128, "prefill"),
+    # many queries, one key slice each (keys on M): several 72-key tiles with
+    # a ragged last one, 64 and 2 x 64 heads, dense HCA rows by TMA boxes
+    ("csa_bf16_prefill_h64_tiles", "csa", "bf16", "bf16", 1, 300, 400, 64, 512, 64, 4, 200, 128, "prefill"),
+    ("csa_bf16_prefill_h128_2seq", "csa", "bf16", "bf16", 2, 100, 300, 128, 512, 64, 4, 96, 128, "prefill"),
+    ("hca_bf16_prefill_many", "hca", "bf16", "bf16", 1, 200, 300, 32, 512, 64, 4, 0, 128, "prefill"),
     # few queries at random positions: key slices of a cluster that hold no keys
     ("csa_bf16_split_ragged", "csa", "bf16", "bf16", 2, 3, 600, 16, 512, 64, 4, 64, 128, "prefill"),
     ("csa_fp8_split_ragged", "csa", "bf16", "fp8mix", 1, 5, 900, 64, 512, 64, 4, 128, 128, "prefill"),
