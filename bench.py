@@ -718,8 +718,9 @@ def run_ours(args, world, rank, local):
         wl = wl.with_(T=args.context)
     dev = torch.device(f"cuda:{local}")
     torch.manual_seed(0)
+    fp4_keys = args.fp4 and wl.mode == "decode" and wl.variant == "csa"
     if wl.mode == "decode":
-        step = DecodeStep(wl, dev, seed_offset=rank, fp4=args.fp4 and wl.variant == "csa")
+        step = DecodeStep(wl, dev, seed_offset=rank, fp4=fp4_keys)
     else:
         step = PrefillStep(wl, dev, seed_offset=rank)
     stream = torch.cuda.current_stream()
@@ -865,7 +866,7 @@ def run_ours(args, world, rank, local):
                        "entries_per_seq": entries,
                        "m": wl.m, "topk": wl.topk,
                        "n_h": wl.n_h, "c": wl.c, "kv_format": wl.kv, "n_win": wl.n_win,
-                       "indexer_keys": "mxfp4" if getattr(step, "fp4", False) else "bf16",
+                       "indexer_keys": "mxfp4" if fp4_keys else "bf16",
                        "l2": "inputs larger than L2 (cache streamed every step)"},
             "e2e": {"value": round(units / (e2e_ms / 1e3), 2),
                     "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

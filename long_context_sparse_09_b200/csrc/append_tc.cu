@@ -250,7 +250,7 @@ __device__ __forceinline__ void skinny_body(const CUtensorMap* tmW, const CUtens
   } else if (warp >= 2) {
     // ------------------------------------------- epilogue: TMEM -> smem --
     const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31
-    if (mbar_wait(tfull, 0, abort_sm)) {
+    if (__all_sync(0xffffffffu, mbar_wait(tfull, 0, abort_sm))) {  // warp-uniform: tcgen05.ld follows
       tc_fence_after();
       float v[16];
       tmem_ld16(tbase + ((uint32_t)(quad * 32) << 16), v);

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint32_t* tbase_sm = (uint32_t*)(pvdone + 2);
   volatile int* abort_sm = (volatile int*)(tbase_sm + 1);
   int& valid_sm = *(int*)(tbase_sm + 2);  // the slice had keys (cluster combine)
+  volatile int* stop_sm = (volatile int*)(tbase_sm + 3);  // a loader's wait gave up
   // slice max (base 2) and sum per head for the cluster combine; written
   // after the last tile, when the per-tile key scales are no longer read
   float2* ml_sm = (float2*)meta_scale;  // [64]
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       mbar_init(&pvdone[i], 1);
     }
     *abort_sm = 0;
+    *stop_sm = 0;
     fence_mbar_init();
   }
   if (warp == 4) {
@@ -217,7 +219,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       int e_next = sel_index(j_begin + t);
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % NS;
-        if (!mbar_wait(&kempty[s], ((i / NS) & 1) ^ 1, abort_sm)) break;
+        // the loop holds named barriers: a wait that gives up raises a flag
+        // that every loader reads after the next barrier, so all 128 leave
+        // at the same point
+        if (!mbar_wait(&kempty[s], ((i / NS) & 1) ^ 1, abort_sm)) *stop_sm = 1;
         const int j0 = j_begin + i * KT;
         const int e_sel = e_next;
         e_next = sel_index(j0 + KT + t);
@@ -256,6 +261,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           (void)inwin;
         }
         named_bar(1, 128);
+        if (*stop_sm) break;
         if (t == 0) {
           // whole tile contiguous in one tensor? (entries: dense; window)
           bool ent = true, wnd = true;
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int wp0 = a.win ? a.win_pos0[b] : 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % NS;
-        if (!mbar_wait(&kempty[s], ((i / NS) & 1) ^ 1, abort_sm)) break;
+        if (!mbar_wait(&kempty[s], ((i / NS) & 1) ^ 1, abort_sm)) *stop_sm = 1;
         float sc_reg = 1.f;
         if (t < KT) {
           const int j = j_begin + i * KT + t;
@@ -359,6 +365,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           if ((t & 31) == 0) reinterpret_cast<unsigned*>(&meta_mask[s])[t >> 5] = bits;
         }
         named_bar(1, 128);
+        if (*stop_sm) break;
         uint8_t* dstK = sK + s * L::KSTAGE;
         // all 18 loads in flight, then widen and store
         uint4 v[18];
@@ -478,7 +485,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       for (int i = 0; i < ntiles; ++i) {
         const int bb = i & 1, s = i % NS;  // S / P buffer, key stage
         const bool mine = half == bb;
-        if (!mbar_wait(&sfull[bb], (i >> 1) & 1, abort_sm)) { ok = false; break; }
+        // (every lane of the warp takes the same exit: the loop holds warp
+        // collectives)
+        if (!__all_sync(0xffffffffu, mbar_wait(&sfull[bb], (i >> 1) & 1, abort_sm))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         float sv[KT];
 #pragma unroll
@@ -532,7 +544,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         resc = __shfl_sync(0xffffffffu, resc, src);
         if (__any_sync(0xffffffffu, resc)) {
           // O must not be in flight: wait for the previous tile's P V
-          if (!mbar_wait(&pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_sm)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(&pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_sm))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t orow = trow + ((uint32_t)(16 * half) << 16);
           for (int c0 = 0; c0 < 256; c0 += 16) {
@@ -557,7 +572,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         l = l * alpha + lsum;
         l = __shfl_sync(0xffffffffu, l, src);
         // P buffer bb was read by the P V of tile i-2
-        if (i >= 2 && !mbar_wait(&pvdone[bb], ((i - 2) >> 1) & 1, abort_sm)) { ok = false; break; }
+        if (i >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(&pvdone[bb], ((i - 2) >> 1) & 1, abort_sm))) {
+          ok = false;
+          break;
+        }
         if (mine) {
           uint8_t* prow = sP + bb * L::NP * kPBytes + hl * 128;
 #pragma unroll

@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     int an = 0;
     for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++an) {
       const int acc = an & 1;
-      if (!mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm)) break;
+      // (the warp leaves together: the loop holds warp collectives)
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm))) break;
       tc_fence_after();
       const int m0 = (tile / a.tiles_n) * kGm, n0 = (tile % a.tiles_n) * kGn;
       const int row = m0 + quad * 32 + lane;
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     bool dead = false;
     for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++an) {
       const int acc = an & 1;
-      if (!dead && !mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm)) dead = true;
+      if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (an >> 1) & 1, abort_sm));
       tc_fence_after();
       const int mt = tile / a.nt, n = tile % a.nt;
       const int b = mt / a.mt_per_seq, j = mt % a.mt_per_seq;

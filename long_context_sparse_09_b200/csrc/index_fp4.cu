@@ -289,7 +289,9 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           // the query of this group: q^I rounded to MXFP4 per head and block
           // of 32, as exact f16 values in the 128-byte swizzled K-major slot
           const int slot = qn & 1;
-          if (!mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_sm)) break;
+          // (the warp leaves together: the loop holds warp collectives)
+          if (!__all_sync(0xffffffffu, mbar_wait(&qempty[slot], ((qn >> 1) & 1) ^ 1, abort_sm)))
+            break;
           uint8_t* qs = qsl + slot * kF4QSlot;
           const int r = cur.g;
           for (int it = dt; it < nhI * kF4Blocks; it += 128) {
@@ -345,9 +347,10 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           ++qn;
         }
         const int s = i % kF4SC;
-        if (!mbar_wait(&cfull[s], (i / kF4SC) & 1, abort_sm)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&cfull[s], (i / kF4SC) & 1, abort_sm))) break;
         const int sa = i % kF4SA;
-        if (!mbar_wait(&aempty[sa], ((i / kF4SA) & 1) ^ 1, abort_sm)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&aempty[sa], ((i / kF4SA) & 1) ^ 1, abort_sm)))
+          break;
         tc_fence_after();
         const uint8_t* crow = cst + s * kF4CodeTile + row * kF4CodeBytes;
         const uint32_t sw = *reinterpret_cast<const uint32_t*>(sst + s * kF4ScaleTile + row * 4);
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         const bool first = cur.first(i), last = cur.last(prefix);
         const int slot = qn & 1;
         if (first) {
-          if (!dead && !mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_sm)) dead = true;
+          if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&qfull[slot], (qn >> 1) & 1, abort_sm));
           nv = n_visible(__ldg(a.q_pos + cur.g), a.m, a.N);
         }
         if (hist && cur.g != hist_r) {  // query changed: flush its histogram
@@ -423,8 +426,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           named_bar(2, 256);
           hist_r = cur.g;
         }
-        if ((i & 1) == alt && !dead && !mbar_wait(&tfull[i % kF4Acc], (i / kF4Acc) & 1, abort_sm))
-          dead = true;
+        if ((i & 1) == alt && !dead)
+          dead = !__all_sync(0xffffffffu, mbar_wait(&tfull[i % kF4Acc], (i / kF4Acc) & 1, abort_sm));
         if ((i & 1) == alt && !dead) {
           const int acc = i % kF4Acc;
           tc_fence_after();

@@ -258,6 +258,9 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
       TileCursor cur;
       cur.init(prefix, a.ngroups, start, count);
       int an = 0, hist_r = cur.g;
+      // after a wait gives up the warp keeps walking the list without work,
+      // so that every epilogue warp takes the same named barriers
+      bool dead = false;
       float wreg[G == 1 ? 64 : 1];
       int w_r = -1;
       constexpr int NQM = (NE == 4 || kAlt) ? G : G / 2;  // queries of this warp
@@ -293,7 +296,12 @@ __global__ void __launch_bounds__(IdxTcCfg<G, KB, S, NE, NQ>::kThreads, 1)
           continue;
         }
         const int acc = an % nacc;
-        if (!mbar_wait(&tfull[acc], (an / nacc) & 1, abort_sm)) break;
+        if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (an / nacc) & 1, abort_sm));
+        if (dead) {
+          ++an;
+          cur.next(prefix, a.ngroups);
+          continue;
+        }
         tc_fence_after();
         const int s = cur.t * kTileM + quad * 32 + lane;
         float sc[G];
