@@ -269,6 +269,17 @@ __global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
   const int c = a.c;
   const int S = a.nsplit;
   const float zs = a.sink[head];
+  // R_{-t0} of this thread's first four dims, started before the partials
+  // arrive (c = 4 blockDim.x covers every dim in one pass)
+  const int t0 = a.q_pos[r];
+  const int e_first = 4 * threadIdx.x;
+  float rc0 = 1.f, rs0 = 0.f, rc1 = 1.f, rs1 = 0.f;
+  const bool rope_now = e_first < c && e_first >= c - a.rd;
+  if (rope_now) {
+    const int p0 = (e_first - (c - a.rd)) >> 1;
+    rope_cs(-(double)t0, p0, a.rd, a.base, &rc0, &rs0);
+    rope_cs(-(double)t0, p0 + 1, a.rd, a.base, &rc1, &rs1);
+  }
   // split maxima and sums (S <= 256)
   float mloc = -INFINITY;
   for (int s = threadIdx.x; s < S; s += blockDim.x)
@@ -286,7 +297,6 @@ __global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
   if (threadIdx.x == 0) s_den = dsum + expf(zs - M);
   __syncthreads();
   const float inv = 1.0f / s_den;
-  const int t0 = a.q_pos[r];
   T* dst = reinterpret_cast<T*>(a.out) + ((size_t)r * a.n_h + head) * c;
   const size_t stride = R * a.n_h * (size_t)c / 4;  // float4 stride between splits
   for (int e = 4 * threadIdx.x; e < c; e += 4 * blockDim.x) {
@@ -311,7 +321,16 @@ __global__ void __launch_bounds__(128) attend_combine(AttnArgs a) {
       acc.z = fmaf(f, v.z, acc.z); acc.w = fmaf(f, v.w, acc.w);
     }
     acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-    derotate4(acc, e, c, a.rd, t0, a.base);
+    if (e == e_first && rope_now) {  // the factors computed at the start
+      float x0 = acc.x, x1 = acc.y;
+      acc.x = x0 * rc0 - x1 * rs0;
+      acc.y = x0 * rs0 + x1 * rc0;
+      x0 = acc.z; x1 = acc.w;
+      acc.z = x0 * rc1 - x1 * rs1;
+      acc.w = x0 * rs1 + x1 * rc1;
+    } else {
+      derotate4(acc, e, c, a.rd, t0, a.base);
+    }
     store4<T>(dst + e, acc);
   }
 }
