@@ -46,9 +46,14 @@ L2_BYTES = 126 * 1000 * 1000  # B200 L2 capacity
 # source file it was measured on (the value is dropped once the file changes).
 NCU_TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on
-    # pro_csa_decode_1m with 2 sequences (134.30 MB read + 3.48 MB written),
+    # pro_csa_decode_1m with 2 sequences (134.30 MB read + 3.38 MB written),
     # scaled by the units of a full launch (4 sequences)
-    ("index_scores", "pro_csa_decode_1m"): (275.55e6, "c749cc826acd"),
+    ("index_scores", "pro_csa_decode_1m"): (275.37e6, "266b1e616614"),
+    # ncu --set full on flash_csa_prefill_32k cut to 8,192 tokens (565.12 MB
+    # read + 484.08 MB written: the queries read and the outputs written once;
+    # the gathered rows come from L2), scaled by the queries of a full launch
+    # (32,768: traffic grows in proportion)
+    ("attend", "flash_csa_prefill_32k"): (4196.78e6, "b8cd68c0a9a9"),
 }
 
 
