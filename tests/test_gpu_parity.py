@@ -146,6 +146,10 @@ ATTN_CASES = [
     ("csa_bf16_prefill_h64_tiles", "csa", "bf16", "bf16", 1, 300, 400, 64, 512, 64, 4, 200, 128, "prefill"),
     ("csa_bf16_prefill_h128_2seq", "csa", "bf16", "bf16", 2, 100, 300, 128, 512, 64, 4, 96, 128, "prefill"),
     ("hca_bf16_prefill_many", "hca", "bf16", "bf16", 1, 200, 300, 32, 512, 64, 4, 0, 128, "prefill"),
+    # no window: queries before the first complete entry have no key at all
+    # (all weight on the sink), interleaved with the others in each CTA's
+    # walk over more queries than SMs
+    ("hca_bf16_prefill_nowin", "hca", "bf16", "bf16", 1, 400, 24, 16, 512, 64, 4, 0, 0, "prefill"),
     # few queries at random positions: key slices of a cluster that hold no keys
     ("csa_bf16_split_ragged", "csa", "bf16", "bf16", 2, 3, 600, 16, 512, 64, 4, 64, 128, "prefill"),
     ("csa_fp8_split_ragged", "csa", "bf16", "fp8mix", 1, 5, 900, 64, 512, 64, 4, 128, 128, "prefill"),
