@@ -706,3 +706,52 @@ def test_fp4_index_scores_on_representable_inputs():
     np.testing.assert_array_equal(s4[fin], oracle.round_bf16(ref[fin]))
     idx, _ = oracle.topk(s4, np.array([oracle.nvis(int(t), wl.m, N) for t in t0s]), 8)
     assert P.topk_recall(idx, idx).tolist() == [1.0, 1.0]
+
+
+# ------------------------------------------------- cache size per token ---
+# The compressed cache per token and layer that "02 · DeepSeek-V4: 压缩注意力
+# 撑起 1M 上下文" section 2.5 works out for V4-Pro (tests/golden/
+# kv_elements_per_token.txt).
+
+def _golden_kv_elements():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "kv_elements_per_token.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    return {r[0]: int(r[1]) for r in rows}
+
+
+def _compress_weights(wl, d, r):
+    W = {}
+    for k, width in (("Wkv_a", wl.c), ("Wz_a", wl.c), ("Wkv_b", wl.c), ("Wz_b", wl.c),
+                     ("WIkv_a", wl.c_I), ("WIz_a", wl.c_I), ("WIkv_b", wl.c_I),
+                     ("WIz_b", wl.c_I)):
+        if width:
+            W[k] = r.normal(0, d ** -0.5, (d, width))
+    for k, width in (("B_a", wl.c), ("B_b", wl.c), ("BI_a", wl.c_I), ("BI_b", wl.c_I)):
+        if width:
+            W[k] = r.normal(0, 0.3, (wl.m, width))
+    return W
+
+
+def test_cache_elements_per_token_match_the_worked_example():
+    """The oracle's whole-sequence compressor stores c/m + c_I/m elements per
+    token for a CSA layer and c/m' for an HCA layer: the page's 160 and 4 at
+    the V4-Pro widths, and about 4,900 over its 30 CSA and 31 HCA layers."""
+    gold = _golden_kv_elements()
+    r = rng(11)
+    d, T = 16, 256
+    pro = WORKLOADS["pro_csa_decode_1m"]
+    hca = WORKLOADS["hca_decode_1m"].with_(c=pro.c)
+    assert (pro.c, pro.c_I, pro.m, hca.m) == (512, 128, 4, 128)
+    kv, kI, win = P.compress_seq(pro, _compress_weights(pro, d, r), r.normal(0, 1, (T, d)))
+    assert kv.shape == (T // pro.m, pro.c) and kI.shape == (T // pro.m, pro.c_I)
+    assert win.shape == (T, pro.c)  # the window side output, one row per token
+    csa = (kv.size + kI.size) / T
+    kv_h, kI_h, _ = P.compress_seq(hca, _compress_weights(hca, d, r), r.normal(0, 1, (T, d)))
+    assert kI_h is None and kv_h.shape == (T // hca.m, hca.c)
+    hca_el = kv_h.size / T
+    assert csa == gold["csa_layer_elements_per_token"]
+    assert hca_el == gold["hca_layer_elements_per_token"]
+    total = gold["pro_csa_layers"] * csa + gold["pro_hca_layers"] * hca_el
+    assert abs(total - gold["pro_elements_per_token_about"]) <= 0.01 * gold[
+        "pro_elements_per_token_about"]
