@@ -145,6 +145,8 @@ ATTN_CASES = [
     # a ragged last one, 64 and 2 x 64 heads, dense HCA rows by TMA boxes
     ("csa_bf16_prefill_h64_tiles", "csa", "bf16", "bf16", 1, 300, 400, 64, 512, 64, 4, 200, 128, "prefill"),
     ("csa_bf16_prefill_h128_2seq", "csa", "bf16", "bf16", 2, 100, 300, 128, 512, 64, 4, 96, 128, "prefill"),
+    # FP8-mixed rows (64-key tiles) over more single-slice queries than SMs
+    ("csa_fp8_prefill_many", "csa", "bf16", "fp8mix", 1, 300, 400, 64, 512, 64, 4, 96, 128, "prefill"),
     ("hca_bf16_prefill_many", "hca", "bf16", "bf16", 1, 200, 300, 32, 512, 64, 4, 0, 128, "prefill"),
     # no window: queries before the first complete entry have no key at all
     # (all weight on the sink), interleaved with the others in each CTA's
